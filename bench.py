@@ -1,0 +1,457 @@
+"""Benchmark of the packed-KV hot path: one step = one full block-by-block decode.
+
+A step appends every block of K/V of every layer into the packed cache
+(quantize + bit-pack) and runs each block's packed-KV attention, in decode
+order (block-major: for s in blocks, for l in layers). Inputs are seeded
+synthetic K/V/Q shaped like the workload, resident in HBM before timing.
+
+Prints ONE JSON line on rank 0. `value` = query tokens x layers decoded per
+second (B * N * L per step) over the whole step, max over ranks; per-kernel
+numbers (quantize+pack GB/s, attention tokens/s, roofline fractions) are in
+the `quant_pack` / `attention` / `roofline` keys.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload var_d30] [--bits 3]
+  python bench.py --impl reference ...   # the CPU oracle, bounded sample
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, default_softmax_scale, make_kv, make_q  # noqa: E402
+
+METRIC = "KV quant+pack GB/s; packed-KV attention tokens/s; % of HBM/tensor roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------------ algorithmic work
+def word_rows(n, bits):
+    c = 32 // bits
+    return (n + c - 1) // c
+
+
+def quant_bytes(w, bits, s):
+    """Algorithmic HBM bytes of one append (K and V) of block s of one layer."""
+    esize = 4 if w.kv_dtype == "f32" else 2
+    B, H, D, n = w.batch, w.heads, w.head_dim, w.block_tokens[s]
+    per = esize * B * H * n * D + 4 * B * H * word_rows(n, bits) * D + 8 * B * H * D
+    return 2 * per
+
+
+def attn_work(w, bits, s):
+    """(flops, bytes) of the attention of block s of one layer (fp32 output)."""
+    B, H, D, n = w.batch, w.heads, w.head_dim, w.block_tokens[s]
+    P = w.prefix(s) + n
+    flops = 4 * B * H * n * P * D
+    words = sum(word_rows(w.block_tokens[k], bits) for k in range(s + 1))
+    byts = 2 * B * H * n * D + 4 * B * H * n * D + 8 * B * H * D * words + 16 * B * H * D * (s + 1)
+    return flops, byts
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    if world != n_gpus and rank == 0:
+        print(f"warning: --gpus {n_gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def oracle_unit(w, bits, layer_kv, q, b, h, sigma):
+    """One (b, h) unit of one layer through the oracle: append every block of
+    K and V, then every block's attention. Returns seconds."""
+    import numpy as np
+
+    import oracle.vq_oracle as vo
+    k, v = layer_kv
+    t0 = time.perf_counter()
+    kh = k[b:b + 1, h:h + 1].float().numpy()
+    vh = v[b:b + 1, h:h + 1].float().numpy()
+    qh = q[b:b + 1, h:h + 1].float().numpy()
+    pk, sk, zk = vo.cache_append(kh, w.block_tokens, bits)
+    pv, sv, zv = vo.cache_append(vh, w.block_tokens, bits)
+    for s, n in enumerate(w.block_tokens):
+        khat = vo.dequantize_cache(pk, sk, zk, w.block_tokens, 1, 1, w.head_dim, bits, s)
+        vhat = vo.dequantize_cache(pv, sv, zv, w.block_tokens, 1, 1, w.head_dim, bits, s)
+        p0 = w.prefix(s)
+        out = vo.attention_f64(qh[:, :, p0:p0 + n], khat, vhat, sigma)
+        assert np.isfinite(out).all()
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_sample(w, bits, budget_s=15.0, max_units=64):
+    """Time the oracle on (b, h) units of layer 0 until ~budget_s; return
+    (tokens_per_s scaled to the whole step, units, seconds)."""
+    k, v = _small_kv(w)
+    q = _small_q(w)
+    sigma = default_softmax_scale(w)
+    total, units = 0.0, 0
+    while units < max_units and (total < budget_s or units == 0):
+        b = units % k.shape[0]
+        h = (units // k.shape[0]) % w.heads
+        total += oracle_unit(w, bits, (k, v), q, b, h, sigma)
+        units += 1
+    per_unit = total / units
+    # one step = B*H*L units; value = B*N*L tokens per step time
+    tokens_per_s = w.batch * w.tokens * w.layers / (per_unit * w.batch * w.heads * w.layers)
+    return tokens_per_s, units, total
+
+
+def _small_kv(w):
+    """Layer-0 K/V of a batch of at most two (same distribution) for the CPU sample."""
+    import dataclasses
+    return make_kv(dataclasses.replace(w, batch=min(2, w.batch)), 0, device="cpu")
+
+
+def _small_q(w):
+    import dataclasses
+    return make_q(dataclasses.replace(w, batch=min(2, w.batch)), 0, device="cpu")
+
+
+# ------------------------------------------------------------------ the reference arm (oracle)
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    bits = args.bits or w.bits[0]
+    import dataclasses
+    wk = dataclasses.replace(w, batch=min(w.batch, 2))
+    k, v = make_kv(wk, 0, device="cpu")
+    q = make_q(wk, 0, device="cpu")
+    sigma = default_softmax_scale(w)
+    times = []
+    u = 0
+    for i in range(args.warmup + args.steps):
+        dt = 0.0
+        for _ in range(args.ref_units):
+            b, h = u % wk.batch, (u // wk.batch) % w.heads
+            dt += oracle_unit(w, bits, (k, v), q, b, h, sigma)
+            u += 1
+        if i >= args.warmup:
+            times.append(dt)
+    per_unit = sum(times) / len(times) / args.ref_units
+    value = w.tokens / (per_unit * w.heads)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_unit * args.ref_units * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "bits": bits, "layers": w.layers, "heads": w.heads, "head_dim": w.head_dim,
+                   "batch": w.batch, "blocks": w.num_blocks, "tokens": w.tokens},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: {args.ref_units} (batch, head) units of layer 0 through the oracle (append of all "
+                                   "blocks of K and V + every block's float64 attention), scaled by B*H*L units"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    from bit_kv_cache_25_b200 import vq
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = WORKLOADS[args.workload]
+    bits = args.bits or w.bits[0]
+    L, S, B, H, D, N = w.layers, w.num_blocks, w.batch, w.heads, w.head_dim, w.tokens
+    sigma = default_softmax_scale(w)
+    seed = 1000003 * rank
+
+    desc = vq.CacheDesc(B, H, D, bits, w.block_tokens)
+    ks, vs, qs, caches = [], [], [], []
+    for layer in range(L):
+        k, v = make_kv(w, layer, seed=seed, device=dev)
+        ks.append(k)
+        vs.append(v)
+        qs.append(make_q(w, layer, seed=seed, device=dev))
+        caches.append(vq.LayerCache(desc, device=dev))
+    nmax = max(w.block_tokens)
+    out = torch.empty((B, H, nmax, D), dtype=torch.float32, device=dev)
+    outs = [out[:, :, :n] for n in w.block_tokens]
+    stream = torch.cuda.current_stream()
+
+    # events around every launch of every timed step, to split the step into kernels
+    n_launch = 2 * L * S
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(args.steps)]
+
+    def step(ev):
+        i = 0
+        if ev is not None:
+            ev[0].record(stream)
+        for s in range(S):
+            p0, n = w.prefix(s), w.block_tokens[s]
+            for layer in range(L):
+                vq.vq_cache_append(desc, caches[layer], s, ks[layer][:, :, p0:p0 + n], vs[layer][:, :, p0:p0 + n],
+                                   stream=stream)
+                if ev is not None:
+                    ev[i + 1].record(stream)
+                i += 1
+                vq.vq_attention_block(desc, caches[layer], s, qs[layer][:, :, p0:p0 + n], sigma, outs[s],
+                                      stream=stream)
+                if ev is not None:
+                    ev[i + 1].record(stream)
+                i += 1
+
+    for _ in range(args.warmup):
+        step(None)
+    torch.cuda.synchronize()
+    assert vq.vq_poll_device_error() == 0
+
+    q_bytes = sum(quant_bytes(w, bits, s) for s in range(S)) * L
+    a_flops = sum(attn_work(w, bits, s)[0] for s in range(S)) * L
+    a_bytes = sum(attn_work(w, bits, s)[1] for s in range(S)) * L
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    t_quant = t_attn = 0.0
+    for ev in evs:
+        for j in range(n_launch):
+            dt = ev[j].elapsed_time(ev[j + 1])
+            if j % 2 == 0:
+                t_quant += dt
+            else:
+                t_attn += dt
+    barrier(world)
+    elapsed_ms = start.elapsed_time(stop)
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    assert vq.vq_poll_device_error() == 0
+    clocks = clk.summary()
+
+    ms_step = elapsed_ms / args.steps
+    tokens_step = B * N * L
+    value = world * tokens_step / (ms_step / 1e3)
+    peaks, peak_src = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tc = peaks["bf16_tflops_sustained"]
+    q_ms = t_quant / args.steps
+    a_ms = t_attn / args.steps
+    q_gbs = q_bytes / (q_ms / 1e3) / 1e9
+    a_gbs = a_bytes / (a_ms / 1e3) / 1e9
+    a_tflops = a_flops / (a_ms / 1e3) / 1e12
+    a_bound = "hbm" if a_bytes / (hbm * 1e9) >= a_flops / (tc * 1e12) else "tensor"
+    a_frac = (a_gbs / hbm) if a_bound == "hbm" else (a_tflops / tc)
+    if a_ms >= q_ms:
+        roof = {"kernel": "attention", "bound": a_bound, "achieved": a_gbs if a_bound == "hbm" else a_tflops,
+                "peak": hbm if a_bound == "hbm" else tc, "unit": "GB/s" if a_bound == "hbm" else "TFLOP/s",
+                "frac": a_frac, "traffic": None}
+    else:
+        roof = {"kernel": "quant_pack", "bound": "hbm", "achieved": q_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": q_gbs / hbm, "traffic": None}
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "bits": bits, "layers": L, "heads": H, "head_dim": D, "batch": B,
+                   "blocks": S, "tokens": N, "kv_dtype": w.kv_dtype, "per_rank": "one full decode per step",
+                   "l2": f"inputs {sum(t.numel() * t.element_size() for t in ks + vs + qs) / 1e9:.1f} GB > L2, no flush",
+                   "token_unit": "B*N*L query tokens x layers per step (append + attention)"},
+        "quant_pack": {"ms_per_step": q_ms, "gbs": q_gbs, "frac_hbm": q_gbs / hbm,
+                       "bytes_per_step": q_bytes},
+        "attention": {"ms_per_step": a_ms, "tokens_per_s": tokens_step / (a_ms / 1e3), "gbs": a_gbs,
+                      "tflops": a_tflops, "bound": a_bound, "frac_roofline": a_frac,
+                      "flops_per_step": a_flops, "bytes_per_step": a_bytes},
+        "roofline": roof,
+        "clocks": clocks,
+        "gpu_launches": n_launch * args.steps,
+    }
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, vq, w, bits, desc, caches, outs, dev, world)
+    if rank == 0 and not args.no_cpu:
+        tps, units, secs = cpu_sample(w, bits, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{units} (batch, head) units of layer 0 through the oracle (append of all "
+                                          f"blocks + float64 attention of every block), {secs:.1f} s, scaled by "
+                                          f"B*H*L units per step"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, vq, w, bits, desc, caches, outs, dev, world):
+    """Same decode through the public API with host inputs: every step copies each
+    layer's K, V, Q from pinned host memory, runs its appends and attentions, and
+    copies its outputs back. The host holds one layer of inputs, reused for
+    every layer; the device holds one layer of inputs at a time."""
+    L, S = w.layers, w.num_blocks
+    k0, v0 = make_kv(w, 0, seed=7, device="cpu")
+    q0 = make_q(w, 0, seed=7, device="cpu")
+    hk, hv, hq = k0.pin_memory(), v0.pin_memory(), q0.pin_memory()
+    dk, dv, dq = torch.empty_like(hk, device=dev), torch.empty_like(hv, device=dev), torch.empty_like(hq, device=dev)
+    B, H, D, N = w.batch, w.heads, w.head_dim, w.tokens
+    dout = torch.empty((B, H, N, D), dtype=torch.float32, device=dev)
+    hout = torch.empty((B, H, N, D), dtype=torch.float32).pin_memory()
+    sigma = default_softmax_scale(w)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for layer in range(L):
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dq.copy_(hq, non_blocking=True)
+            for s in range(S):
+                p0, n = w.prefix(s), w.block_tokens[s]
+                vq.vq_cache_append(desc, caches[layer], s, dk[:, :, p0:p0 + n], dv[:, :, p0:p0 + n], stream=stream)
+                vq.vq_attention_block(desc, caches[layer], s, dq[:, :, p0:p0 + n], sigma, dout[:, :, p0:p0 + n],
+                                      stream=stream)
+            hout.copy_(dout, non_blocking=True)
+
+    steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(1):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world)
+    h2d = L * sum(t.numel() * t.element_size() for t in (hk, hv, hq))
+    d2h = L * hout.numel() * hout.element_size()
+    return {"value": world * B * N * L / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="var_d30", choices=sorted(WORKLOADS))
+    ap.add_argument("--bits", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-units", type=int, default=8)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,79 @@
+// Internal (C++) interface between the C-ABI entry points and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace vq {
+
+// One tensor of a quantize+pack launch: the block's input slab and where the
+// packed words and per-group scale/zero of that block go.
+struct QuantTensor {
+  const void* x;        // element (b,h,t,c) at x[b*sb + h*sh + t*st + c]
+  int64_t sb, sh, st;   // strides in elements
+  uint32_t* packed;     // [B][H][W][D]
+  float* scale;         // [B][H][D]
+  float* zero;          // [B][H][D]
+};
+
+struct QuantParams {
+  QuantTensor t[2];     // K then V (or a single tensor)
+  int B, H, D;
+  int n;                // tokens in the block
+  int W;                // word-rows of the block
+  int bits;
+  int esize;            // 2 (bf16) or 4 (fp32)
+  int vecs_per_row;     // D * esize / 16
+  int units;            // tensors * B * H
+  int G;                // units per CTA (C == 1)
+  int C;                // CTAs per unit (cluster size); G == 1 when C > 1
+  int wr_chunk;         // word-rows per CTA
+  int rows_chunk;       // staged token rows per unit per CTA (n when C == 1)
+};
+
+size_t quant_smem_bytes(int G, int D, int rows_chunk, int rowbytes);
+int quant_threads();
+cudaError_t launch_quant_pack(const QuantParams& p, cudaStream_t stream);
+
+struct DequantParams {
+  const uint32_t* packed;  // [B][H][W][D]
+  const float* scale;      // [B][H][D]
+  const float* zero;
+  float* out;              // [B][H][n][D]
+  int B, H, D, n, W, bits;
+};
+cudaError_t launch_dequant(const DequantParams& p, cudaStream_t stream);
+
+// Attention of one block's queries over the packed cache of blocks 0..s.
+struct AttnBlockInfo {
+  int64_t word_off;  // word offset of block k's packed region (per tensor)
+  int n;             // tokens of block k
+  int W;             // word-rows of block k
+};
+
+constexpr int kMaxBlocks = 64;
+constexpr int kMaxDevices = 64;  // per-process device ordinals with cached function attributes
+
+struct AttnParams {
+  const uint32_t* packed_k;
+  const uint32_t* packed_v;
+  const float* scale_k;
+  const float* zero_k;
+  const float* scale_v;
+  const float* zero_v;
+  const uint16_t* q;           // bf16
+  int64_t q_sb, q_sh, q_st;
+  void* out;
+  int64_t o_sb, o_sh, o_st;
+  int out_f32;                 // 1: float32 output, 0: bf16
+  int B, H, D, bits;
+  int s;                       // current block
+  int n_q;                     // queries (tokens of block s)
+  float softmax_scale;
+  AttnBlockInfo blk[kMaxBlocks];
+};
+cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream);
+
+}  // namespace vq

@@ -1,0 +1,294 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Codes, packed words, scales and zeros must be bit-exact. Attention outputs must
+be within max-abs 2e-3 x RMS(reference) of the float64 oracle run on the
+oracle's own dequantized cache. Inputs come from the seeded workload generator
+(drawn on the GPU, copied to the host for the oracle).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.vq_oracle as vo
+from workloads import WORKLOADS, Workload, default_softmax_scale, make_kv, make_q
+
+pytestmark = pytest.mark.gpu
+
+ATTN_TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def vq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_kv_cache_25_b200 import vq as _vq
+    return _vq
+
+
+def _host(t):
+    return t.float().cpu().numpy()
+
+
+def _append_all(vq, w: Workload, bits, k, v):
+    desc = vq.CacheDesc(w.batch, w.heads, w.head_dim, bits, w.block_tokens)
+    cache = vq.LayerCache(desc)
+    for s, n in enumerate(w.block_tokens):
+        p0 = w.prefix(s)
+        vq.vq_cache_append(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+    torch.cuda.synchronize()
+    assert vq.vq_poll_device_error() == 0
+    return desc, cache
+
+
+def _check_cache_bit_exact(vq, w, bits, desc, cache, k, v, bsel):
+    B, H, D = w.batch, w.heads, w.head_dim
+    offs = cache.block_word_offset
+    for name, x, packed, scale, zero in (("k", k, cache.packed_k, cache.scale_k, cache.zero_k),
+                                         ("v", v, cache.packed_v, cache.scale_v, cache.zero_v)):
+        xh = _host(x[bsel])
+        pk = packed.cpu().numpy().view(np.uint32)
+        sc = scale.cpu().numpy()
+        zr = zero.cpu().numpy()
+        for s, n in enumerate(w.block_tokens):
+            p0 = w.prefix(s)
+            W = desc.word_rows(s)
+            words, s_ref, z_ref = vo.quantize_pack_block(xh[:, :, p0:p0 + n], bits)
+            got_w = pk[offs[s]:offs[s + 1]].reshape(B, H, W, D)[bsel]
+            got_s = sc[s * B * H * D:(s + 1) * B * H * D].reshape(B, H, D)[bsel]
+            got_z = zr[s * B * H * D:(s + 1) * B * H * D].reshape(B, H, D)[bsel]
+            np.testing.assert_array_equal(got_s.view(np.uint32), s_ref.view(np.uint32), err_msg=f"{name} scale s={s}")
+            np.testing.assert_array_equal(got_z.view(np.uint32), z_ref.view(np.uint32), err_msg=f"{name} zero s={s}")
+            if not np.array_equal(got_w, words):
+                bad = np.argwhere(got_w != words)
+                raise AssertionError(f"{name} packed words differ at block {s}: {len(bad)} words, first {bad[:3]}")
+
+
+def _oracle_cache(w, bits, x_host):
+    """Oracle's own cache of the selected batch rows: (packed, scale, zero)."""
+    return vo.cache_append(x_host, w.block_tokens, bits)
+
+
+def _check_attention(vq, w, bits, desc, cache, q, k, v, bsel, rows_for_block):
+    sigma = default_softmax_scale(w)
+    B, H, D = w.batch, w.heads, w.head_dim
+    kh_host, vh_host = _host(k[bsel]), _host(v[bsel])
+    ok_, sk, zk = _oracle_cache(w, bits, kh_host)
+    ov_, sv, zv = _oracle_cache(w, bits, vh_host)
+    nb = len(bsel)
+    worst = 0.0
+    for s, n in enumerate(w.block_tokens):
+        rows = rows_for_block(s, n)
+        if rows is None:
+            continue
+        p0 = w.prefix(s)
+        out = torch.full((B, H, n, D), float("nan"), dtype=torch.float32, device="cuda")
+        vq.vq_attention_block(desc, cache, s, q[:, :, p0:p0 + n], sigma, out)
+        torch.cuda.synchronize()
+        got = out[bsel].cpu().numpy()[:, :, rows]
+        khat = vo.dequantize_cache(ok_, sk, zk, w.block_tokens, nb, H, D, bits, s)
+        vhat = vo.dequantize_cache(ov_, sv, zv, w.block_tokens, nb, H, D, bits, s)
+        qs = _host(q[bsel][:, :, p0:p0 + n])[:, :, rows]
+        ref = vo.attention_f64(qs, khat, vhat, sigma)
+        rms = float(np.sqrt(np.mean(ref ** 2)))
+        err = float(np.max(np.abs(got - ref))) / rms
+        worst = max(worst, err)
+        assert np.all(np.isfinite(got)), f"block {s}: non-finite output"
+        assert err <= ATTN_TOL, f"block {s}: max|err|/rms = {err:.3e}"
+    assert vq.vq_poll_device_error() == 0
+    return worst
+
+
+def _all_rows(s, n):
+    return slice(0, n)
+
+
+def _sampled_rows(last_blocks):
+    def f(s, n):
+        if s >= last_blocks:
+            return slice(0, n)
+        return slice(0, min(n, 64))
+    return f
+
+
+# ---------------------------------------------------------------- small configs: everything
+@pytest.mark.parametrize("name", ["tiny", "var_d16"])
+def test_small_configs_full_parity(vq, name):
+    w = WORKLOADS[name]
+    k, v = make_kv(w, 0, device="cuda")
+    q = make_q(w, 0, device="cuda")
+    for bits in w.bits:
+        desc, cache = _append_all(vq, w, bits, k, v)
+        bsel = list(range(w.batch))
+        _check_cache_bit_exact(vq, w, bits, desc, cache, k, v, bsel)
+        _check_attention(vq, w, bits, desc, cache, q, k, v, bsel, _all_rows)
+
+
+# ---------------------------------------------------------------- full-size configs, sampled
+@pytest.mark.parametrize("name", ["var_d20", "var_d30", "infinity_2b"])
+def test_full_size_configs_parity(vq, name):
+    w = WORKLOADS[name]
+    layer = 1
+    k, v = make_kv(w, layer, device="cuda")
+    q = make_q(w, layer, device="cuda")
+    bsel = [0, w.batch - 1]
+    for bits in w.bits:
+        desc, cache = _append_all(vq, w, bits, k, v)
+        _check_cache_bit_exact(vq, w, bits, desc, cache, k, v, bsel)
+        last = w.num_blocks - 2
+        _check_attention(vq, w, bits, desc, cache, q, k, v, bsel,
+                         lambda s, n: (slice(0, n) if s >= last else (slice(0, min(n, 64)) if s % 3 == 0 else None)))
+        del cache
+        torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- edge cases
+def _ragged_kv(sched, D, H=3, B=1, dtype=torch.bfloat16, seed=5):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    N = sum(sched)
+    k = torch.randn((B, H, N, D), generator=g, device="cuda") * 4
+    k[..., 3] *= 40
+    v = torch.randn((B, H, N, D), generator=g, device="cuda") + 2
+    q = torch.randn((B, H, N, D), generator=g, device="cuda").to(torch.bfloat16)
+    return k.to(dtype), v.to(dtype), q
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_ragged_blocks_all_bit_widths(vq, D):
+    """Odd block sizes (1, INT3 word-row tails, cluster-split blocks) for bits 2/3/4/8;
+    dequantize is bit-exact too."""
+    sched = [1, 2, 7, 11, 81, 300, 1100, 4095]
+    k, v, q = _ragged_kv(sched, D)
+    B, H = 1, 3
+    for bits in (2, 3, 4, 8):
+        desc = vq.CacheDesc(B, H, D, bits, sched)
+        cache = vq.LayerCache(desc)
+        p0 = 0
+        kh = _host(k)
+        for s, n in enumerate(sched):
+            vq.vq_cache_append(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+            W = desc.word_rows(s)
+            offs = cache.block_word_offset
+            packed = cache.packed_k[offs[s]:offs[s + 1]]
+            scale = cache.scale_k[s * B * H * D:(s + 1) * B * H * D]
+            zero = cache.zero_k[s * B * H * D:(s + 1) * B * H * D]
+            deq = torch.empty((B, H, n, D), dtype=torch.float32, device="cuda")
+            vq.vq_dequantize(desc, s, packed, scale, zero, deq)
+            torch.cuda.synchronize()
+            words, s_ref, z_ref = vo.quantize_pack_block(kh[:, :, p0:p0 + n], bits)
+            np.testing.assert_array_equal(packed.cpu().numpy().view(np.uint32).reshape(B, H, W, D), words)
+            np.testing.assert_array_equal(scale.cpu().numpy().view(np.uint32), s_ref.reshape(-1).view(np.uint32))
+            np.testing.assert_array_equal(zero.cpu().numpy().view(np.uint32), z_ref.reshape(-1).view(np.uint32))
+            x_ref = vo.dequantize(words, s_ref, z_ref, bits, n)
+            np.testing.assert_array_equal(deq.cpu().numpy().view(np.uint32), x_ref.view(np.uint32))
+            p0 += n
+        assert vq.vq_poll_device_error() == 0
+        if bits in (3, 4):
+            _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D)
+
+
+def _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D):
+    B, H = 1, 3
+    sigma = 1.0 / np.sqrt(D)
+    ok_, sk, zk = vo.cache_append(_host(k), sched, bits)
+    ov_, sv, zv = vo.cache_append(_host(v), sched, bits)
+    p0 = 0
+    for s, n in enumerate(sched):
+        out = torch.empty((B, H, n, D), dtype=torch.float32, device="cuda")
+        vq.vq_attention_block(desc, cache, s, q[:, :, p0:p0 + n], float(sigma), out)
+        torch.cuda.synchronize()
+        rows = slice(0, min(n, 300))
+        khat = vo.dequantize_cache(ok_, sk, zk, sched, B, H, D, bits, s)
+        vhat = vo.dequantize_cache(ov_, sv, zv, sched, B, H, D, bits, s)
+        ref = vo.attention_f64(_host(q[:, :, p0:p0 + n])[:, :, rows], khat, vhat, sigma)
+        got = out.cpu().numpy()[:, :, rows]
+        err = np.max(np.abs(got - ref)) / np.sqrt(np.mean(ref ** 2))
+        assert err <= ATTN_TOL, (s, n, err)
+        p0 += n
+
+
+def test_strided_inputs_and_outputs(vq):
+    """K/V/Q given as [B][N][H][D] tensors viewed as [B][H][N][D] (row stride H*D),
+    output written into a [B][n][H][D] buffer; same bytes as contiguous inputs."""
+    B, H, D, sched, bits = 2, 4, 64, [4, 16, 64, 256], 4
+    N = sum(sched)
+    g = torch.Generator(device="cuda").manual_seed(11)
+    kt = (torch.randn((B, N, H, D), generator=g, device="cuda") * 3).to(torch.bfloat16)
+    vt = torch.randn((B, N, H, D), generator=g, device="cuda").to(torch.bfloat16)
+    qt = torch.randn((B, N, H, D), generator=g, device="cuda").to(torch.bfloat16)
+    k, v, q = kt.permute(0, 2, 1, 3), vt.permute(0, 2, 1, 3), qt.permute(0, 2, 1, 3)
+    desc = vq.CacheDesc(B, H, D, bits, sched)
+    c1, c2 = vq.LayerCache(desc), vq.LayerCache(desc)
+    p0 = 0
+    for s, n in enumerate(sched):
+        vq.vq_cache_append(desc, c1, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+        vq.vq_cache_append(desc, c2, s, k[:, :, p0:p0 + n].contiguous(), v[:, :, p0:p0 + n].contiguous())
+        p0 += n
+    torch.cuda.synchronize()
+    assert torch.equal(c1.packed_k, c2.packed_k) and torch.equal(c1.packed_v, c2.packed_v)
+    assert torch.equal(c1.scale_v, c2.scale_v) and torch.equal(c1.zero_k, c2.zero_k)
+    s = len(sched) - 1
+    n = sched[s]
+    p0 = N - n
+    o_strided = torch.empty((B, n, H, D), dtype=torch.float32, device="cuda")
+    o_contig = torch.empty((B, H, n, D), dtype=torch.float32, device="cuda")
+    vq.vq_attention_block(desc, c1, s, q[:, :, p0:p0 + n], 0.125, o_strided.permute(0, 2, 1, 3))
+    vq.vq_attention_block(desc, c1, s, q[:, :, p0:p0 + n].contiguous(), 0.125, o_contig)
+    torch.cuda.synchronize()
+    assert torch.equal(o_strided.permute(0, 2, 1, 3), o_contig)
+
+
+def test_degenerate_groups(vq):
+    """Constant channels (scale 0), a zero min stored as +0, a single-token block,
+    and a group whose range is in the float32 subnormal range."""
+    B, H, D = 1, 1, 64
+    sched = [1, 20]
+    x = torch.randn((B, H, 21, D), device="cuda", dtype=torch.float32)
+    x[..., 5] = 3.0                          # constant channel
+    x[..., 1:, 6] = x[..., 1:, 6].abs()      # channel with min exactly -0.0
+    x[..., 1, 6] = -0.0
+    x[..., 1:, 7] = 1e-40 * torch.arange(20, device="cuda", dtype=torch.float32)  # subnormal range
+    for bits in (3, 4):
+        desc = vq.CacheDesc(B, H, D, bits, sched)
+        for s, (p0, n) in enumerate(((0, 1), (1, 20))):
+            W = desc.word_rows(s)
+            packed = torch.zeros(B * H * W * D, dtype=torch.int32, device="cuda")
+            scale = torch.zeros(B * H * D, device="cuda")
+            zero = torch.zeros(B * H * D, device="cuda")
+            vq.vq_quantize_pack_block(desc, s, x[:, :, p0:p0 + n], packed, scale, zero)
+            torch.cuda.synchronize()
+            words, s_ref, z_ref = vo.quantize_pack_block(_host(x[:, :, p0:p0 + n]), bits)
+            np.testing.assert_array_equal(packed.cpu().numpy().view(np.uint32).reshape(words.shape), words)
+            np.testing.assert_array_equal(scale.cpu().numpy().view(np.uint32), s_ref.reshape(-1).view(np.uint32))
+            np.testing.assert_array_equal(zero.cpu().numpy().view(np.uint32), z_ref.reshape(-1).view(np.uint32))
+            if n == 1:
+                assert torch.all(scale == 0) and torch.all(packed == 0)
+    assert vq.vq_poll_device_error() == 0
+
+
+def test_reappend_overwrites(vq):
+    w = WORKLOADS["var_d16"]
+    k, v = make_kv(w, 3, device="cuda")
+    bits = 3
+    desc, c1 = _append_all(vq, w, bits, k, v)
+    snapshot = c1.packed_k.clone(), c1.scale_v.clone()
+    s = 7
+    p0, n = w.prefix(s), w.block_tokens[s]
+    vq.vq_cache_append(desc, c1, s, v[:, :, p0:p0 + n], k[:, :, p0:p0 + n])   # different data
+    vq.vq_cache_append(desc, c1, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])   # original again
+    torch.cuda.synchronize()
+    assert torch.equal(c1.packed_k, snapshot[0]) and torch.equal(c1.scale_v, snapshot[1])
+
+
+def test_bf16_output(vq):
+    w = WORKLOADS["tiny"]
+    k, v = make_kv(w, 0, device="cuda")
+    q = make_q(w, 0, device="cuda")
+    desc, cache = _append_all(vq, w, 4, k, v)
+    s = w.num_blocks - 1
+    p0, n = w.prefix(s), w.block_tokens[s]
+    o32 = torch.empty((1, 1, n, 64), dtype=torch.float32, device="cuda")
+    o16 = torch.empty((1, 1, n, 64), dtype=torch.bfloat16, device="cuda")
+    vq.vq_attention_block(desc, cache, s, q[:, :, p0:p0 + n], 0.125, o32)
+    vq.vq_attention_block(desc, cache, s, q[:, :, p0:p0 + n], 0.125, o16)
+    torch.cuda.synchronize()
+    assert torch.equal(o32.to(torch.bfloat16), o16)
