@@ -203,9 +203,27 @@ cudaError_t launch_attention_f32(const AttnParams& p, cudaStream_t stream) {
 }
 
 }  // namespace
+}  // namespace vq
+
+#include "attention_tc.cuh"
+
+namespace vq {
+namespace {
+
+// Blocks with at least this many queries run on the tensor cores; smaller ones
+// (mostly padding in a 128-row MMA tile) on the CUDA-core kernel.
+constexpr int kTcMinQueries = 64;
+
+}  // namespace
 
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
   if (p.B * p.H > 65535) return cudaErrorInvalidConfiguration;
+  if (p.n_q >= kTcMinQueries) {
+    if (p.bits == 4 && p.D == 64) return launch_attention_tc<4, 64>(p, stream);
+    if (p.bits == 4 && p.D == 128) return launch_attention_tc<4, 128>(p, stream);
+    if (p.bits == 3 && p.D == 64) return launch_attention_tc<3, 64>(p, stream);
+    if (p.bits == 3 && p.D == 128) return launch_attention_tc<3, 128>(p, stream);
+  }
   if (p.bits == 4 && p.D == 64) return launch_attention_f32<4, 64>(p, stream);
   if (p.bits == 4 && p.D == 128) return launch_attention_f32<4, 128>(p, stream);
   if (p.bits == 3 && p.D == 64) return launch_attention_f32<3, 64>(p, stream);
