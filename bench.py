@@ -261,6 +261,9 @@ def run_ours(args):
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
     w = WORKLOADS[args.workload]
+    if args.layers:
+        import dataclasses
+        w = dataclasses.replace(w, layers=args.layers)   # smaller case for profiler captures
     bits = args.bits or w.bits[0]
     L, S, B, H, D, N = w.layers, w.num_blocks, w.batch, w.heads, w.head_dim, w.tokens
     sigma = default_softmax_scale(w)
@@ -279,30 +282,51 @@ def run_ours(args):
     outs = [out[:, :, :n] for n in w.block_tokens]
     stream = torch.cuda.current_stream()
 
-    # events around every launch of every timed step, to split the step into kernels
-    n_launch = 2 * L * S
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(args.steps)]
-
-    def step(ev):
-        i = 0
-        if ev is not None:
-            ev[0].record(stream)
-        for s in range(S):
+    def enqueue(blocks, layers, do_quant=True, do_attn=True):
+        for s in blocks:
             p0, n = w.prefix(s), w.block_tokens[s]
-            for layer in range(L):
-                vq.vq_cache_append(desc, caches[layer], s, ks[layer][:, :, p0:p0 + n], vs[layer][:, :, p0:p0 + n],
-                                   stream=stream)
-                if ev is not None:
-                    ev[i + 1].record(stream)
-                i += 1
-                vq.vq_attention_block(desc, caches[layer], s, qs[layer][:, :, p0:p0 + n], sigma, outs[s],
-                                      stream=stream)
-                if ev is not None:
-                    ev[i + 1].record(stream)
-                i += 1
+            for layer in layers:
+                if do_quant:
+                    vq.vq_cache_append(desc, caches[layer], s, ks[layer][:, :, p0:p0 + n],
+                                       vs[layer][:, :, p0:p0 + n])
+                if do_attn:
+                    vq.vq_attention_block(desc, caches[layer], s, qs[layer][:, :, p0:p0 + n], sigma, outs[s])
+
+    # The whole step, and each kernel family per block, captured once as CUDA
+    # graphs: replays launch without host gaps, so CUDA events around a replay
+    # time the kernels themselves.
+    all_blocks, all_layers = range(S), range(L)
+    enqueue(all_blocks, all_layers)           # eager warm-up: configures kernel attributes
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    graphs = {}
+    with torch.cuda.stream(cap):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            enqueue(all_blocks, all_layers)
+        graphs["step"] = g
+        for s in all_blocks:
+            for kind in ("quant", "attn"):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap):
+                    enqueue([s], all_layers, do_quant=(kind == "quant"), do_attn=(kind == "attn"))
+                graphs[(kind, s)] = g
+    torch.cuda.current_stream().wait_stream(cap)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def timed(g, reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
 
     for _ in range(args.warmup):
-        step(None)
+        graphs["step"].replay()
     torch.cuda.synchronize()
     assert vq.vq_poll_device_error() == 0
 
@@ -314,24 +338,32 @@ def run_ours(args):
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
         start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
+        for _ in range(args.steps):
+            graphs["step"].replay()
         stop.record(stream)
         torch.cuda.synchronize()
-    t_quant = t_attn = 0.0
-    for ev in evs:
-        for j in range(n_launch):
-            dt = ev[j].elapsed_time(ev[j + 1])
-            if j % 2 == 0:
-                t_quant += dt
-            else:
-                t_attn += dt
+        # per-kernel, per-block times (same replays, each family alone)
+        by_block = []
+        t_quant = t_attn = 0.0
+        for s in range(S):
+            tq = timed(graphs[("quant", s)], args.steps)
+            ta = timed(graphs[("attn", s)], args.steps)
+            t_quant += tq
+            t_attn += ta
+            qb = quant_bytes(w, bits, s) * L
+            af, ab = attn_work(w, bits, s)
+            by_block.append({"block": s, "n": w.block_tokens[s], "quant_ms": round(tq, 4),
+                             "quant_gbs": round(qb / (tq / 1e3) / 1e9, 1), "attn_ms": round(ta, 4),
+                             "attn_gbs": round(ab * L / (ta / 1e3) / 1e9, 1),
+                             "attn_tflops": round(af * L / (ta / 1e3) / 1e12, 2)})
     barrier(world)
     elapsed_ms = start.elapsed_time(stop)
     elapsed_ms = max_over_ranks(elapsed_ms, world)
+    t_quant *= args.steps
+    t_attn *= args.steps
     assert vq.vq_poll_device_error() == 0
     clocks = clk.summary()
-
+    n_launch = 2 * L * S
     ms_step = elapsed_ms / args.steps
     tokens_step = B * N * L
     value = world * tokens_step / (ms_step / 1e3)
@@ -370,6 +402,9 @@ def run_ours(args):
         "roofline": roof,
         "clocks": clocks,
         "gpu_launches": n_launch * args.steps,
+        "timing": "step = one CUDA-graph replay of the whole decode; per-kernel times from graphs of each kernel "
+                  "family per block, replayed alone",
+        "by_block": by_block,
     }
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, vq, w, bits, desc, caches, outs, dev, world)
@@ -445,6 +480,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-units", type=int, default=8)
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling only)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

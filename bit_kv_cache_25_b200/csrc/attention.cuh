@@ -14,9 +14,11 @@
 // so the integer codes enter the products exactly and the per-block scales are
 // applied once per (query, block, channel).
 //
-// This is the general kernel: float32 CUDA-core arithmetic, one CTA per
-// (b, h, 32 queries), 4 warps x 8 queries, 32 keys per step (one per lane),
-// online softmax in float32.
+// This file holds the kernel for blocks with few queries (fewer than
+// kTcMinQueries): one CTA per (b, h), one warp per query, lanes across
+// channels. Each key's logit is a warp reduction over channels; the softmax is
+// online in fp32 (one pass over the keys). The packed words of a word-row are
+// read once per warp and serve its cpw keys from L1.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -28,177 +30,109 @@
 namespace vq {
 namespace {
 
-constexpr int kAttnQ = 32;       // queries per CTA
-constexpr int kAttnWarps = 4;    // 8 queries per warp
-constexpr int kAttnQW = kAttnQ / kAttnWarps;
-constexpr int kAttnKeys = 32;    // keys per step
+constexpr int kSmallWarps = 4;
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float(static_cast<uint32_t>(h) << 16); }
 
-template <int D>
-struct AttnF32Smem {
-  float q[kAttnQ][D + 4];          // q' = sigma * q * sk for the current key block
-  float qs[kAttnQ][D];             // sigma * q
-  float bias[kAttnQ];              // sigma * q . zk
-  float kt[D][kAttnKeys + 1];      // key codes, [channel][key]
-  float v[kAttnKeys][D];           // value codes, [key][channel]
-  float p[kAttnWarps][kAttnQW][kAttnKeys];
-  float meta[4][D];                // sk, zk, sv, zv of the current block
-};
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;  // butterfly of commutative adds: identical on every lane
+}
 
 template <int BITS, int D>
-__global__ void __launch_bounds__(kAttnWarps * 32) attention_f32_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(kSmallWarps * 32) attention_small_kernel(const __grid_constant__ AttnParams p) {
   constexpr int CPW = 32 / BITS;
   constexpr uint32_t MASK = (1u << BITS) - 1u;
-  constexpr int CPL = D / 32;  // output channels per lane
-  extern __shared__ __align__(16) unsigned char attn_smem_raw[];
-  AttnF32Smem<D>& S = *reinterpret_cast<AttnF32Smem<D>*>(attn_smem_raw);
-  auto& sQ = S.q;
-  auto& sQs = S.qs;
-  auto& sBias = S.bias;
-  auto& sKT = S.kt;
-  auto& sV = S.v;
-  auto& sP = S.p;
-  auto& sMeta = S.meta;
-
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  const int bh = blockIdx.y;
+  constexpr int J = D / 32;  // channels per lane
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int bh = blockIdx.x;
   const int b = bh / p.H;
   const int h = bh - b * p.H;
-  const int q0 = blockIdx.x * kAttnQ;
-  const int BHD = p.B * p.H * D;
+  const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
 
-  // sigma * q for this CTA's queries (rows past n_q are zero)
-  for (int e = tid; e < kAttnQ * D; e += blockDim.x) {
-    const int qi = e / D;
-    const int c = e - qi * D;
-    float v = 0.0f;
-    if (q0 + qi < p.n_q) v = bf16_to_f32(p.q[b * p.q_sb + h * p.q_sh + int64_t(q0 + qi) * p.q_st + c]);
-    sQs[qi][c] = __fmul_rn(p.softmax_scale, v);
-  }
-
-  float m[kAttnQW], l[kAttnQW], o[kAttnQW][CPL];
+  for (int qi = warp; qi < p.n_q; qi += kSmallWarps) {
+    const uint16_t* qrow = p.q + b * p.q_sb + h * p.q_sh + static_cast<int64_t>(qi) * p.q_st;
+    float qs[J], o[J];
 #pragma unroll
-  for (int i = 0; i < kAttnQW; ++i) {
-    m[i] = -INFINITY;
-    l[i] = 0.0f;
+    for (int j = 0; j < J; ++j) {
+      qs[j] = __fmul_rn(p.softmax_scale, bf16_to_f32(qrow[lane + 32 * j]));
+      o[j] = 0.0f;
+    }
+    float m = -INFINITY, l = 0.0f;
+    for (int kb = 0; kb <= p.s; ++kb) {
+      const AttnBlockInfo bi = p.blk[kb];
+      float qp[J], sv[J], zv[J], u[J];
+      float bias = 0.0f;
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) o[i][j] = 0.0f;
-  }
-
-  for (int kb = 0; kb <= p.s; ++kb) {
-    const AttnBlockInfo bi = p.blk[kb];
-    __syncthreads();
-    for (int c = tid; c < D; c += blockDim.x) {
-      const int64_t mo = int64_t(kb) * BHD + int64_t(bh) * D + c;
-      sMeta[0][c] = p.scale_k[mo];
-      sMeta[1][c] = p.zero_k[mo];
-      sMeta[2][c] = p.scale_v[mo];
-      sMeta[3][c] = p.zero_v[mo];
-    }
-    __syncthreads();
-    for (int e = tid; e < kAttnQ * D; e += blockDim.x) {
-      const int qi = e / D;
-      const int c = e - qi * D;
-      sQ[qi][c] = __fmul_rn(sQs[qi][c], sMeta[0][c]);
-    }
-    if (tid < kAttnQ) {
-      float acc = 0.0f;
-      for (int c = 0; c < D; ++c) acc = fmaf(sQs[tid][c], sMeta[1][c], acc);
-      sBias[tid] = acc;
-    }
-    const uint32_t* pk = p.packed_k + bi.word_off + int64_t(bh) * bi.W * D;
-    const uint32_t* pv = p.packed_v + bi.word_off + int64_t(bh) * bi.W * D;
-
-    for (int t0 = 0; t0 < bi.n; t0 += kAttnKeys) {
-      __syncthreads();
-      for (int e = tid; e < kAttnKeys * D; e += blockDim.x) {
-        const int kk = e / D;
-        const int c = e - kk * D;
-        const int t = t0 + kk;
-        float ck = 0.0f, cv = 0.0f;
-        if (t < bi.n) {
-          const int w = t / CPW;
-          const int sh = BITS * (t - w * CPW);
-          ck = static_cast<float>((pk[int64_t(w) * D + c] >> sh) & MASK);
-          cv = static_cast<float>((pv[int64_t(w) * D + c] >> sh) & MASK);
-        }
-        sKT[c][kk] = ck;
-        sV[kk][c] = cv;
+      for (int j = 0; j < J; ++j) {
+        const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + lane + 32 * j;
+        qp[j] = __fmul_rn(qs[j], p.scale_k[mo]);
+        bias = fmaf(qs[j], p.zero_k[mo], bias);
+        sv[j] = p.scale_v[mo];
+        zv[j] = p.zero_v[mo];
+        u[j] = 0.0f;
       }
-      __syncthreads();
-      const bool valid = (t0 + lane) < bi.n;
-      const int nk = min(kAttnKeys, bi.n - t0);
+      bias = warp_sum(bias);
+      float rs = 0.0f;
+      const uint32_t* pk = p.packed_k + bi.word_off + static_cast<int64_t>(bh) * bi.W * D;
+      const uint32_t* pv = p.packed_v + bi.word_off + static_cast<int64_t>(bh) * bi.W * D;
+      for (int w = 0; w < bi.W; ++w) {
+        uint32_t wk[J], wv[J];
 #pragma unroll
-      for (int i = 0; i < kAttnQW; ++i) {
-        const int qi = warp * kAttnQW + i;
-        float s = sBias[qi];
-#pragma unroll 8
-        for (int c = 0; c < D; ++c) s = fmaf(sQ[qi][c], sKT[c][lane], s);
-        s = valid ? s : -INFINITY;
-        float mx = s;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float m_new = fmaxf(m[i], mx);
-        const float alpha = expf(m[i] - m_new);  // exp(-inf) = 0 on the first step
-        const float pr = valid ? expf(s - m_new) : 0.0f;
-        float sum = pr;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        sP[warp][i][lane] = pr;
-        __syncwarp();
-#pragma unroll
-        for (int j = 0; j < CPL; ++j) {
-          const int c = lane + 32 * j;
-          float u = 0.0f;
-          for (int t = 0; t < nk; ++t) u = fmaf(sP[warp][i][t], sV[t][c], u);
-          o[i][j] = fmaf(o[i][j], alpha, fmaf(sMeta[2][c], u, sMeta[3][c] * sum));
+        for (int j = 0; j < J; ++j) {
+          wk[j] = pk[static_cast<int64_t>(w) * D + lane + 32 * j];
+          wv[j] = pv[static_cast<int64_t>(w) * D + lane + 32 * j];
         }
-        l[i] = fmaf(l[i], alpha, sum);
-        m[i] = m_new;
-        __syncwarp();
+        const int nslot = min(CPW, bi.n - w * CPW);
+#pragma unroll
+        for (int i = 0; i < CPW; ++i) {
+          if (i >= nslot) break;
+          float dot = 0.0f;
+#pragma unroll
+          for (int j = 0; j < J; ++j) dot = fmaf(qp[j], static_cast<float>((wk[j] >> (BITS * i)) & MASK), dot);
+          const float sc = warp_sum(dot) + bias;
+          if (sc > m) {  // uniform across the warp
+            const float alpha = expf(m - sc);
+            m = sc;
+            l *= alpha;
+            rs *= alpha;
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+              o[j] *= alpha;
+              u[j] *= alpha;
+            }
+          }
+          const float pr = expf(sc - m);
+          l += pr;
+          rs += pr;
+#pragma unroll
+          for (int j = 0; j < J; ++j) u[j] = fmaf(pr, static_cast<float>((wv[j] >> (BITS * i)) & MASK), u[j]);
+        }
       }
+#pragma unroll
+      for (int j = 0; j < J; ++j) o[j] = fmaf(u[j], sv[j], fmaf(rs, zv[j], o[j]));
     }
-  }
-
+    const float inv = 1.0f / l;
+    const int64_t obase = b * p.o_sb + h * p.o_sh + static_cast<int64_t>(qi) * p.o_st;
 #pragma unroll
-  for (int i = 0; i < kAttnQW; ++i) {
-    const int qi = q0 + warp * kAttnQW + i;
-    if (qi >= p.n_q) continue;
-    const float inv = 1.0f / l[i];
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-      const int c = lane + 32 * j;
-      const float val = o[i][j] * inv;
-      const int64_t off = b * p.o_sb + h * p.o_sh + int64_t(qi) * p.o_st + c;
+    for (int j = 0; j < J; ++j) {
+      const float val = o[j] * inv;
       if (p.out_f32) {
-        static_cast<float*>(p.out)[off] = val;
+        static_cast<float*>(p.out)[obase + lane + 32 * j] = val;
       } else {
-        const uint32_t u = __float_as_uint(val);
-        const uint32_t r = (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;  // round to nearest even
-        static_cast<uint16_t*>(p.out)[off] = static_cast<uint16_t>(r);
+        const uint32_t x = __float_as_uint(val);
+        static_cast<uint16_t*>(p.out)[obase + lane + 32 * j] =
+            static_cast<uint16_t>((x + 0x7fffu + ((x >> 16) & 1u)) >> 16);  // round to nearest even
       }
     }
   }
 }
 
 template <int BITS, int D>
-cudaError_t launch_attention_f32(const AttnParams& p, cudaStream_t stream) {
-  dim3 grid((p.n_q + kAttnQ - 1) / kAttnQ, p.B * p.H);
-  const int smem = static_cast<int>(sizeof(AttnF32Smem<D>));
-  static bool configured[kMaxDevices] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(attention_f32_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
-  attention_f32_kernel<BITS, D><<<grid, kAttnWarps * 32, smem, stream>>>(p);
+cudaError_t launch_attention_small(const AttnParams& p, cudaStream_t stream) {
+  attention_small_kernel<BITS, D><<<p.B * p.H, kSmallWarps * 32, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -206,28 +140,29 @@ cudaError_t launch_attention_f32(const AttnParams& p, cudaStream_t stream) {
 }  // namespace vq
 
 #include "attention_tc.cuh"
+#include "attention_ws.cuh"
 
 namespace vq {
 namespace {
 
 // Blocks with at least this many queries run on the tensor cores; smaller ones
 // (mostly padding in a 128-row MMA tile) on the CUDA-core kernel.
-constexpr int kTcMinQueries = 64;
+constexpr int kTcMinQueries = 16;
 
 }  // namespace
 
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
-  if (p.B * p.H > 65535) return cudaErrorInvalidConfiguration;
   if (p.n_q >= kTcMinQueries) {
+    if (p.B * p.H > 65535) return cudaErrorInvalidConfiguration;
     if (p.bits == 4 && p.D == 64) return launch_attention_tc<4, 64>(p, stream);
     if (p.bits == 4 && p.D == 128) return launch_attention_tc<4, 128>(p, stream);
     if (p.bits == 3 && p.D == 64) return launch_attention_tc<3, 64>(p, stream);
     if (p.bits == 3 && p.D == 128) return launch_attention_tc<3, 128>(p, stream);
   }
-  if (p.bits == 4 && p.D == 64) return launch_attention_f32<4, 64>(p, stream);
-  if (p.bits == 4 && p.D == 128) return launch_attention_f32<4, 128>(p, stream);
-  if (p.bits == 3 && p.D == 64) return launch_attention_f32<3, 64>(p, stream);
-  if (p.bits == 3 && p.D == 128) return launch_attention_f32<3, 128>(p, stream);
+  if (p.bits == 4 && p.D == 64) return launch_attention_small<4, 64>(p, stream);
+  if (p.bits == 4 && p.D == 128) return launch_attention_small<4, 128>(p, stream);
+  if (p.bits == 3 && p.D == 64) return launch_attention_small<3, 64>(p, stream);
+  if (p.bits == 3 && p.D == 128) return launch_attention_small<3, 128>(p, stream);
   return cudaErrorInvalidValue;
 }
 

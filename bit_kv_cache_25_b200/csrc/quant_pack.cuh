@@ -48,13 +48,14 @@ constexpr float kRoundMagic = 12582912.0f;
 
 struct QuantSmem {
   // layout inside dynamic shared memory (byte offsets)
-  uint32_t bar, mnk, mxk, mn, inv, stage;
+  uint32_t bar, mnk, mxk, mn, inv, stage, stage_bytes;
   uint32_t total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline QuantSmem quant_smem_layout(int G, int D, int rows_chunk, int rowbytes) {
+// `stages` staging buffers of G slabs of rows_chunk rows each.
+__host__ __device__ inline QuantSmem quant_smem_layout(int G, int D, int rows_chunk, int rowbytes, int stages) {
   QuantSmem L;
   L.bar = 0;
   L.mnk = 16;
@@ -62,7 +63,8 @@ __host__ __device__ inline QuantSmem quant_smem_layout(int G, int D, int rows_ch
   L.mn = L.mxk + 4u * G * D;
   L.inv = L.mn + 4u * G * D;
   L.stage = align_up(L.inv + 4u * G * D, 128);
-  L.total = L.stage + static_cast<uint32_t>(G) * rows_chunk * rowbytes;
+  L.stage_bytes = align_up(static_cast<uint32_t>(G) * rows_chunk * rowbytes, 128);
+  L.total = L.stage + stages * L.stage_bytes;
   return L;
 }
 
@@ -123,211 +125,300 @@ struct F32Vec {
   }
 };
 
+// Work of one CTA-step: `units` consecutive units starting at `unit0`, each
+// restricted to the token rows [row0, row0 + rows) / word-rows [wr0, wr0 + wrs).
+struct QuantStep {
+  int unit0, units, row0, rows, wr0, wrs;
+};
+
+// Warp 0: stage the slabs of one step into `stage` (completion on `bar`).
+__device__ __forceinline__ void quant_issue_copies(const QuantParams& p, const QuantStep& st, unsigned char* stage,
+                                                   uint64_t* bar, int rowbytes) {
+  const int tid = threadIdx.x;
+  if (tid >= 32) return;
+  const uint32_t total = static_cast<uint32_t>(st.units) * st.rows * rowbytes;
+  if (tid == 0) mbar_arrive_expect_tx(bar, total);
+  __syncwarp();
+  const int BH = p.B * p.H;
+  for (int g = 0; g < st.units; ++g) {
+    const int unit = st.unit0 + g;
+    const QuantTensor& T = p.t[unit / BH];
+    const int bh = unit % BH;
+    const int64_t base = (bh / p.H) * T.sb + (bh % p.H) * T.sh;
+    const unsigned char* src = static_cast<const unsigned char*>(T.x) + (base + int64_t(st.row0) * T.st) * p.esize;
+    unsigned char* dst = stage + static_cast<size_t>(g) * p.rows_chunk * rowbytes;
+    if (T.st * p.esize == rowbytes) {
+      if (tid == 0) bulk_copy_g2s(dst, src, static_cast<uint32_t>(st.rows) * rowbytes, bar);
+    } else {
+      for (int r = tid; r < st.rows; r += 32)
+        bulk_copy_g2s(dst + r * rowbytes, src + int64_t(r) * T.st * p.esize, rowbytes, bar);
+    }
+  }
+}
+
+// Pass 1: per-task min/max over the task's cpw rows, merged into the
+// per-(unit, channel) key slots with shared-memory atomics.
 template <class Vec, int BITS>
-__global__ void __launch_bounds__(kQuantThreads) quant_pack_kernel(const __grid_constant__ QuantParams p) {
+__device__ __forceinline__ void quant_pass1(const QuantParams& p, const QuantStep& st, const unsigned char* stage,
+                                            int32_t* mnk, int32_t* mxk) {
   constexpr int CPW = 32 / BITS;
   constexpr int CH = Vec::kCh;
-  extern __shared__ __align__(128) unsigned char smem[];
-
-  const int D = p.D;
   const int V = p.vecs_per_row;
   const int rowbytes = V * 16;
-  const int rows_chunk = p.rows_chunk;
-  const QuantSmem L = quant_smem_layout(p.G, D, rows_chunk, rowbytes);
+  const int D = p.D;
+  const int tpu = st.wrs * V;
+  for (int task = threadIdx.x; task < st.units * tpu; task += blockDim.x) {
+    const int g = task / tpu;
+    const int r = task - g * tpu;
+    const int wl = r / V;
+    const int j = r - wl * V;
+    const int tl0 = wl * CPW;
+    const int nvalid = min(CPW, st.rows - tl0);
+    const unsigned char* src = stage + (static_cast<size_t>(g) * p.rows_chunk + tl0) * rowbytes + j * 16;
+    uint32_t mn[4], mx[4];
+    Vec::minmax_init(mn, mx, lds128(src));
+#pragma unroll
+    for (int i = 1; i < CPW; ++i)
+      if (i < nvalid) Vec::minmax_acc(mn, mx, lds128(src + i * rowbytes));
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      atomicMin(&mnk[g * D + j * CH + c], float_key(Vec::ch(mn, c)));
+      atomicMax(&mxk[g * D + j * CH + c], float_key(Vec::ch(mx, c)));
+    }
+  }
+}
+
+// Per group: scale = (max - min) / (2^b - 1) (IEEE division), zero = min + 0,
+// inv = min(1/scale, FLT_MAX) (IEEE reciprocal), written to shared memory for
+// pass 2 and (when `write`) to the output arrays.
+template <int BITS>
+__device__ __forceinline__ void quant_finalize(const QuantParams& p, const QuantStep& st, int32_t kmn, int32_t kmx,
+                                               int i, float* s_mn, float* s_inv, bool write) {
+  const int D = p.D;
+  const float mn = key_float(kmn);
+  const float mx = key_float(kmx);
+  const float diff = __fsub_rn(mx, mn);
+  const float scale = __fdiv_rn(diff, static_cast<float>((1 << BITS) - 1));
+  const float zero = __fadd_rn(mn, 0.0f);
+  const float inv = (scale > 0.0f) ? fminf(__frcp_rn(scale), FLT_MAX) : 0.0f;
+  s_mn[i] = mn;
+  s_inv[i] = inv;
+  if (write) {
+    const int BH = p.B * p.H;
+    const int g = i / D;
+    const int c = i - g * D;
+    const int unit = st.unit0 + g;
+    const QuantTensor& T = p.t[unit / BH];
+    const int bh = unit % BH;
+    T.scale[static_cast<size_t>(bh) * D + c] = scale;
+    T.zero[static_cast<size_t>(bh) * D + c] = zero;
+  }
+}
+
+// Pass 2: encode and pack. d = x - min and t = d * inv, each correctly rounded,
+// then round half to even by adding 1.5 * 2^23: the rounded value's low
+// mantissa bits are the code (t <= 2^b - 1 + tiny, so no clamp is needed).
+// Codes are summed into the word with shifts; the magic bits are removed once.
+template <class Vec, int BITS>
+__device__ __forceinline__ void quant_pass2(const QuantParams& p, const QuantStep& st, const unsigned char* stage,
+                                            const float* s_mn, const float* s_inv) {
+  constexpr int CPW = 32 / BITS;
+  constexpr int CH = Vec::kCh;
+  const int V = p.vecs_per_row;
+  const int rowbytes = V * 16;
+  const int D = p.D;
+  const int BH = p.B * p.H;
+  const int tpu = st.wrs * V;
+  for (int task = threadIdx.x; task < st.units * tpu; task += blockDim.x) {
+    const int g = task / tpu;
+    const int r = task - g * tpu;
+    const int wl = r / V;
+    const int j = r - wl * V;
+    const int tl0 = wl * CPW;
+    const int nvalid = min(CPW, st.rows - tl0);
+    const unsigned char* src = stage + (static_cast<size_t>(g) * p.rows_chunk + tl0) * rowbytes + j * 16;
+    float mn[CH], inv[CH];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      mn[c] = s_mn[g * D + j * CH + c];
+      inv[c] = s_inv[g * D + j * CH + c];
+    }
+    uint32_t acc[CH];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) acc[c] = 0u;
+    uint32_t corr = 0u;
+#pragma unroll
+    for (int i = 0; i < CPW; ++i) {
+      if (i < nvalid) {
+        const uint4 v = lds128(src + i * rowbytes);
+        corr += kRoundMagicBits << (BITS * i);
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const float d = __fsub_rn(Vec::elem(v, c), mn[c]);
+          const float t = __fmul_rn(d, inv[c]);
+          const float rq = __fadd_rn(t, kRoundMagic);
+          acc[c] += __float_as_uint(rq) << (BITS * i);
+        }
+      }
+    }
+    const int unit = st.unit0 + g;
+    const QuantTensor& T = p.t[unit / BH];
+    const int bh = unit % BH;
+    uint32_t* dst = T.packed + (static_cast<size_t>(bh) * p.W + st.wr0 + wl) * D + j * CH;
+#pragma unroll
+    for (int q = 0; q < CH / 4; ++q)
+      reinterpret_cast<uint4*>(dst)[q] =
+          make_uint4(acc[4 * q] - corr, acc[4 * q + 1] - corr, acc[4 * q + 2] - corr, acc[4 * q + 3] - corr);
+  }
+}
+
+// Blocks whose (tensor, b, h) slab fits one CTA: a persistent loop over groups
+// of G units with a two-stage bulk-copy pipeline, so the next group's slabs
+// are in flight while this group is reduced, encoded and stored.
+template <class Vec, int BITS>
+__global__ void __launch_bounds__(kQuantThreads) quant_pack_stream_kernel(const __grid_constant__ QuantParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int D = p.D;
+  const int rowbytes = p.vecs_per_row * 16;
+  const QuantSmem L = quant_smem_layout(p.G, D, p.rows_chunk, rowbytes, 2);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);
   int32_t* mnk = reinterpret_cast<int32_t*>(smem + L.mnk);
   int32_t* mxk = reinterpret_cast<int32_t*>(smem + L.mxk);
   float* s_mn = reinterpret_cast<float*>(smem + L.mn);
   float* s_inv = reinterpret_cast<float*>(smem + L.inv);
-  unsigned char* stage = smem + L.stage;
+  const int tid = threadIdx.x;
+  const int groups = (p.units + p.G - 1) / p.G;
 
+  auto step_of = [&](int grp) {
+    QuantStep st;
+    st.unit0 = grp * p.G;
+    st.units = min(p.G, p.units - st.unit0);
+    st.row0 = 0;
+    st.rows = p.n;
+    st.wr0 = 0;
+    st.wrs = p.W;
+    return st;
+  };
+
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  int grp = blockIdx.x;
+  if (grp < groups) quant_issue_copies(p, step_of(grp), smem + L.stage, &bar[0], rowbytes);
+  bool ok = true;
+  for (int it = 0; grp < groups; ++it, grp += gridDim.x) {
+    const QuantStep st = step_of(grp);
+    const int stg = it & 1;
+    // prefetch the next group into the other stage (its last reader finished
+    // at the barrier that ended the previous iteration)
+    const int nxt = grp + gridDim.x;
+    if (nxt < groups) quant_issue_copies(p, step_of(nxt), smem + L.stage + (stg ^ 1) * L.stage_bytes, &bar[stg ^ 1], rowbytes);
+    for (int i = tid; i < st.units * D; i += blockDim.x) {
+      mnk[i] = INT32_MAX;
+      mxk[i] = INT32_MIN;
+    }
+    ok = __syncthreads_and(mbar_wait_bounded(&bar[stg], (it >> 1) & 1));
+    if (!ok) break;
+    const unsigned char* stage = smem + L.stage + stg * L.stage_bytes;
+    quant_pass1<Vec, BITS>(p, st, stage, mnk, mxk);
+    __syncthreads();
+    for (int i = tid; i < st.units * D; i += blockDim.x) quant_finalize<BITS>(p, st, mnk[i], mxk[i], i, s_mn, s_inv, true);
+    __syncthreads();
+    quant_pass2<Vec, BITS>(p, st, stage, s_mn, s_inv);
+    fence_proxy_async_smem();  // generic reads of this stage before the next bulk copy overwrites it
+    __syncthreads();
+  }
+}
+
+// Blocks whose slab is split over a cluster of C CTAs: each CTA stages its
+// chunk of word-rows; the per-channel partial min/max are combined through
+// distributed shared memory, so HBM is read exactly once.
+template <class Vec, int BITS>
+__global__ void __launch_bounds__(kQuantThreads) quant_pack_cluster_kernel(const __grid_constant__ QuantParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int D = p.D;
+  const int rowbytes = p.vecs_per_row * 16;
+  const QuantSmem L = quant_smem_layout(1, D, p.rows_chunk, rowbytes, 1);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);
+  int32_t* mnk = reinterpret_cast<int32_t*>(smem + L.mnk);
+  int32_t* mxk = reinterpret_cast<int32_t*>(smem + L.mxk);
+  float* s_mn = reinterpret_cast<float*>(smem + L.mn);
+  float* s_inv = reinterpret_cast<float*>(smem + L.inv);
+  constexpr int CPW = 32 / BITS;
   const int C = p.C;
-  const uint32_t rank = (C > 1) ? cluster_ctarank() : 0u;
-  const int cta_unit0 = (C > 1) ? static_cast<int>(blockIdx.x) / C : static_cast<int>(blockIdx.x) * p.G;
-  const int wr0 = static_cast<int>(rank) * p.wr_chunk;   // first word-row of this CTA's chunk
-  const int row0 = wr0 * CPW;                            // first token of the chunk
-  const int G = p.G;
-  const int n = p.n;
-  const int BH = p.B * p.H;
+  const uint32_t rank = cluster_ctarank();
   const int tid = threadIdx.x;
 
-  // number of this CTA's units that exist (the last CTA may be partial)
-  const int units_here = min(G, p.units - cta_unit0);
-  const int wr_here = max(0, min(p.wr_chunk, p.W - wr0));
-  const int rows_here = max(0, min(rows_chunk, n - row0));
+  QuantStep st;
+  st.unit0 = static_cast<int>(blockIdx.x) / C;
+  st.units = 1;
+  st.wr0 = static_cast<int>(rank) * p.wr_chunk;
+  st.wrs = max(0, min(p.wr_chunk, p.W - st.wr0));
+  st.row0 = st.wr0 * CPW;
+  st.rows = max(0, min(p.rows_chunk, p.n - st.row0));
 
-  // ---- stage the slab chunks in shared memory
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_barrier_init();
   }
-  for (int i = tid; i < G * D; i += blockDim.x) {
+  for (int i = tid; i < D; i += blockDim.x) {
     mnk[i] = INT32_MAX;
     mxk[i] = INT32_MIN;
   }
   __syncthreads();
-
-  if (tid < 32) {
-    const uint32_t total = static_cast<uint32_t>(units_here) * rows_here * rowbytes;
-    if (tid == 0) mbar_arrive_expect_tx(bar, total);
-    __syncwarp();
-    if (rows_here > 0) {
-      for (int g = 0; g < units_here; ++g) {
-        const int unit = cta_unit0 + g;
-        const int tsel = unit / BH;
-        const int bh = unit % BH;
-        const QuantTensor& T = p.t[tsel];
-        const int64_t base = (bh / p.H) * T.sb + (bh % p.H) * T.sh;
-        const unsigned char* src = static_cast<const unsigned char*>(T.x) + (base + int64_t(row0) * T.st) * p.esize;
-        unsigned char* dst = stage + static_cast<size_t>(g) * rows_chunk * rowbytes;
-        if (T.st * p.esize == rowbytes) {
-          if (tid == 0) bulk_copy_g2s(dst, src, static_cast<uint32_t>(rows_here) * rowbytes, bar);
-        } else {
-          for (int r = tid; r < rows_here; r += 32)
-            bulk_copy_g2s(dst + r * rowbytes, src + int64_t(r) * T.st * p.esize, rowbytes, bar);
-        }
-      }
-    }
-  }
-  const bool staged = mbar_wait_bounded(bar, 0);
-
-  // ---- pass 1: per-channel min/max
-  const int tasks_per_unit = wr_here * V;
-  const int ntask = units_here * tasks_per_unit;
-  if (staged) {
-    for (int task = tid; task < ntask; task += blockDim.x) {
-      const int g = task / tasks_per_unit;
-      const int r = task - g * tasks_per_unit;
-      const int wl = r / V;
-      const int j = r - wl * V;
-      const int tl0 = wl * CPW;
-      const int nvalid = min(CPW, rows_here - tl0);
-      const unsigned char* src = stage + (static_cast<size_t>(g) * rows_chunk + tl0) * rowbytes + j * 16;
-      uint32_t mn[4], mx[4];
-      Vec::minmax_init(mn, mx, lds128(src));
-#pragma unroll
-      for (int i = 1; i < CPW; ++i)
-        if (i < nvalid) Vec::minmax_acc(mn, mx, lds128(src + i * rowbytes));
-#pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        atomicMin(&mnk[g * D + j * CH + c], float_key(Vec::ch(mn, c)));
-        atomicMax(&mxk[g * D + j * CH + c], float_key(Vec::ch(mx, c)));
-      }
-    }
-  }
+  quant_issue_copies(p, st, smem + L.stage, bar, rowbytes);
+  const bool staged = __syncthreads_and(mbar_wait_bounded(bar, 0));
+  if (staged) quant_pass1<Vec, BITS>(p, st, smem + L.stage, mnk, mxk);
   __syncthreads();
 
-  // ---- combine across the cluster (one unit per cluster)
-  int32_t fmn = 0, fmx = 0;
-  if (C > 1) {
-    cluster_sync();  // every CTA's partials are complete and visible
-    if (tid < D) {
-      fmn = INT32_MAX;
-      fmx = INT32_MIN;
-      for (int r = 0; r < C; ++r) {
-        fmn = min(fmn, dsmem_ld_s32(&mnk[tid], r));
-        fmx = max(fmx, dsmem_ld_s32(&mxk[tid], r));
-      }
-    }
-    cluster_arrive();  // done reading peers; the matching wait is at the end
-  }
-
-  // ---- per-group scale, zero, reciprocal
-  for (int i = tid; i < units_here * D; i += blockDim.x) {
-    const int32_t kmn = (C > 1) ? fmn : mnk[i];
-    const int32_t kmx = (C > 1) ? fmx : mxk[i];
-    const float mn = key_float(kmn);
-    const float mx = key_float(kmx);
-    const float diff = __fsub_rn(mx, mn);
-    const float scale = __fdiv_rn(diff, static_cast<float>((1 << BITS) - 1));
-    const float zero = __fadd_rn(mn, 0.0f);
-    const float inv = (scale > 0.0f) ? fminf(__frcp_rn(scale), FLT_MAX) : 0.0f;
-    s_mn[i] = mn;
-    s_inv[i] = inv;
-    if (rank == 0 && staged) {
-      const int g = i / D;
-      const int c = i - g * D;
-      const int unit = cta_unit0 + g;
-      const QuantTensor& T = p.t[unit / BH];
-      const int bh = unit % BH;
-      T.scale[static_cast<size_t>(bh) * D + c] = scale;
-      T.zero[static_cast<size_t>(bh) * D + c] = zero;
+  cluster_sync();  // every CTA's partials are complete and visible
+  int32_t fmn = INT32_MAX, fmx = INT32_MIN;
+  if (tid < D) {
+    for (int r = 0; r < C; ++r) {
+      fmn = min(fmn, dsmem_ld_s32(&mnk[tid], r));
+      fmx = max(fmx, dsmem_ld_s32(&mxk[tid], r));
     }
   }
+  cluster_arrive();  // done reading peers; the matching wait is at the end
+  if (tid < D) quant_finalize<BITS>(p, st, fmn, fmx, tid, s_mn, s_inv, rank == 0 && staged);
   __syncthreads();
-
-  // ---- pass 2: encode and pack
-  if (staged) {
-    for (int task = tid; task < ntask; task += blockDim.x) {
-      const int g = task / tasks_per_unit;
-      const int r = task - g * tasks_per_unit;
-      const int wl = r / V;
-      const int j = r - wl * V;
-      const int tl0 = wl * CPW;
-      const int nvalid = min(CPW, rows_here - tl0);
-      const unsigned char* src = stage + (static_cast<size_t>(g) * rows_chunk + tl0) * rowbytes + j * 16;
-      float mn[CH], inv[CH];
-#pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        mn[c] = s_mn[g * D + j * CH + c];
-        inv[c] = s_inv[g * D + j * CH + c];
-      }
-      uint32_t acc[CH];
-#pragma unroll
-      for (int c = 0; c < CH; ++c) acc[c] = 0u;
-      uint32_t corr = 0u;
-#pragma unroll
-      for (int i = 0; i < CPW; ++i) {
-        if (i < nvalid) {
-          const uint4 v = lds128(src + i * rowbytes);
-          corr += kRoundMagicBits << (BITS * i);
-#pragma unroll
-          for (int c = 0; c < CH; ++c) {
-            const float d = __fsub_rn(Vec::elem(v, c), mn[c]);
-            const float t = __fmul_rn(d, inv[c]);
-            const float rq = __fadd_rn(t, kRoundMagic);
-            acc[c] += __float_as_uint(rq) << (BITS * i);
-          }
-        }
-      }
-      const int unit = cta_unit0 + g;
-      const QuantTensor& T = p.t[unit / BH];
-      const int bh = unit % BH;
-      uint32_t* dst = T.packed + (static_cast<size_t>(bh) * p.W + wr0 + wl) * D + j * CH;
-#pragma unroll
-      for (int q = 0; q < CH / 4; ++q)
-        reinterpret_cast<uint4*>(dst)[q] =
-            make_uint4(acc[4 * q] - corr, acc[4 * q + 1] - corr, acc[4 * q + 2] - corr, acc[4 * q + 3] - corr);
-    }
-  }
-
-  if (C > 1) cluster_wait();  // peers may still read this CTA's partials until here
+  if (staged) quant_pass2<Vec, BITS>(p, st, smem + L.stage, s_mn, s_inv);
+  cluster_wait();  // peers may still read this CTA's partials until here
 }
 
 template <class Vec, int BITS>
 cudaError_t launch_typed(const QuantParams& p, cudaStream_t stream) {
-  auto kern = quant_pack_kernel<Vec, BITS>;
+  const bool cluster = p.C > 1;
+  auto kern = cluster ? quant_pack_cluster_kernel<Vec, BITS> : quant_pack_stream_kernel<Vec, BITS>;
   const int rowbytes = p.vecs_per_row * 16;
-  const QuantSmem L = quant_smem_layout(p.G, p.D, p.rows_chunk, rowbytes);
+  const QuantSmem L = quant_smem_layout(cluster ? 1 : p.G, p.D, p.rows_chunk, rowbytes, cluster ? 1 : 2);
   // Function attributes are set once per device and size, outside any stream
   // work, so launches can be captured into CUDA graphs.
-  static int configured_smem[kMaxDevices] = {};
+  static int configured_smem[2][kMaxDevices] = {};
   static bool configured_cluster[kMaxDevices] = {};
+  static int sm_count[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (static_cast<int>(L.total) > configured_smem[dev]) {
+  if (static_cast<int>(L.total) > configured_smem[cluster][dev]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
     if (e != cudaSuccess) return e;
-    configured_smem[dev] = static_cast<int>(L.total);
+    configured_smem[cluster][dev] = static_cast<int>(L.total);
+  }
+  if (sm_count[dev] == 0) {
+    e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.blockDim = dim3(kQuantThreads);
   cfg.dynamicSmemBytes = L.total;
   cfg.stream = stream;
-  if (p.C > 1) {
+  if (cluster) {
     if (p.C > 8 && !configured_cluster[dev]) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e != cudaSuccess) return e;
@@ -341,15 +432,18 @@ cudaError_t launch_typed(const QuantParams& p, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   } else {
-    cfg.gridDim = dim3((p.units + p.G - 1) / p.G);
+    // persistent: enough CTAs to fill every SM at the residency shared memory allows
+    const int groups = (p.units + p.G - 1) / p.G;
+    const int per_sm = max(1, min(8, static_cast<int>((227u * 1024u) / (L.total + 1024u))));
+    cfg.gridDim = dim3(min(groups, sm_count[dev] * per_sm));
   }
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 }  // namespace
 
-size_t quant_smem_bytes(int G, int D, int rows_chunk, int rowbytes) {
-  return quant_smem_layout(G, D, rows_chunk, rowbytes).total;
+size_t quant_smem_bytes(int G, int D, int rows_chunk, int rowbytes, int stages) {
+  return quant_smem_layout(G, D, rows_chunk, rowbytes, stages).total;
 }
 
 int quant_threads() { return kQuantThreads; }

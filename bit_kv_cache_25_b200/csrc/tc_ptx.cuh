@@ -28,6 +28,20 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_byte_addr) {
   return d;
 }
 
+// The same physical layout read as an MN-major operand: element (mn, k) at
+// sw128_offset(k, mn, rows_k) is the canonical MN-major 128B-swizzle layout with
+// 64-element MN groups `lbo_bytes` apart (= rows_k * 128) and 8-row K groups
+// 1024 bytes apart. One MMA k-step (16 K rows) starts 2048 bytes further on.
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t smem_byte_addr, uint32_t lbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu);  // start address
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;  // LBO: MN-group stride
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;                  // SBO: K-group (8 rows) stride
+  d |= static_cast<uint64_t>(1u) << 46;                          // descriptor version (sm100)
+  d |= static_cast<uint64_t>(2u) << 61;                          // layout: SWIZZLE_128B
+  return d;
+}
+
 // Byte offset of 16-bit element (row, k) inside a K-major SW128 tile of `rows`
 // rows (rows % 8 == 0), k counted over all slabs.
 __host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int k, int rows) {
@@ -39,10 +53,11 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int k, int ro
 }
 
 // Instruction descriptor: kind::f16 with f16 A and B, f32 accumulator,
-// both operands K-major, M x N.
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+// A K-major, B K-major (b_mn_major = false) or MN-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major = false) {
   return (1u << 4)                                   // D format: F32
          | (0u << 7) | (0u << 10)                    // A, B format: F16
+         | ((b_mn_major ? 1u : 0u) << 16)            // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
@@ -101,6 +116,35 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ---- packed fp32x2 arithmetic (sm_100a), each lane correctly rounded
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ float f2lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// 2^x, hardware approximation (MUFU.EX2), subnormal results flushed to zero
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// {lo, hi} fp32 -> fp16x2 (lo in the low half), round to nearest even
+__device__ __forceinline__ uint32_t cvt_half2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");

@@ -100,9 +100,11 @@ bool plan_quant(vq::QuantParams& p) {
     p.C = 1;
     p.wr_chunk = p.W;
     p.rows_chunk = p.n;
+    // several small slabs per CTA step, so a step has about one task per thread
     const int tasks = p.W * p.vecs_per_row;
     int G = vq::quant_threads() / tasks;
     if (G < 1) G = 1;
+    if (G > 8) G = 8;
     while (G > 1 && int64_t(G) * slab > kSingle) --G;
     if (G > p.units) G = p.units;
     p.G = G;

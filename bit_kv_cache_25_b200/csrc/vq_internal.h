@@ -33,7 +33,7 @@ struct QuantParams {
   int rows_chunk;       // staged token rows per unit per CTA (n when C == 1)
 };
 
-size_t quant_smem_bytes(int G, int D, int rows_chunk, int rowbytes);
+size_t quant_smem_bytes(int G, int D, int rows_chunk, int rowbytes, int stages);
 int quant_threads();
 cudaError_t launch_quant_pack(const QuantParams& p, cudaStream_t stream);
 
