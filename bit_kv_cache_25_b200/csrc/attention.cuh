@@ -154,10 +154,14 @@ constexpr int kTcMinQueries = 16;
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
   if (p.n_q >= kTcMinQueries) {
     if (p.B * p.H > 65535) return cudaErrorInvalidConfiguration;
+    // head_dim 64: the single-warpgroup pipeline (110 KB shared memory, two
+    // CTAs per SM) wins on the VAR shapes, whose per-CTA work is short;
+    // head_dim 128: the warp-specialized kernel keeps the tensor cores busier
+    // on the long Infinity-shaped blocks.
     if (p.bits == 4 && p.D == 64) return launch_attention_tc<4, 64>(p, stream);
-    if (p.bits == 4 && p.D == 128) return launch_attention_tc<4, 128>(p, stream);
+    if (p.bits == 4 && p.D == 128) return launch_attention_ws<4, 128>(p, stream);
     if (p.bits == 3 && p.D == 64) return launch_attention_tc<3, 64>(p, stream);
-    if (p.bits == 3 && p.D == 128) return launch_attention_tc<3, 128>(p, stream);
+    if (p.bits == 3 && p.D == 128) return launch_attention_ws<3, 128>(p, stream);
   }
   if (p.bits == 4 && p.D == 64) return launch_attention_small<4, 64>(p, stream);
   if (p.bits == 4 && p.D == 128) return launch_attention_small<4, 128>(p, stream);

@@ -57,8 +57,8 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x
 // `stages` staging buffers of G slabs of rows_chunk rows each.
 __host__ __device__ inline QuantSmem quant_smem_layout(int G, int D, int rows_chunk, int rowbytes, int stages) {
   QuantSmem L;
-  L.bar = 0;
-  L.mnk = 16;
+  L.bar = 0;    // up to 4 mbarriers
+  L.mnk = 32;
   L.mxk = L.mnk + 4u * G * D;
   L.mn = L.mxk + 4u * G * D;
   L.inv = L.mn + 4u * G * D;
@@ -273,14 +273,15 @@ __device__ __forceinline__ void quant_pass2(const QuantParams& p, const QuantSte
 }
 
 // Blocks whose (tensor, b, h) slab fits one CTA: a persistent loop over groups
-// of G units with a two-stage bulk-copy pipeline, so the next group's slabs
-// are in flight while this group is reduced, encoded and stored.
+// of G units with a p.stages-deep bulk-copy pipeline, so the next groups'
+// slabs are in flight while this group is reduced, encoded and stored.
 template <class Vec, int BITS>
 __global__ void __launch_bounds__(kQuantThreads) quant_pack_stream_kernel(const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int D = p.D;
   const int rowbytes = p.vecs_per_row * 16;
-  const QuantSmem L = quant_smem_layout(p.G, D, p.rows_chunk, rowbytes, 2);
+  const int NST = p.stages;
+  const QuantSmem L = quant_smem_layout(p.G, D, p.rows_chunk, rowbytes, NST);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);
   int32_t* mnk = reinterpret_cast<int32_t*>(smem + L.mnk);
   int32_t* mxk = reinterpret_cast<int32_t*>(smem + L.mxk);
@@ -301,26 +302,32 @@ __global__ void __launch_bounds__(kQuantThreads) quant_pack_stream_kernel(const 
   };
 
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (int i = 0; i < NST; ++i) mbar_init(&bar[i], 1);
     fence_barrier_init();
   }
   __syncthreads();
-  int grp = blockIdx.x;
-  if (grp < groups) quant_issue_copies(p, step_of(grp), smem + L.stage, &bar[0], rowbytes);
+  // prologue: the first NST-1 groups of this CTA
+  for (int k = 0; k < NST - 1; ++k) {
+    const int grp = blockIdx.x + k * gridDim.x;
+    if (grp < groups) quant_issue_copies(p, step_of(grp), smem + L.stage + k * L.stage_bytes, &bar[k], rowbytes);
+  }
   bool ok = true;
-  for (int it = 0; grp < groups; ++it, grp += gridDim.x) {
+  int it = 0;
+  for (int grp = blockIdx.x; grp < groups; ++it, grp += gridDim.x) {
     const QuantStep st = step_of(grp);
-    const int stg = it & 1;
-    // prefetch the next group into the other stage (its last reader finished
-    // at the barrier that ended the previous iteration)
-    const int nxt = grp + gridDim.x;
-    if (nxt < groups) quant_issue_copies(p, step_of(nxt), smem + L.stage + (stg ^ 1) * L.stage_bytes, &bar[stg ^ 1], rowbytes);
+    const int stg = it % NST;
+    // keep NST-1 groups in flight: the stage refilled here was last read by
+    // the previous iteration, which ended with a barrier
+    const int ahead = grp + (NST - 1) * gridDim.x;
+    if (ahead < groups) {
+      const int s2 = (it + NST - 1) % NST;
+      quant_issue_copies(p, step_of(ahead), smem + L.stage + s2 * L.stage_bytes, &bar[s2], rowbytes);
+    }
     for (int i = tid; i < st.units * D; i += blockDim.x) {
       mnk[i] = INT32_MAX;
       mxk[i] = INT32_MIN;
     }
-    ok = __syncthreads_and(mbar_wait_bounded(&bar[stg], (it >> 1) & 1));
+    ok = __syncthreads_and(mbar_wait_bounded(&bar[stg], (it / NST) & 1));
     if (!ok) break;
     const unsigned char* stage = smem + L.stage + stg * L.stage_bytes;
     quant_pass1<Vec, BITS>(p, st, stage, mnk, mxk);
@@ -328,7 +335,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_pack_stream_kernel(const 
     for (int i = tid; i < st.units * D; i += blockDim.x) quant_finalize<BITS>(p, st, mnk[i], mxk[i], i, s_mn, s_inv, true);
     __syncthreads();
     quant_pass2<Vec, BITS>(p, st, stage, s_mn, s_inv);
-    fence_proxy_async_smem();  // generic reads of this stage before the next bulk copy overwrites it
+    fence_proxy_async_smem();  // generic reads of this stage before a later bulk copy overwrites it
     __syncthreads();
   }
 }
@@ -394,7 +401,7 @@ cudaError_t launch_typed(const QuantParams& p, cudaStream_t stream) {
   const bool cluster = p.C > 1;
   auto kern = cluster ? quant_pack_cluster_kernel<Vec, BITS> : quant_pack_stream_kernel<Vec, BITS>;
   const int rowbytes = p.vecs_per_row * 16;
-  const QuantSmem L = quant_smem_layout(cluster ? 1 : p.G, p.D, p.rows_chunk, rowbytes, cluster ? 1 : 2);
+  const QuantSmem L = quant_smem_layout(cluster ? 1 : p.G, p.D, p.rows_chunk, rowbytes, cluster ? 1 : p.stages);
   // Function attributes are set once per device and size, outside any stream
   // work, so launches can be captured into CUDA graphs.
   static int configured_smem[2][kMaxDevices] = {};

@@ -31,6 +31,7 @@ struct QuantParams {
   int C;                // CTAs per unit (cluster size); G == 1 when C > 1
   int wr_chunk;         // word-rows per CTA
   int rows_chunk;       // staged token rows per unit per CTA (n when C == 1)
+  int stages;           // staging buffers of the single-CTA (C == 1) pipeline
 };
 
 size_t quant_smem_bytes(int G, int D, int rows_chunk, int rowbytes, int stages);
