@@ -145,11 +145,19 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest value over all ranks (device timings are reduced with MAX)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank_step: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput: every rank decodes its own batch (replicas), so the
+    job processes world x tokens per step in the slowest rank's step time."""
+    return world * tokens_per_rank_step / (ms_per_step_max / 1e3)
 
 
 # ------------------------------------------------------------------ CPU oracle sample
@@ -366,7 +374,7 @@ def run_ours(args):
     n_launch = 2 * L * S
     ms_step = elapsed_ms / args.steps
     tokens_step = B * N * L
-    value = world * tokens_step / (ms_step / 1e3)
+    value = weak_scaling_value(tokens_step, world, ms_step)
     peaks, peak_src = load_peaks()
     hbm = peaks["hbm_gbs"]
     tc = peaks["bf16_tflops_sustained"]

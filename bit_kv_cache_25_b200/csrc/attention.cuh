@@ -159,9 +159,9 @@ cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
     // head_dim 128: the warp-specialized kernel keeps the tensor cores busier
     // on the long Infinity-shaped blocks.
     if (p.bits == 4 && p.D == 64) return launch_attention_tc<4, 64>(p, stream);
-    if (p.bits == 4 && p.D == 128) return launch_attention_ws<4, 128>(p, stream);
+    if (p.bits == 4 && p.D == 128) return launch_attention_ws<4, 128, 1>(p, stream);
     if (p.bits == 3 && p.D == 64) return launch_attention_tc<3, 64>(p, stream);
-    if (p.bits == 3 && p.D == 128) return launch_attention_ws<3, 128>(p, stream);
+    if (p.bits == 3 && p.D == 128) return launch_attention_ws<3, 128, 1>(p, stream);
   }
   if (p.bits == 4 && p.D == 64) return launch_attention_small<4, 64>(p, stream);
   if (p.bits == 4 && p.D == 128) return launch_attention_small<4, 128>(p, stream);

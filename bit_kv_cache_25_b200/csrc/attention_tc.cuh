@@ -131,6 +131,9 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
   const int q0 = blockIdx.x * 128;
   const int row = tid;
   const bool row_valid = (q0 + row) < p.n_q;
+  // warps whose 32 rows are all past n_q skip the per-row work (q', softmax,
+  // fold, epilogue); their P and U rows are never read back
+  const bool warp_active = __any_sync(0xffffffffu, row_valid);
   const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
 
   // zero the K/V operand buffers once: rows past a tile's valid keys are read by
@@ -322,8 +325,8 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
 
   load_meta(0);
   __syncthreads();
-  float bias_q[2], up_q[2];
-  build_q(0, bias_q[0], up_q[0]);
+  float bias_q[2] = {0.0f, 0.0f}, up_q[2] = {1.0f, 1.0f};
+  if (warp_active) build_q(0, bias_q[0], up_q[0]);
   bool ok = __syncthreads_and(mbar_wait_bounded(&bar_stg[0], 0));
   if (ok) unpack(cur, 0, 0);
   fence_proxy_async_smem();
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
     // (4) fold the previous block into O when tile g starts a new block (PV(g-1),
     // the last PV of that block, is complete); this must precede (5), which may
     // reuse the previous block's meta buffer
-    if (first_of_block && prev_kb >= 0) {
+    if (first_of_block && prev_kb >= 0 && warp_active) {
       const float* meta = reinterpret_cast<const float*>(sm + C::META) + (prev_kb & 1) * 4 * D;
 #pragma unroll 1
       for (int c16 = 0; c16 < D; c16 += 16) {
@@ -392,7 +395,7 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
       __syncthreads();  // every thread's fold has finished reading the meta buffer reused here
       load_meta(nxt.kb);
       __syncthreads();
-      build_q(nxt.kb, bias_q[nxt.kb & 1], up_q[nxt.kb & 1]);
+      if (warp_active) build_q(nxt.kb, bias_q[nxt.kb & 1], up_q[nxt.kb & 1]);
     }
     fence_proxy_async_smem();
     tc::fence_before_sync();
@@ -410,6 +413,7 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
     // TMEM: p = 2^(S * up * log2 e + (bias - m) * log2 e), one FFMA and one EX2;
     // hi = p with its low 13 mantissa bits cleared (exact in fp16 for
     // p >= 2^-14), lo = p - hi (exact); both rounded to fp16.
+    if (warp_active) {
     const float bias = bias_q[cur.kb & 1];
     const float up = up_q[cur.kb & 1];
     const uint32_t t_s = tmem + lane_off + C::COL_S + (g & 1) * 64;
@@ -510,6 +514,7 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
       }
     }
     rs += tc::f2lo(rs2) + tc::f2hi(rs2);
+    }  // warp_active
     fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
@@ -525,7 +530,7 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
     ok = __syncthreads_and(mbar_wait_bounded(&bar_pv[(g - 1) & 1], ((g - 1) >> 1) & 1));
     tc::fence_after_sync();
   }
-  if (ok) {
+  if (ok && warp_active) {
     const float* meta = reinterpret_cast<const float*>(sm + C::META) + (prev_kb & 1) * 4 * D;
     const float inv = 1.0f / (l_tot + rs);
     const int64_t obase = b * p.o_sb + h * p.o_sh + static_cast<int64_t>(q0 + row) * p.o_st;

@@ -10,12 +10,15 @@
 //     every tcgen05.mma: QK^T of tile g into S[g % 2], then PV of tile g-1;
 //   unpack warpgroup (128 threads): packed words -> fp16 K and V code tiles
 //     (2-buffer ring), the same [64 keys][D] 128B-swizzled layout for both;
-//   softmax warpgroup (128 threads, one query row each): reads S from TMEM,
-//     writes P hi/lo (2-buffer ring), rebuilds q' once per key block, folds
-//     each finished block's U into O and writes the output.
+//   softmax warpgroups (NQT of them, 128 threads each, one query row per
+//     thread): read S from TMEM, write P hi/lo, rebuild q' once per key block,
+//     fold each finished block's U into O and write the output.
+// With NQT = 2 (head_dim 64) a CTA owns 256 queries: both query tiles share
+// every unpacked K/V tile, and the two softmax warpgroups take turns on the
+// tensor cores (one computes while the other's MMAs run).
 // Barriers (count): stg_full (tx bytes), stg_empty (128), kv_full (128),
-// kv_empty (MMA commit), q_full (128), s_full (commit), s_empty (128),
-// p_full (128), p_empty (commit; also "PV of that tile is done").
+// kv_empty (MMA commit), and per query tile: q_full (128), s_full (commit),
+// s_empty (128), p_full (128), p_empty (commit; also "PV of that tile is done").
 #pragma once
 
 #include <cuda_fp16.h>
@@ -30,10 +33,11 @@
 namespace vq {
 namespace {
 
-constexpr int kWsThreads = 288;  // softmax WG (0-127), unpack WG (128-255), control warp (256-287)
-
-template <int BITS, int D>
+template <int BITS, int D, int NQT>
 struct WsCfg {
+  static constexpr int THREADS = NQT * 128 + 128 + 32;    // softmax WGs, unpack WG, control warp
+  static constexpr int UNPACK_T0 = NQT * 128;             // first unpack thread
+  static constexpr int CTRL_WARP = NQT * 4 + 4;
   static constexpr int CPW = 32 / BITS;
   static constexpr uint32_t MASK = (1u << BITS) - 1u;
   static constexpr int KT = 64;                           // keys per tile
@@ -41,31 +45,34 @@ struct WsCfg {
   static constexpr int STAGE_WORDS = MAXW * D;            // per tensor
   static constexpr int NSTG = (D == 64) ? 3 : 2;          // packed-word stages
   static constexpr int NKV = 2;                           // fp16 K/V tile buffers
+  static constexpr int NPB = (NQT == 1) ? 2 : 1;          // P buffers per query tile
   // shared memory (byte offsets from a 1024-aligned base)
-  static constexpr int Q_HI = 0;                          // [128][D] fp16
-  static constexpr int Q_LO = Q_HI + 128 * D * 2;
-  static constexpr int KV0 = Q_LO + 128 * D * 2;          // NKV x {K [64][D], V [64][D]}
+  static constexpr int Q_SZ = 128 * D * 2;                // one of hi / lo
+  static constexpr int Q0 = 0;                            // NQT x {q' hi [128][D], q' lo [128][D]}
+  static constexpr int KV0 = Q0 + NQT * 2 * Q_SZ;         // NKV x {K [64][D], V [64][D]}
   static constexpr int TILE_SZ = KT * D * 2;
   static constexpr int KV_SZ = 2 * TILE_SZ;
-  static constexpr int P0 = KV0 + NKV * KV_SZ;            // 2 x {P hi [128][64], P lo [128][64]}
+  static constexpr int P0 = KV0 + NKV * KV_SZ;            // NQT x NPB x {P hi [128][64], P lo [128][64]}
   static constexpr int PT_SZ = 128 * KT * 2;
   static constexpr int P_SZ = 2 * PT_SZ;
-  static constexpr int STG0 = P0 + 2 * P_SZ;
+  static constexpr int STG0 = P0 + NQT * NPB * P_SZ;
   static constexpr int STG_SZ = 2 * STAGE_WORDS * 4;
-  static constexpr int META = STG0 + NSTG * STG_SZ;       // 3 x [4][D] fp32: sk, zk, sv, zv
-  static constexpr int BARS = META + 3 * 4 * D * 4;
-  static constexpr int NBARS = 2 * NSTG + 2 * NKV + 1 + 2 * 2 + 2 * 2;
+  static constexpr int META = STG0 + NSTG * STG_SZ;       // NQT x 3 x [4][D] fp32: sk, zk, sv, zv
+  static constexpr int BARS = META + NQT * 3 * 4 * D * 4;
+  static constexpr int NBARS = 2 * NSTG + 2 * NKV + NQT * (1 + 2 + 2 + 2 * NPB);
   static constexpr int TMEM_SLOT = BARS + NBARS * 8;
   static constexpr int SMEM = TMEM_SLOT + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;
   static_assert(KV0 % 1024 == 0 && TILE_SZ % 1024 == 0 && P0 % 1024 == 0 && PT_SZ % 1024 == 0, "tile alignment");
   static_assert(STG0 % 128 == 0 && STG_SZ % 128 == 0, "stage alignment");
   static_assert(SMEM_ALLOC <= 232448, "shared memory");
-  // tensor memory columns
-  static constexpr int COL_S = 0;                         // 2 x 64
-  static constexpr int COL_U = 128;                       // D
-  static constexpr int COL_O = 128 + D;                   // D
-  static constexpr int TMEM_COLS = (128 + 2 * D <= 256) ? 256 : 512;
+  // tensor memory columns: per query tile qt, S[2] at qt*128, U and O after all S
+  static constexpr int COL_S = 0;
+  static constexpr int COL_U = NQT * 128;                 // + qt * D
+  static constexpr int COL_O = NQT * 128 + NQT * D;       // + qt * D
+  static constexpr int TMEM_USED = NQT * (128 + 2 * D);
+  static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
+  static_assert(TMEM_USED <= 512, "tensor memory");
 };
 
 // Bounded wait that works for every role: on timeout the device error word is
@@ -85,11 +92,13 @@ __device__ __forceinline__ void ws_next(const AttnParams& p, WsTile& t) {
   }
 }
 
-template <int BITS, int D>
-__global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __grid_constant__ AttnParams p) {
-  using C = WsCfg<BITS, D>;
+template <int BITS, int D, int NQT>
+__global__ void __launch_bounds__(WsCfg<BITS, D, NQT>::THREADS, 1)
+    attention_ws_kernel(const __grid_constant__ AttnParams p) {
+  using C = WsCfg<BITS, D, NQT>;
   constexpr int CPW = C::CPW;
   constexpr int KT = C::KT;
+  constexpr int NPB = C::NPB;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -99,11 +108,13 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
   uint64_t* stg_empty = stg_full + C::NSTG;
   uint64_t* kv_full = stg_empty + C::NSTG;
   uint64_t* kv_empty = kv_full + C::NKV;
-  uint64_t* q_full = kv_empty + C::NKV;
-  uint64_t* s_full = q_full + 1;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* p_empty = p_full + 2;
+  uint64_t* qbars = kv_empty + C::NKV;  // per query tile: q_full, s_full[2], s_empty[2], p_full[NPB], p_empty[NPB]
+  constexpr int QB = 1 + 2 + 2 + 2 * NPB;
+  auto q_full = [&](int qt) { return qbars + qt * QB; };
+  auto s_full = [&](int qt, int i) { return qbars + qt * QB + 1 + i; };
+  auto s_empty = [&](int qt, int i) { return qbars + qt * QB + 3 + i; };
+  auto p_full = [&](int qt, int i) { return qbars + qt * QB + 5 + i; };
+  auto p_empty = [&](int qt, int i) { return qbars + qt * QB + 5 + NPB + i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::TMEM_SLOT);
 
   const int tid = threadIdx.x;
@@ -111,7 +122,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
   const int bh = blockIdx.y;
   const int b = bh / p.H;
   const int h = bh - b * p.H;
-  const int q0 = blockIdx.x * 128;
+  const int cta_q0 = blockIdx.x * 128 * NQT;
+  // query tiles of this CTA that hold at least one query
+  const int nqt = min(NQT, (p.n_q - cta_q0 + 127) / 128);
   const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
 
   // ---- set-up: TMEM (warp 0), barriers (thread 0), zeroed K/V tiles (unpack WG)
@@ -128,19 +141,23 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
       mbar_init(&kv_full[i], 128);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(q_full, 128);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
-      mbar_init(&p_full[i], 128);
-      mbar_init(&p_empty[i], 1);
+    for (int qt = 0; qt < NQT; ++qt) {
+      mbar_init(q_full(qt), 128);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(s_full(qt, i), 1);
+        mbar_init(s_empty(qt, i), 128);
+      }
+      for (int i = 0; i < NPB; ++i) {
+        mbar_init(p_full(qt, i), 128);
+        mbar_init(p_empty(qt, i), 1);
+      }
     }
     fence_barrier_init();
   }
-  if (tid >= 128 && tid < 256) {
+  if (tid >= C::UNPACK_T0 && tid < C::UNPACK_T0 + 128) {
     // rows past a tile's valid keys are read by the MMAs (times zero
     // probabilities) and must hold finite values
-    for (int i = C::KV0 + (tid - 128) * 16; i < C::P0; i += 128 * 16) tc::sts128(sbase + i, 0u, 0u, 0u, 0u);
+    for (int i = C::KV0 + (tid - C::UNPACK_T0) * 16; i < C::P0; i += 128 * 16) tc::sts128(sbase + i, 0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
   tc::fence_before_sync();
@@ -148,7 +165,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == C::CTRL_WARP) {
     // =========================================================== control warp
     if ((tid & 31) == 0) {
       auto issue_copy = [&](const WsTile& t, int stage) {
@@ -164,13 +181,24 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
       };
       const uint32_t idesc_pv = tc::idesc_f16_f32(128, D, /*b_mn_major=*/true);
       constexpr uint32_t kLbo = KT * 128;
+      auto issue_pv = [&](int qt, int gp, int nk16, bool first) {
+        const uint32_t vbuf = sbase + C::KV0 + (gp % C::NKV) * C::KV_SZ + C::TILE_SZ;
+        const uint32_t pb = sbase + C::P0 + (qt * NPB + gp % NPB) * C::P_SZ;
+        const uint32_t tu = tmem + C::COL_U + qt * D;
+        for (int kk = 0; kk < nk16 / 16; ++kk)
+          tc::mma_f16_ss(tu, tc::sw128_desc(pb + kk * 32), tc::sw128_desc_mn(vbuf + kk * 2048, kLbo), idesc_pv,
+                         (first && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < nk16 / 16; ++kk)
+          tc::mma_f16_ss(tu, tc::sw128_desc(pb + C::PT_SZ + kk * 32), tc::sw128_desc_mn(vbuf + kk * 2048, kLbo),
+                         idesc_pv, 1u);
+        tc::commit(p_empty(qt, gp % NPB));
+      };
       // prefetch the first NSTG tiles
       WsTile cp{0, 0};
-      int ncopied = 0;
-      for (; ncopied < C::NSTG && cp.kb <= p.s; ++ncopied, ws_next(p, cp)) issue_copy(cp, ncopied);
+      for (int k = 0; k < C::NSTG && cp.kb <= p.s; ++k, ws_next(p, cp)) issue_copy(cp, k);
 
       bool ok = true;
-      WsTile t{0, 0}, prev{0, 0};
+      WsTile t{0, 0};
       int prev_nk16 = 0;
       bool prev_first = true;
       int g = 0;
@@ -185,47 +213,42 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
           issue_copy(cp, st);
           ws_next(p, cp);
         }
-        // ---- QK(g) -> S[g % 2]
+        // ---- QK(g) of every query tile -> S[qt][g % 2]
         if (!(ok = ws_wait(&kv_full[g % C::NKV], (g / C::NKV) & 1))) break;
-        if (first && !(ok = ws_wait(q_full, t.kb & 1))) break;
-        if (!(ok = ws_wait(&s_empty[g & 1], ((g >> 1) & 1) ^ 1))) break;
-        tc::fence_after_sync();
-        {
-          const uint32_t idesc = tc::idesc_f16_f32(128, nk16);
-          const uint32_t kbuf = sbase + C::KV0 + (g % C::NKV) * C::KV_SZ;
+        const uint32_t idesc = tc::idesc_f16_f32(128, nk16);
+        const uint32_t kbuf = sbase + C::KV0 + (g % C::NKV) * C::KV_SZ;
+        for (int qt = 0; qt < nqt && ok; ++qt) {
+          if (first && !(ok = ws_wait(q_full(qt), t.kb & 1))) break;
+          if (!(ok = ws_wait(s_empty(qt, g & 1), ((g >> 1) & 1) ^ 1))) break;
+          tc::fence_after_sync();
+          const uint32_t qb = sbase + C::Q0 + qt * 2 * C::Q_SZ;
+          const uint32_t ts = tmem + C::COL_S + qt * 128 + (g & 1) * 64;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t koff = (kk & 3) * 32;
-            tc::mma_f16_ss(tmem + C::COL_S + (g & 1) * 64,
-                           tc::sw128_desc(sbase + C::Q_HI + (kk >> 2) * 128 * 128 + koff),
+            tc::mma_f16_ss(ts, tc::sw128_desc(qb + (kk >> 2) * 128 * 128 + koff),
                            tc::sw128_desc(kbuf + (kk >> 2) * KT * 128 + koff), idesc, kk > 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t koff = (kk & 3) * 32;
-            tc::mma_f16_ss(tmem + C::COL_S + (g & 1) * 64,
-                           tc::sw128_desc(sbase + C::Q_LO + (kk >> 2) * 128 * 128 + koff),
+            tc::mma_f16_ss(ts, tc::sw128_desc(qb + C::Q_SZ + (kk >> 2) * 128 * 128 + koff),
                            tc::sw128_desc(kbuf + (kk >> 2) * KT * 128 + koff), idesc, 1u);
           }
-          tc::commit(&s_full[g & 1]);
+          tc::commit(s_full(qt, g & 1));
         }
-        // ---- PV(g-1) -> U
+        if (!ok) break;
+        // ---- PV(g-1) of every query tile -> U[qt]
         if (g >= 1) {
           const int gp = g - 1;
-          if (!(ok = ws_wait(&p_full[gp & 1], (gp >> 1) & 1))) break;
-          tc::fence_after_sync();
-          const uint32_t vbuf = sbase + C::KV0 + (gp % C::NKV) * C::KV_SZ + C::TILE_SZ;
-          const uint32_t pb = sbase + C::P0 + (gp & 1) * C::P_SZ;
-          for (int kk = 0; kk < prev_nk16 / 16; ++kk)
-            tc::mma_f16_ss(tmem + C::COL_U, tc::sw128_desc(pb + kk * 32), tc::sw128_desc_mn(vbuf + kk * 2048, kLbo),
-                           idesc_pv, (prev_first && kk == 0) ? 0u : 1u);
-          for (int kk = 0; kk < prev_nk16 / 16; ++kk)
-            tc::mma_f16_ss(tmem + C::COL_U, tc::sw128_desc(pb + C::PT_SZ + kk * 32),
-                           tc::sw128_desc_mn(vbuf + kk * 2048, kLbo), idesc_pv, 1u);
-          tc::commit(&p_empty[gp & 1]);
+          for (int qt = 0; qt < nqt && ok; ++qt) {
+            if (!(ok = ws_wait(p_full(qt, gp % NPB), (gp / NPB) & 1))) break;
+            tc::fence_after_sync();
+            issue_pv(qt, gp, prev_nk16, prev_first);
+          }
+          if (!ok) break;
           tc::commit(&kv_empty[gp % C::NKV]);
         }
-        prev = t;
         prev_nk16 = nk16;
         prev_first = first;
         ws_next(p, t);
@@ -233,25 +256,17 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
       // ---- PV of the last tile
       if (ok && g >= 1) {
         const int gp = g - 1;
-        if (ws_wait(&p_full[gp & 1], (gp >> 1) & 1)) {
+        for (int qt = 0; qt < nqt && ok; ++qt) {
+          if (!(ok = ws_wait(p_full(qt, gp % NPB), (gp / NPB) & 1))) break;
           tc::fence_after_sync();
-          const uint32_t vbuf = sbase + C::KV0 + (gp % C::NKV) * C::KV_SZ + C::TILE_SZ;
-          const uint32_t pb = sbase + C::P0 + (gp & 1) * C::P_SZ;
-          for (int kk = 0; kk < prev_nk16 / 16; ++kk)
-            tc::mma_f16_ss(tmem + C::COL_U, tc::sw128_desc(pb + kk * 32), tc::sw128_desc_mn(vbuf + kk * 2048, kLbo),
-                           idesc_pv, (prev_first && kk == 0) ? 0u : 1u);
-          for (int kk = 0; kk < prev_nk16 / 16; ++kk)
-            tc::mma_f16_ss(tmem + C::COL_U, tc::sw128_desc(pb + C::PT_SZ + kk * 32),
-                           tc::sw128_desc_mn(vbuf + kk * 2048, kLbo), idesc_pv, 1u);
-          tc::commit(&p_empty[gp & 1]);
-          tc::commit(&kv_empty[gp % C::NKV]);
+          issue_pv(qt, gp, prev_nk16, prev_first);
         }
+        if (ok) tc::commit(&kv_empty[gp % C::NKV]);
       }
-      (void)prev;
     }
-  } else if (tid >= 128) {
+  } else if (tid >= C::UNPACK_T0) {
     // =========================================================== unpack warpgroup
-    const int ut = tid - 128;
+    const int ut = tid - C::UNPACK_T0;
     WsTile t{0, 0};
     for (int g = 0; t.kb <= p.s; ++g, ws_next(p, t)) {
       const int st = g % C::NSTG;
@@ -296,13 +311,22 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
       mbar_arrive(&stg_empty[st]);
       mbar_arrive(&kv_full[kvb]);
     }
-  } else {
-    // =========================================================== softmax warpgroup
-    const int row = tid;
+  } else if ((tid >> 7) < nqt) {
+    // =========================================================== softmax warpgroup qt
+    const int qt = tid >> 7;
+    const int row = tid & 127;
+    const int q0 = cta_q0 + qt * 128;
     const bool row_valid = (q0 + row) < p.n_q;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t col_u = C::COL_U + qt * D;
+    const uint32_t col_o = C::COL_O + qt * D;
+    const uint32_t qb = sbase + C::Q0 + qt * 2 * C::Q_SZ;
     const uint16_t* qrow = p.q + b * p.q_sb + h * p.q_sh + static_cast<int64_t>(q0 + row) * p.q_st;
-    auto meta_of = [&](int kb) { return reinterpret_cast<float*>(sm + C::META) + (kb % 3) * 4 * D; };
+    // each query tile keeps its own three meta buffers (blocks kb % 3): the
+    // tiles of a CTA may be up to two key tiles apart
+    auto meta_of = [&](int kb) { return reinterpret_cast<float*>(sm + C::META) + (qt * 3 + kb % 3) * 4 * D; };
+    // named barrier among this warpgroup's 128 threads only
+    auto wg_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(1 + qt) : "memory"); };
     auto load_meta = [&](int kb) {
       float* meta = meta_of(kb);
       for (int c = row; c < D; c += 128) {
@@ -313,8 +337,6 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
         meta[3 * D + c] = p.zero_v[mo];
       }
     };
-    // named barrier among the 128 softmax threads only
-    auto sm_sync = [&]() { asm volatile("bar.sync 1, 128;" ::: "memory"); };
     // q' = sigma * q * sk of block kb, scaled by 2^-e, split into fp16 hi/lo
     auto build_q = [&](int kb, float& bias_out, float& up_out) {
       const float* meta = meta_of(kb);
@@ -354,8 +376,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
           lo[k2] = pack_half2(x[0] - hf.x, x[1] - hf.y);
         }
         const uint32_t off = tc::sw128_offset(row, c8, 128);
-        tc::sts128(sbase + C::Q_HI + off, hi[0], hi[1], hi[2], hi[3]);
-        tc::sts128(sbase + C::Q_LO + off, lo[0], lo[1], lo[2], lo[3]);
+        tc::sts128(qb + off, hi[0], hi[1], hi[2], hi[3]);
+        tc::sts128(qb + C::Q_SZ + off, lo[0], lo[1], lo[2], lo[3]);
       }
       bias_out = bias;
       up_out = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
@@ -365,8 +387,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
 #pragma unroll 1
       for (int c16 = 0; c16 < D; c16 += 16) {
         uint32_t u[16], o[16];
-        tc::tmem_ld16(tmem + lane_off + C::COL_U + c16, u);
-        if (have_o) tc::tmem_ld16(tmem + lane_off + C::COL_O + c16, o);
+        tc::tmem_ld16(tmem + lane_off + col_u + c16, u);
+        if (have_o) tc::tmem_ld16(tmem + lane_off + col_o + c16, o);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -374,11 +396,11 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
           o[k] = __float_as_uint(
               fmaf(__uint_as_float(u[k]), meta[2 * D + c16 + k], fmaf(rsum, meta[3 * D + c16 + k], base_o)));
         }
-        tc::tmem_st16(tmem + lane_off + C::COL_O + c16, o);
+        tc::tmem_st16(tmem + lane_off + col_o + c16, o);
       }
       tc::tmem_wait_st();
     };
-    auto scale_tmem = [&](int col, float alpha) {
+    auto scale_tmem = [&](uint32_t col, float alpha) {
 #pragma unroll 1
       for (int c16 = 0; c16 < D; c16 += 16) {
         uint32_t r[16];
@@ -393,10 +415,10 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
 
     float bias_q[3], up_q[3];
     load_meta(0);
-    sm_sync();
+    wg_sync();
     build_q(0, bias_q[0], up_q[0]);
     fence_proxy_async_smem();
-    mbar_arrive(q_full);
+    mbar_arrive(q_full(qt));
 
     bool ok = true;
     float m_ref = -INFINITY, l_tot = 0.0f, rs = 0.0f;
@@ -411,19 +433,19 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
       const int nk16 = (nk + 15) & ~15;
       const bool first = (t.t0 == 0);
       const bool last_of_block = (nx.kb != t.kb);
-      if (!(ok = ws_wait(&s_full[g & 1], (g >> 1) & 1))) break;
+      if (!(ok = ws_wait(s_full(qt, g & 1), (g >> 1) & 1))) break;
       tc::fence_after_sync();
       // q' for the next block: QK(g) (the last one reading q') has completed
       if (last_of_block && nx.kb <= p.s) {
         load_meta(nx.kb);
-        sm_sync();
+        wg_sync();
         build_q(nx.kb, bias_q[nx.kb % 3], up_q[nx.kb % 3]);
         fence_proxy_async_smem();
-        mbar_arrive(q_full);
+        mbar_arrive(q_full(qt));
       }
       // fold the previous block once its last PV (tile g-1) is done
       if (first && g >= 1) {
-        if (!(ok = ws_wait(&p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1))) break;
+        if (!(ok = ws_wait(p_empty(qt, (g - 1) % NPB), ((g - 1) / NPB) & 1))) break;
         tc::fence_after_sync();
         fold(last_kb, rs, have_o);
         l_tot += rs;
@@ -431,10 +453,10 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
         have_o = true;
       }
       last_kb = t.kb;
-      // softmax of S[g % 2]
+      // softmax of S[qt][g % 2]
       const float bias = bias_q[t.kb % 3];
       const float up = up_q[t.kb % 3];
-      const uint32_t t_s = tmem + lane_off + C::COL_S + (g & 1) * 64;
+      const uint32_t t_s = tmem + lane_off + C::COL_S + qt * 128 + (g & 1) * 64;
       const bool partial = nk < nk16;
       float smax = -INFINITY;
 #pragma unroll
@@ -465,23 +487,25 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
       }
       rs *= alpha;
       l_tot *= alpha;
+      // PV(g - NPB) has finished reading the P buffer written below; with
+      // NPB == 1 that is PV(g-1), which also makes U safe to rescale
       const bool any_rescale = __any_sync(0xffffffffu, rescale);
-      if (any_rescale && !first) {
-        // U holds this block's earlier tiles; PV(g-1) must be done before rescaling it
-        if (!(ok = ws_wait(&p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1))) break;
+      if ((NPB == 1 || (any_rescale && !first)) && g >= 1) {
+        if (!(ok = ws_wait(p_empty(qt, (g - 1) % NPB), ((g - 1) / NPB) & 1))) break;
         tc::fence_after_sync();
-        scale_tmem(C::COL_U, alpha);
       }
-      if (any_rescale && have_o) scale_tmem(C::COL_O, alpha);
-      // P buffer g % 2 is free once PV(g-2) is done
-      if (g >= 2 && !(ok = ws_wait(&p_empty[g & 1], ((g - 2) >> 1) & 1))) break;
+      if (NPB == 2 && g >= 2) {
+        if (!(ok = ws_wait(p_empty(qt, g % NPB), ((g - 2) / NPB) & 1))) break;
+      }
+      if (any_rescale && !first) scale_tmem(col_u, alpha);
+      if (any_rescale && have_o) scale_tmem(col_o, alpha);
       constexpr float kLog2e = 1.4426950408889634f;
       const uint64_t up2x2 = tc::f2pack(up * kLog2e, up * kLog2e);
       const float c2 = (bias - m_ref) * kLog2e;
       const uint64_t c2x2 = tc::f2pack(c2, c2);
       const uint64_t neg1x2 = tc::f2pack(-1.0f, -1.0f);
       uint64_t rs2 = tc::f2pack(0.0f, 0.0f);
-      const uint32_t pb = sbase + C::P0 + (g & 1) * C::P_SZ;
+      const uint32_t pb = sbase + C::P0 + (qt * NPB + g % NPB) * C::P_SZ;
 #pragma unroll
       for (int c16 = 0; c16 < 64; c16 += 16) {
         if (c16 < nk16) {
@@ -517,15 +541,15 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
         }
       }
       rs += tc::f2lo(rs2) + tc::f2hi(rs2);
-      // S[g % 2] fully read, P[g % 2] written, U/O rescales complete
+      // S[qt][g % 2] fully read, P written, U/O rescales complete
       fence_proxy_async_smem();
       tc::fence_before_sync();
-      mbar_arrive(&s_empty[g & 1]);
-      mbar_arrive(&p_full[g & 1]);
+      mbar_arrive(s_empty(qt, g & 1));
+      mbar_arrive(p_full(qt, g % NPB));
       t = nx;
     }
     // ---- last block: wait for its final PV, fold and write the output
-    if (ok && g >= 1) ok = ws_wait(&p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1);
+    if (ok && g >= 1) ok = ws_wait(p_empty(qt, (g - 1) % NPB), ((g - 1) / NPB) & 1);
     if (ok && g >= 1) {
       tc::fence_after_sync();
       const float* meta = meta_of(last_kb);
@@ -534,8 +558,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
 #pragma unroll 1
       for (int c16 = 0; c16 < D; c16 += 16) {
         uint32_t u[16], o[16];
-        tc::tmem_ld16(tmem + lane_off + C::COL_U + c16, u);
-        if (have_o) tc::tmem_ld16(tmem + lane_off + C::COL_O + c16, o);
+        tc::tmem_ld16(tmem + lane_off + col_u + c16, u);
+        if (have_o) tc::tmem_ld16(tmem + lane_off + col_o + c16, o);
         tc::tmem_wait_ld();
         float v[16];
 #pragma unroll
@@ -575,21 +599,22 @@ __global__ void __launch_bounds__(kWsThreads, 1) attention_ws_kernel(const __gri
   if (warp == 0) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int BITS, int D>
+template <int BITS, int D, int NQT>
 cudaError_t launch_attention_ws(const AttnParams& p, cudaStream_t stream) {
-  using C = WsCfg<BITS, D>;
+  using C = WsCfg<BITS, D, NQT>;
   static bool configured[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(attention_ws_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+    e = cudaFuncSetAttribute(attention_ws_kernel<BITS, D, NQT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  dim3 grid((p.n_q + 127) / 128, p.B * p.H);
-  attention_ws_kernel<BITS, D><<<grid, kWsThreads, C::SMEM_ALLOC, stream>>>(p);
+  dim3 grid((p.n_q + 128 * NQT - 1) / (128 * NQT), p.B * p.H);
+  attention_ws_kernel<BITS, D, NQT><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -157,7 +157,10 @@ __device__ __forceinline__ void quant_issue_copies(const QuantParams& p, const Q
 }
 
 // Pass 1: per-task min/max over the task's cpw rows, merged into the
-// per-(unit, channel) key slots with shared-memory atomics.
+// per-(unit, channel) key slots. When a whole warp works on one unit, the
+// lanes that share a channel vector (lane % V) first combine their keys with
+// shuffles and only V lanes issue shared-memory atomics; otherwise every lane
+// issues its own. Min and max are idempotent, so any merge order is exact.
 template <class Vec, int BITS>
 __device__ __forceinline__ void quant_pass1(const QuantParams& p, const QuantStep& st, const unsigned char* stage,
                                             int32_t* mnk, int32_t* mxk) {
@@ -167,23 +170,61 @@ __device__ __forceinline__ void quant_pass1(const QuantParams& p, const QuantSte
   const int rowbytes = V * 16;
   const int D = p.D;
   const int tpu = st.wrs * V;
-  for (int task = threadIdx.x; task < st.units * tpu; task += blockDim.x) {
-    const int g = task / tpu;
+  const int ntask = st.units * tpu;
+  const int lane = threadIdx.x & 31;
+  const int wbase = threadIdx.x & ~31;
+  for (int base = 0; base < ntask; base += blockDim.x) {
+    const int task = base + threadIdx.x;
+    const bool valid = task < ntask;
+    const int g = valid ? task / tpu : 0;
     const int r = task - g * tpu;
     const int wl = r / V;
     const int j = r - wl * V;
-    const int tl0 = wl * CPW;
-    const int nvalid = min(CPW, st.rows - tl0);
-    const unsigned char* src = stage + (static_cast<size_t>(g) * p.rows_chunk + tl0) * rowbytes + j * 16;
-    uint32_t mn[4], mx[4];
-    Vec::minmax_init(mn, mx, lds128(src));
+    int32_t kmn[CH], kmx[CH];
+    if (valid) {
+      const int tl0 = wl * CPW;
+      const int nvalid = min(CPW, st.rows - tl0);
+      const unsigned char* src = stage + (static_cast<size_t>(g) * p.rows_chunk + tl0) * rowbytes + j * 16;
+      uint32_t mn[4], mx[4];
+      Vec::minmax_init(mn, mx, lds128(src));
 #pragma unroll
-    for (int i = 1; i < CPW; ++i)
-      if (i < nvalid) Vec::minmax_acc(mn, mx, lds128(src + i * rowbytes));
+      for (int i = 1; i < CPW; ++i)
+        if (i < nvalid) Vec::minmax_acc(mn, mx, lds128(src + i * rowbytes));
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
-      atomicMin(&mnk[g * D + j * CH + c], float_key(Vec::ch(mn, c)));
-      atomicMax(&mxk[g * D + j * CH + c], float_key(Vec::ch(mx, c)));
+      for (int c = 0; c < CH; ++c) {
+        kmn[c] = float_key(Vec::ch(mn, c));
+        kmx[c] = float_key(Vec::ch(mx, c));
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        kmn[c] = INT32_MAX;
+        kmx[c] = INT32_MIN;
+      }
+    }
+    const int t_first = base + wbase;
+    const bool uniform = (t_first + 31 < ntask) && (t_first / tpu == (t_first + 31) / tpu);
+    if (uniform) {  // warp-uniform branch
+      for (int off = V; off < 32; off <<= 1) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          kmn[c] = min(kmn[c], __shfl_xor_sync(0xffffffffu, kmn[c], off));
+          kmx[c] = max(kmx[c], __shfl_xor_sync(0xffffffffu, kmx[c], off));
+        }
+      }
+      if (lane < V) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          atomicMin(&mnk[g * D + j * CH + c], kmn[c]);
+          atomicMax(&mxk[g * D + j * CH + c], kmx[c]);
+        }
+      }
+    } else if (valid) {
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        atomicMin(&mnk[g * D + j * CH + c], kmn[c]);
+        atomicMax(&mxk[g * D + j * CH + c], kmx[c]);
+      }
     }
   }
 }
@@ -215,10 +256,12 @@ __device__ __forceinline__ void quant_finalize(const QuantParams& p, const Quant
   }
 }
 
-// Pass 2: encode and pack. d = x - min and t = d * inv, each correctly rounded,
-// then round half to even by adding 1.5 * 2^23: the rounded value's low
-// mantissa bits are the code (t <= 2^b - 1 + tiny, so no clamp is needed).
-// Codes are summed into the word with shifts; the magic bits are removed once.
+// Pass 2: encode and pack. d = x - min and t = d * inv, each correctly rounded
+// (__fsub_rn / __fmul_rn are never contracted into an FMA), then round half to
+// even by adding 1.5 * 2^23: the rounded value's low mantissa bits are the code
+// (t <= 2^b - 1 + tiny, so no clamp is needed). Codes are summed into the word
+// with shifts; the magic bits are removed once. (Packed f32x2 arithmetic is
+// not used here: ptxas may fuse a packed multiply and add into one rounding.)
 template <class Vec, int BITS>
 __device__ __forceinline__ void quant_pass2(const QuantParams& p, const QuantStep& st, const unsigned char* stage,
                                             const float* s_mn, const float* s_inv) {

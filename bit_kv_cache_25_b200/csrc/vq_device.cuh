@@ -61,11 +61,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // already suspends for a hardware-chosen time). Returns false on timeout after
 // recording kDevErrWaitTimeout; the caller must then skip its dependent work
 // but still take every barrier its CTA or cluster expects.
+// The limit (2^25 polls, with a short sleep after the first 64) is seconds
+// long: far beyond any legitimate wait inside one kernel, short enough to end a
+// kernel whose producer never arrives.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  uint32_t max_iters = (1u << 22)) {
+                                                  uint32_t max_iters = (1u << 25)) {
   for (uint32_t it = 0; it < max_iters; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (it > 64) __nanosleep(64);
+    if (it > 64) __nanosleep(100);
   }
   atomicOr(&g_device_error, kDevErrWaitTimeout);
   return false;

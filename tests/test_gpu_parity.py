@@ -164,6 +164,7 @@ def test_ragged_blocks_all_bit_widths(vq, D):
         cache = vq.LayerCache(desc)
         p0 = 0
         kh = _host(k)
+        vh = _host(v)
         for s, n in enumerate(sched):
             vq.vq_cache_append(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
             W = desc.word_rows(s)
@@ -175,6 +176,12 @@ def test_ragged_blocks_all_bit_widths(vq, D):
             vq.vq_dequantize(desc, s, packed, scale, zero, deq)
             torch.cuda.synchronize()
             words, s_ref, z_ref = vo.quantize_pack_block(kh[:, :, p0:p0 + n], bits)
+            v_words, v_s, v_z = vo.quantize_pack_block(vh[:, :, p0:p0 + n], bits)
+            np.testing.assert_array_equal(
+                cache.packed_v[offs[s]:offs[s + 1]].cpu().numpy().view(np.uint32).reshape(B, H, W, D), v_words)
+            np.testing.assert_array_equal(
+                cache.scale_v[s * B * H * D:(s + 1) * B * H * D].cpu().numpy().view(np.uint32),
+                v_s.reshape(-1).view(np.uint32))
             np.testing.assert_array_equal(packed.cpu().numpy().view(np.uint32).reshape(B, H, W, D), words)
             np.testing.assert_array_equal(scale.cpu().numpy().view(np.uint32), s_ref.reshape(-1).view(np.uint32))
             np.testing.assert_array_equal(zero.cpu().numpy().view(np.uint32), z_ref.reshape(-1).view(np.uint32))
@@ -193,7 +200,7 @@ def _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D):
     ov_, sv, zv = vo.cache_append(_host(v), sched, bits)
     p0 = 0
     for s, n in enumerate(sched):
-        out = torch.empty((B, H, n, D), dtype=torch.float32, device="cuda")
+        out = torch.full((B, H, n, D), float("nan"), dtype=torch.float32, device="cuda")
         vq.vq_attention_block(desc, cache, s, q[:, :, p0:p0 + n], float(sigma), out)
         torch.cuda.synchronize()
         rows = slice(0, min(n, 300))
@@ -202,8 +209,9 @@ def _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D):
         ref = vo.attention_f64(_host(q[:, :, p0:p0 + n])[:, :, rows], khat, vhat, sigma)
         got = out.cpu().numpy()[:, :, rows]
         err = np.max(np.abs(got - ref)) / np.sqrt(np.mean(ref ** 2))
-        assert err <= ATTN_TOL, (s, n, err)
+        assert err <= ATTN_TOL, (bits, s, n, err)
         p0 += n
+    assert vq.vq_poll_device_error() == 0
 
 
 def test_strided_inputs_and_outputs(vq):
