@@ -139,8 +139,7 @@ cudaError_t launch_attention_small(const AttnParams& p, cudaStream_t stream) {
 }  // namespace
 }  // namespace vq
 
-#include "attention_tc.cuh"
-#include "attention_ws.cuh"
+#include "attention_pipe.cuh"
 
 namespace vq {
 namespace {
@@ -153,15 +152,18 @@ constexpr int kTcMinQueries = 16;
 
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
   if (p.n_q >= kTcMinQueries) {
-    if (p.B * p.H > 65535) return cudaErrorInvalidConfiguration;
-    // head_dim 64: the single-warpgroup pipeline (110 KB shared memory, two
-    // CTAs per SM) wins on the VAR shapes, whose per-CTA work is short;
-    // head_dim 128: the warp-specialized kernel keeps the tensor cores busier
-    // on the long Infinity-shaped blocks.
-    if (p.bits == 4 && p.D == 64) return launch_attention_tc<4, 64>(p, stream);
-    if (p.bits == 4 && p.D == 128) return launch_attention_ws<4, 128, 1>(p, stream);
-    if (p.bits == 3 && p.D == 64) return launch_attention_tc<3, 64>(p, stream);
-    if (p.bits == 3 && p.D == 128) return launch_attention_ws<3, 128, 1>(p, stream);
+    // one query tile per work item when the block has at most 128 queries
+    // (two CTAs per SM at head_dim 64), else pairs of query tiles sharing
+    // every dequantized K/V tile
+    const bool pair = p.n_q > 128;
+    if (p.bits == 4 && p.D == 64) return pair ? launch_attention_pipe<4, 64, 2>(p, stream)
+                                              : launch_attention_pipe<4, 64, 1>(p, stream);
+    if (p.bits == 4 && p.D == 128) return pair ? launch_attention_pipe<4, 128, 2>(p, stream)
+                                               : launch_attention_pipe<4, 128, 1>(p, stream);
+    if (p.bits == 3 && p.D == 64) return pair ? launch_attention_pipe<3, 64, 2>(p, stream)
+                                              : launch_attention_pipe<3, 64, 1>(p, stream);
+    if (p.bits == 3 && p.D == 128) return pair ? launch_attention_pipe<3, 128, 2>(p, stream)
+                                               : launch_attention_pipe<3, 128, 1>(p, stream);
   }
   if (p.bits == 4 && p.D == 64) return launch_attention_small<4, 64>(p, stream);
   if (p.bits == 4 && p.D == 128) return launch_attention_small<4, 128>(p, stream);

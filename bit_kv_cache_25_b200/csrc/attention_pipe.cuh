@@ -1,0 +1,773 @@
+// Packed-KV block attention: persistent, warp-specialized, on the sm_100a
+// tensor cores (tcgen05.mma, fp32 accumulators in tensor memory, bulk copies).
+//
+// The queries of block s attend to every cached token of blocks 0..s.
+//
+// Operands. Each key tile (at most 64 tokens of one block) is dequantized in
+// shared memory to the cache's own fp32 values x^ = fma(code, scale, zero),
+// times a power of two 2^-e chosen per (batch, head) so that the largest |x^|
+// over blocks 0..s lies in [2^14, 2^15), and split into two fp16 parts:
+// hi = x^ with its mantissa cut to 10 bits (exact in fp16), lo = x^ - hi
+// rounded to fp16, so hi + lo = x^ (1 + O(2^-21)). The bf16 queries are exact
+// in fp16 after a power-of-two scale per row. Per tile and query tile of 128
+// rows, all accumulation in fp32:
+//   S  = q . (K^hi + K^lo)^T                      2 MMAs per 16-wide k-step
+//   O += Phi . V^hi + Plo . V^hi + Phi . V^lo     3 MMAs per 16-key step
+// with P = exp(logit - m) split the same way into fp16 hi/lo and written to
+// tensor memory over S. The dropped Plo . V^lo term is below 2^-20 of O. No
+// per-block state is needed: the scales live in the operands, so O collects
+// every block directly.
+//
+// Roles of one CTA (NQT query tiles of 128 rows of one (batch, head)):
+//   control warp, one thread: bulk copies of each tile's packed K/V words and
+//     of its block's four scale/zero vectors into a stage ring, and every
+//     tcgen05.mma: QK^T of tile g, then PV of tile g-1;
+//   unpack warpgroup: stage -> dequantized fp16 hi/lo K and V tiles (ring of
+//     NKV slots), plus the per-(batch, head) powers of two;
+//   one softmax warpgroup per query tile (one row per thread): query load and
+//     conversion, online softmax with a lazy reference maximum (O is rescaled
+//     in tensor memory only when a row maximum grows by more than kPipeTau),
+//     normalisation and output.
+// The CTA is persistent: it walks work items (batch*head, group of NQT query
+// tiles) with a stride of gridDim.x. Every ring runs on across items, so the
+// next item's copies, unpacking and first QK^T overlap this item's last tiles,
+// and a query tile's output is written while its next item's first softmax
+// is already done.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tc_ptx.cuh"
+#include "vq_device.cuh"
+#include "vq_internal.h"
+
+namespace vq {
+namespace {
+
+constexpr float kPipeTau = 8.0f;  // lazy-rescale threshold (natural-log units); p <= e^8 fits fp16
+
+template <int BITS, int D, int NQT>
+struct PipeCfg {
+  static constexpr int KT = 64;                            // keys per tile
+  static constexpr int CPW = 32 / BITS;
+  static constexpr uint32_t MASK = (1u << BITS) - 1u;
+  static constexpr int MAXW = (KT + CPW - 1) / CPW + 1;    // packed word-rows one tile can touch
+  static constexpr int STAGE_WORDS = MAXW * D;             // per tensor
+  static constexpr int NS = (D == 64) ? 3 : 2;             // S slots per query tile (tensor memory)
+  static constexpr int NKV = (D == 64) ? 3 : 2;            // dequantized K/V tile slots
+  static constexpr int NSTG = (D == 64) ? 4 : 2;           // packed-word stages
+  static constexpr bool STAGE_Q = (D == 64);               // next item's queries prefetched by cp.async
+  // one CTA per SM (416 threads, 128 registers each); with a single query
+  // tile the unpacking gets twice the warps, since it then bounds the tile rate
+  static constexpr int UNPACK_WARPS = (NQT == 2) ? 4 : 8;
+  static constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
+  static constexpr int KSPLIT = UNPACK_THREADS / 128;      // unpack threads per (tensor, word-row, octet)
+  static constexpr int UNPACK_T0 = NQT * 128;
+  static constexpr int CTRL_WARP = (NQT * 128 + UNPACK_THREADS) / 32;
+  static constexpr int THREADS = NQT * 128 + UNPACK_THREADS + 32;
+  static_assert(CPW % KSPLIT == 0, "key slots per word split evenly");
+  // ---- shared memory (byte offsets from a 1024-aligned base)
+  static constexpr int Q_SZ = 128 * D * 2;                 // fp16 q [128][D], K-major SW128
+  static constexpr int Q0 = 0;
+  static constexpr int TILE_SZ = KT * D * 2;               // fp16 [64][D], K-major SW128
+  static constexpr int KV0 = Q0 + NQT * Q_SZ;              // NKV x {K hi, K lo, V hi, V lo}
+  static constexpr int KV_SZ = 4 * TILE_SZ;
+  static constexpr int QST0 = KV0 + NKV * KV_SZ;           // bf16 [128][D] query staging per query tile
+  static constexpr int QST_SZ = STAGE_Q ? 128 * D * 2 : 0;
+  static constexpr int STG0 = QST0 + NQT * QST_SZ;         // NSTG x {K words, V words, [4][D] fp32 meta}
+  static constexpr int STG_META = 2 * STAGE_WORDS * 4;
+  static constexpr int STG_SZ = STG_META + 4 * D * 4;
+  static constexpr int HDR0 = STG0 + NSTG * STG_SZ;        // NKV x {2^eK, 2^eV, -, -}
+  static constexpr int NRED = 4;                           // exponent reduction slots (> NKV)
+  static constexpr int RED0 = HDR0 + NKV * 16;             // NRED x {K, V} x UNPACK_WARPS floats
+  static constexpr int BARS = RED0 + NRED * 2 * UNPACK_WARPS * 4;
+  static constexpr int NBARS = 2 * NSTG + 2 * NKV + NRED + NQT * (1 + 3 * NS);
+  static constexpr int TMEM_SLOT = BARS + NBARS * 8;
+  static constexpr int SMEM = TMEM_SLOT + 16;
+  static constexpr int SMEM_ALLOC = SMEM + 1024;           // room to align the base
+  static_assert(KV0 % 1024 == 0 && TILE_SZ % 1024 == 0 && Q_SZ % 1024 == 0, "operand alignment");
+  static_assert(STG0 % 16 == 0 && STG_SZ % 16 == 0 && STG_META % 16 == 0, "stage alignment");
+  static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
+  // ---- tensor memory: query tile qt owns columns [256 qt, 256 qt + 256): S slots, then O
+  static constexpr int COL_O = NS * 64;
+  static constexpr int TMEM_COLS = NQT * 256;
+  static_assert(NS * 64 + D <= 256, "tensor memory per query tile");
+};
+
+// 16-byte asynchronous copy global -> shared (L2 only); src_bytes = 0 fills zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// 2^e and 2^-e with amax * 2^-e in [2^14, 2^15) (e = 0 for amax == 0; e clamped to [-100, 100]).
+__device__ __forceinline__ void pipe_pow2(float amax, float& mul, float& inv) {
+  int e = 0;
+  if (amax > 0.0f) {
+    e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu) - 127 - 14;
+    e = max(-100, min(100, e));
+  }
+  mul = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+  inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+}
+
+// fp32 pair -> fp16x2 (lo half = a), round to nearest even
+__device__ __forceinline__ uint32_t pipe_h2(float a, float b) { return tc::cvt_half2(a, b); }
+
+template <int BITS, int D, int NQT>
+__global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
+    attention_pipe_kernel(const __grid_constant__ AttnParams p) {
+  using C = PipeCfg<BITS, D, NQT>;
+  constexpr int CPW = C::CPW;
+  constexpr int KT = C::KT;
+  constexpr int NS = C::NS;
+  constexpr int NKV = C::NKV;
+  constexpr int NSTG = C::NSTG;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  unsigned char* sm = smem_raw + (sbase - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::BARS);
+  uint64_t* stg_full = bars;
+  uint64_t* stg_empty = stg_full + NSTG;
+  uint64_t* kv_full = stg_empty + NSTG;
+  uint64_t* kv_empty = kv_full + NKV;
+  uint64_t* red_bar = kv_empty + NKV;
+  uint64_t* qbars = red_bar + C::NRED;  // per query tile: q_full, s_full[NS], p_full[NS], pv_done[NS]
+  constexpr int QB = 1 + 3 * NS;
+  auto q_full = [&](int qt) { return qbars + qt * QB; };
+  auto s_full = [&](int qt, int i) { return qbars + qt * QB + 1 + i; };
+  auto p_full = [&](int qt, int i) { return qbars + qt * QB + 1 + NS + i; };
+  auto pv_done = [&](int qt, int i) { return qbars + qt * QB + 1 + 2 * NS + i; };
+  float* hdr = reinterpret_cast<float*>(sm + C::HDR0);
+  float* red = reinterpret_cast<float*>(sm + C::RED0);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::TMEM_SLOT);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
+  const int n_qt = (p.n_q + 127) / 128;
+  const int n_groups = (n_qt + NQT - 1) / NQT;
+  const int n_items = p.B * p.H * n_groups;
+  int T = 0;  // key tiles per item
+  for (int kb = 0; kb <= p.s; ++kb) T += (p.blk[kb].n + KT - 1) / KT;
+  auto item_nqt = [&](int item) { return min(NQT, n_qt - (item % n_groups) * NQT); };
+
+  // ---- set-up: TMEM (warp 0), barriers (thread 0), zeroed K/V slots (unpack warpgroup)
+  if (warp == 0) {
+    tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < NSTG; ++i) {
+      mbar_init(&stg_full[i], 1);
+      mbar_init(&stg_empty[i], C::UNPACK_THREADS);
+    }
+    for (int i = 0; i < NKV; ++i) {
+      mbar_init(&kv_full[i], C::UNPACK_THREADS);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < C::NRED; ++i) mbar_init(&red_bar[i], C::UNPACK_WARPS);
+    for (int qt = 0; qt < NQT; ++qt) {
+      mbar_init(q_full(qt), 4);
+      for (int i = 0; i < NS; ++i) {
+        mbar_init(s_full(qt, i), 1);
+        mbar_init(p_full(qt, i), 4);
+        mbar_init(pv_done(qt, i), 1);
+      }
+    }
+    fence_barrier_init();
+  }
+  if (tid >= C::UNPACK_T0 && tid < C::UNPACK_T0 + C::UNPACK_THREADS) {
+    // key rows past a tile's valid keys are read by the MMAs (times zero
+    // probabilities) and must hold finite values
+    for (int i = C::KV0 + (tid - C::UNPACK_T0) * 16; i < C::KV0 + NKV * C::KV_SZ; i += C::UNPACK_THREADS * 16)
+      tc::sts128(sbase + i, 0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::CTRL_WARP) {
+    // =========================================================== control warp
+    if (lane == 0) {
+      // -- copies: walker over (item, block, first key); `copies` = tiles issued
+      int c_item = blockIdx.x, c_kb = 0, c_t0 = 0, copies = 0;
+      bool ok = true;
+      auto copy_next = [&]() -> bool {
+        const int st = copies % NSTG;
+        if (copies >= NSTG && !mbar_wait_bounded(&stg_empty[st], ((copies / NSTG) - 1) & 1)) return false;
+        const int bh = c_item / n_groups;
+        const AttnBlockInfo& bi = p.blk[c_kb];
+        const int wa = c_t0 / CPW;
+        const int wb = min(bi.W - 1, (c_t0 + KT - 1) / CPW);
+        const uint32_t bytes = static_cast<uint32_t>(wb - wa + 1) * D * 4;
+        const int64_t off = bi.word_off + static_cast<int64_t>(bh) * bi.W * D + static_cast<int64_t>(wa) * D;
+        const int64_t mo = c_kb * BHD + static_cast<int64_t>(bh) * D;
+        unsigned char* dst = sm + C::STG0 + st * C::STG_SZ;
+        constexpr uint32_t kMetaBytes = D * 4;
+        mbar_arrive_expect_tx(&stg_full[st], 2 * bytes + 4 * kMetaBytes);
+        bulk_copy_g2s(dst, p.packed_k + off, bytes, &stg_full[st]);
+        bulk_copy_g2s(dst + C::STAGE_WORDS * 4, p.packed_v + off, bytes, &stg_full[st]);
+        bulk_copy_g2s(dst + C::STG_META, p.scale_k + mo, kMetaBytes, &stg_full[st]);
+        bulk_copy_g2s(dst + C::STG_META + kMetaBytes, p.zero_k + mo, kMetaBytes, &stg_full[st]);
+        bulk_copy_g2s(dst + C::STG_META + 2 * kMetaBytes, p.scale_v + mo, kMetaBytes, &stg_full[st]);
+        bulk_copy_g2s(dst + C::STG_META + 3 * kMetaBytes, p.zero_v + mo, kMetaBytes, &stg_full[st]);
+        ++copies;
+        c_t0 += KT;
+        if (c_t0 >= bi.n) {
+          c_t0 = 0;
+          if (++c_kb > p.s) {
+            c_kb = 0;
+            c_item += gridDim.x;
+          }
+        }
+        return true;
+      };
+      for (int k = 0; k < NSTG && c_item < n_items; ++k) copy_next();
+
+      const uint32_t idesc_pv = tc::idesc_f16_f32(128, D, /*b_mn_major=*/true);
+      constexpr uint32_t kLbo = KT * 128;  // 64-channel groups of a [64][D] V tile read MN-major
+      auto issue_qk = [&](int qt, int slot, int kvs, int nk16) {
+        const uint32_t idesc = tc::idesc_f16_f32(128, nk16);
+        const uint32_t qa = sbase + C::Q0 + qt * C::Q_SZ;
+        const uint32_t kh = sbase + C::KV0 + kvs * C::KV_SZ;
+        const uint32_t d = tmem + qt * 256 + slot * 64;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
+            const uint32_t boff = part * C::TILE_SZ + (kk >> 2) * KT * 128 + (kk & 3) * 32;
+            tc::mma_f16_ss(d, tc::sw128_desc(qa + koff), tc::sw128_desc(kh + boff), idesc,
+                           (part == 0 && kk == 0) ? 0u : 1u);
+          }
+        }
+        tc::commit(s_full(qt, slot));
+      };
+      auto issue_pv = [&](int qt, int slot, int kvs, int nk16, bool first) {
+        const uint32_t vh = sbase + C::KV0 + kvs * C::KV_SZ + 2 * C::TILE_SZ;
+        const uint32_t pa = tmem + qt * 256 + slot * 64;
+        const uint32_t o = tmem + qt * 256 + C::COL_O;
+        // (A part, B part): (P hi, V hi), (P lo, V hi), (P hi, V lo)
+#pragma unroll
+        for (int part = 0; part < 3; ++part) {
+          const uint32_t acol = (part == 1) ? 8u : 0u;
+          const uint32_t vb = vh + ((part == 2) ? C::TILE_SZ : 0);
+          for (int kk = 0; kk < nk16 / 16; ++kk)
+            tc::mma_f16_ts(o, pa + 16 * kk + acol, tc::sw128_desc_mn(vb + kk * 2048, kLbo), idesc_pv,
+                           (first && part == 0 && kk == 0) ? 0u : 1u);
+        }
+        tc::commit(pv_done(qt, slot));
+      };
+
+      int nq[NQT], iq[NQT], prev_n[NQT];
+#pragma unroll
+      for (int qt = 0; qt < NQT; ++qt) nq[qt] = iq[qt] = prev_n[qt] = 0;
+      bool prev = false, prev_first = false;
+      int prev_nqt = 0, prev_kvs = 0, prev_nk16 = 0;
+      int gt = 0;
+      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        const int nqt = item_nqt(item);
+        int kb = 0, t0 = 0;
+        for (int j = 0; j < T; ++j, ++gt) {
+          const int nk = min(KT, p.blk[kb].n - t0);
+          const int nk16 = (nk + 15) & ~15;
+          const int kvs = gt % NKV;
+          if (!(ok = mbar_wait_bounded(&kv_full[kvs], (gt / NKV) & 1))) break;
+          // tile gt is unpacked, so its stage is free: refill it NSTG tiles ahead
+          if (c_item < n_items && !(ok = copy_next())) break;
+          if (j == 0) {
+            for (int qt = 0; qt < nqt && ok; ++qt) ok = mbar_wait_bounded(q_full(qt), iq[qt]++ & 1);
+            if (!ok) break;
+          }
+          tc::fence_after_sync();
+          // ---- QK^T of tile gt for every query tile
+          for (int qt = 0; qt < nqt && ok; ++qt) {
+            const int n = nq[qt];
+            const int slot = n % NS;
+            if (n >= NS && !(ok = mbar_wait_bounded(pv_done(qt, slot), ((n / NS) - 1) & 1))) break;
+            tc::fence_after_sync();
+            issue_qk(qt, slot, kvs, nk16);
+          }
+          if (!ok) break;
+          // ---- PV of the previous tile
+          if (prev) {
+            for (int qt = 0; qt < prev_nqt && ok; ++qt) {
+              const int n = prev_n[qt];
+              if (!(ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1))) break;
+              tc::fence_after_sync();
+              issue_pv(qt, n % NS, prev_kvs, prev_nk16, prev_first);
+            }
+            if (!ok) break;
+            tc::commit(&kv_empty[prev_kvs]);
+          }
+          prev = true;
+          prev_first = (j == 0);
+          prev_nqt = nqt;
+          prev_kvs = kvs;
+          prev_nk16 = nk16;
+          for (int qt = 0; qt < nqt; ++qt) prev_n[qt] = nq[qt]++;
+          t0 += KT;
+          if (t0 >= p.blk[kb].n) {
+            ++kb;
+            t0 = 0;
+          }
+        }
+      }
+      if (ok && prev) {
+        for (int qt = 0; qt < prev_nqt && ok; ++qt) {
+          const int n = prev_n[qt];
+          if (!(ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1))) break;
+          tc::fence_after_sync();
+          issue_pv(qt, n % NS, prev_kvs, prev_nk16, prev_first);
+        }
+        if (ok) tc::commit(&kv_empty[prev_kvs]);
+      }
+    }
+  } else if (tid >= C::UNPACK_T0) {
+    // =========================================================== unpack warpgroup
+    const int ut = tid - C::UNPACK_T0;
+    const float cmax = static_cast<float>(C::MASK);
+    // Powers of two of the k-th item of this CTA: max |x^| over blocks 0..s.
+    // Each warp reduces its share of the scale/zero vectors and posts its
+    // maxima in slot k % NRED; the item's first tile reads them all. A warp
+    // runs at most NKV - 1 tiles ahead of another, so NRED > NKV slots never
+    // alias a slot that is still to be read.
+    auto pow2_post = [&](int item, int k) {
+      const int bh = item / n_groups;
+      float ak = 0.0f, av = 0.0f;
+      for (int idx = ut; idx < (p.s + 1) * D; idx += C::UNPACK_THREADS) {
+        const int kb = idx / D;
+        const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + (idx - kb * D);
+        const float sk = __ldg(p.scale_k + mo), zk = __ldg(p.zero_k + mo);
+        const float sv = __ldg(p.scale_v + mo), zv = __ldg(p.zero_v + mo);
+        ak = fmaxf(ak, fmaxf(fabsf(zk), fabsf(fmaf(cmax, sk, zk))));
+        av = fmaxf(av, fmaxf(fabsf(zv), fabsf(fmaf(cmax, sv, zv))));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, o));
+        av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, o));
+      }
+      const int slot = k % C::NRED;
+      if (lane == 0) {
+        red[(slot * 2 + 0) * C::UNPACK_WARPS + (ut >> 5)] = ak;
+        red[(slot * 2 + 1) * C::UNPACK_WARPS + (ut >> 5)] = av;
+        mbar_arrive(&red_bar[slot]);
+      }
+      __syncwarp();
+    };
+    auto pow2_take = [&](int k, float& kmul, float& kinv, float& vmul, float& vinv) -> bool {
+      const int slot = k % C::NRED;
+      if (!mbar_wait_bounded(&red_bar[slot], (k / C::NRED) & 1)) return false;
+      const float* r = red + slot * 2 * C::UNPACK_WARPS;
+      float ak = 0.0f, av = 0.0f;
+#pragma unroll
+      for (int w = 0; w < C::UNPACK_WARPS; ++w) {
+        ak = fmaxf(ak, r[w]);
+        av = fmaxf(av, r[C::UNPACK_WARPS + w]);
+      }
+      pipe_pow2(ak, kmul, kinv);
+      pipe_pow2(av, vmul, vinv);
+      return true;
+    };
+
+    float kmul = 1.0f, kinv = 1.0f, vmul = 1.0f, vinv = 1.0f;
+    if (static_cast<int>(blockIdx.x) < n_items) pow2_post(blockIdx.x, 0);
+    int gt = 0;
+    bool ok = true;
+    for (int item = blockIdx.x, k = 0; ok && item < n_items; item += gridDim.x, ++k) {
+      if (!(ok = pow2_take(k, kmul, kinv, vmul, vinv))) break;
+      int kb = 0, t0 = 0;
+      for (int j = 0; j < T; ++j, ++gt) {
+        const int st = gt % NSTG;
+        const int kvs = gt % NKV;
+        if (!(ok = mbar_wait_bounded(&stg_full[st], (gt / NSTG) & 1))) break;
+        if (!(ok = mbar_wait_bounded(&kv_empty[kvs], ((gt / NKV) & 1) ^ 1))) break;
+        if (j == 0 && ut == 0) {
+          hdr[kvs * 4 + 0] = kmul;
+          hdr[kvs * 4 + 1] = vmul;
+        }
+        const AttnBlockInfo& bi = p.blk[kb];
+        const int wa = t0 / CPW;
+        const int wb = min(bi.W - 1, (t0 + KT - 1) / CPW);
+        const int nw = wb - wa + 1;
+        const unsigned char* stage = sm + C::STG0 + st * C::STG_SZ;
+        const uint32_t kvbase = sbase + C::KV0 + kvs * C::KV_SZ;
+        const int per = nw * (D / 8);
+        for (int task = ut; task < 2 * per * C::KSPLIT; task += C::UNPACK_THREADS) {
+          const int ks = task / (2 * per);  // which CPW / KSPLIT key slots of the word
+          const int tt = task - ks * (2 * per);
+          const int tsel = tt >= per ? 1 : 0;
+          const int r = tt - tsel * per;
+          const int wl = r / (D / 8);
+          const int jj = r - wl * (D / 8);
+          const uint32_t* src =
+              reinterpret_cast<const uint32_t*>(stage) + tsel * C::STAGE_WORDS + wl * D + 8 * jj;
+          // lanes jj and jj+4 of a quarter-warp would hit the same banks with
+          // 32-byte strided 16-byte loads; odd quads read their halves swapped
+          const int sw = (jj >> 2) & 1;
+          const uint4 a0 = *reinterpret_cast<const uint4*>(src + 4 * sw);
+          const uint4 a1 = *reinterpret_cast<const uint4*>(src + 4 * (sw ^ 1));
+          const uint4 a = sw ? a1 : a0;
+          const uint4 bq = sw ? a0 : a1;
+          constexpr int SLOTS = CPW / C::KSPLIT;
+          const int i0 = ks * SLOTS;
+          const uint32_t wd[8] = {a.x >> (BITS * i0), a.y >> (BITS * i0), a.z >> (BITS * i0), a.w >> (BITS * i0),
+                                  bq.x >> (BITS * i0), bq.y >> (BITS * i0), bq.z >> (BITS * i0), bq.w >> (BITS * i0)};
+          const float* meta = reinterpret_cast<const float*>(stage + C::STG_META) + 2 * tsel * D + 8 * jj;
+          const float mul = tsel ? vinv : kinv;
+          uint64_t sc2[4], ze2[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            sc2[u] = tc::f2pack(meta[2 * u] * mul, meta[2 * u + 1] * mul);
+            ze2[u] = tc::f2pack(meta[D + 2 * u] * mul, meta[D + 2 * u + 1] * mul);
+          }
+          const uint32_t dst = kvbase + tsel * 2 * C::TILE_SZ;
+          const int kbase = (wa + wl) * CPW + i0 - t0;  // tile-local key of slot i0
+          const uint64_t magic2 = tc::f2pack(-8388608.0f, -8388608.0f);
+#pragma unroll
+          for (int i = 0; i < SLOTS; ++i) {
+            const int key = kbase + i;
+            if (key < 0 || key >= KT) continue;
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              // code c as the float 2^23 + c, minus 2^23: exact
+              const uint32_t c0 = ((wd[2 * u] >> (BITS * i)) & C::MASK) | 0x4B000000u;
+              const uint32_t c1 = ((wd[2 * u + 1] >> (BITS * i)) & C::MASK) | 0x4B000000u;
+              const uint64_t cf = tc::add2(tc::f2pack(__uint_as_float(c0), __uint_as_float(c1)), magic2);
+              const uint64_t x = tc::fma2(cf, sc2[u], ze2[u]);  // fma(code, scale, zero) * 2^-e
+              const float x0 = tc::f2lo(x), x1 = tc::f2hi(x);
+              const float h0 = __uint_as_float(__float_as_uint(x0) & 0xffffe000u);
+              const float h1 = __uint_as_float(__float_as_uint(x1) & 0xffffe000u);
+              const uint64_t l2 = tc::sub2(x, tc::f2pack(h0, h1));
+              hi[u] = pipe_h2(h0, h1);
+              lo[u] = pipe_h2(tc::f2lo(l2), tc::f2hi(l2));
+            }
+            const uint32_t off = tc::sw128_offset(key, 8 * jj, KT);
+            tc::sts128(dst + off, hi[0], hi[1], hi[2], hi[3]);
+            tc::sts128(dst + C::TILE_SZ + off, lo[0], lo[1], lo[2], lo[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&stg_empty[st]);
+        mbar_arrive(&kv_full[kvs]);
+        // the next item's maxima, while this item's tiles run
+        if (j == 0 && item + static_cast<int>(gridDim.x) < n_items) pow2_post(item + gridDim.x, k + 1);
+        t0 += KT;
+        if (t0 >= bi.n) {
+          ++kb;
+          t0 = 0;
+        }
+      }
+    }
+  } else if ((tid >> 7) < NQT) {
+    // =========================================================== softmax warpgroup qt
+    const int qt = tid >> 7;
+    const int row = tid & 127;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tq = tmem + lane_off + qt * 256;
+    const uint32_t qs = sbase + C::Q0 + qt * C::Q_SZ;
+    const uint32_t qst = sbase + C::QST0 + qt * C::QST_SZ;
+    auto next_item = [&](int item) {
+      for (item += gridDim.x; item < n_items && item_nqt(item) <= qt; item += gridDim.x) {
+      }
+      return item;
+    };
+    auto row_of = [&](int item) { return (item % n_groups) * NQT * 128 + qt * 128 + row; };
+    auto q_ptr = [&](int item) -> const uint16_t* {
+      const int bh = item / n_groups;
+      const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+      return p.q + b * p.q_sb + h * p.q_sh + static_cast<int64_t>(row_of(item)) * p.q_st;
+    };
+    // the next item's query row -> staging (chunk c of the row at c ^ (row & 7))
+    auto stage_q = [&](int item) {
+      const bool valid = row_of(item) < p.n_q;
+      const uint16_t* src = valid ? q_ptr(item) : p.q;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c)
+        cp_async16(qst + (row * (D / 8) + (c ^ (row & 7))) * 16, src + 8 * c, valid ? 16u : 0u);
+      cp_async_commit();
+    };
+    // query row of `item` -> fp16 q * 2^-eq in the K-major SW128 A tile; returns 2^eq.
+    // Two passes over the row (maximum, then conversion), 8 values at a time.
+    auto q_chunk = [&](int item, int c) -> uint4 {
+      if constexpr (C::STAGE_Q) {
+        return lds128(sm + C::QST0 + qt * C::QST_SZ + (row * (D / 8) + (c ^ (row & 7))) * 16);
+      } else {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row_of(item) < p.n_q) v = *reinterpret_cast<const uint4*>(q_ptr(item) + 8 * c);
+        return v;
+      }
+    };
+    auto convert_q = [&](int item) -> float {
+      if constexpr (C::STAGE_Q) cp_async_wait_all();
+      float amax = 0.0f;
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = q_chunk(item, c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[k] << 16)), fabsf(__uint_as_float(w[k] & 0xffff0000u))));
+      }
+      float mul, inv;
+      pipe_pow2(amax, mul, inv);
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = q_chunk(item, c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          h[k] = pipe_h2(__uint_as_float(w[k] << 16) * inv, __uint_as_float(w[k] & 0xffff0000u) * inv);
+        tc::sts128(qs + tc::sw128_offset(row, 8 * c, 128), h[0], h[1], h[2], h[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_full(qt));
+      return mul;
+    };
+    auto epilogue = [&](int item, float l, float vmul) {
+      const int r = row_of(item);
+      const bool valid = r < p.n_q;
+      const int bh = item / n_groups;
+      const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+      const int64_t obase = b * p.o_sb + h * p.o_sh + static_cast<int64_t>(r) * p.o_st;
+      const float scl = vmul / l;
+#pragma unroll 1
+      for (int c16 = 0; c16 < D; c16 += 16) {
+        uint32_t o[16];
+        tc::tmem_ld16(tq + C::COL_O + c16, o);
+        tc::tmem_wait_ld();
+        if (!valid) continue;
+        float* v = reinterpret_cast<float*>(o);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(o[k]) * scl;
+        if (p.out_f32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + c16);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        } else {
+          uint32_t bf[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            uint32_t pair = 0;
+#pragma unroll
+            for (int uu = 0; uu < 2; ++uu) {
+              const uint32_t x = __float_as_uint(v[2 * k + uu]);
+              pair |= ((x + 0x7fffu + ((x >> 16) & 1u)) >> 16) << (16 * uu);
+            }
+            bf[k] = pair;
+          }
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + obase + c16);
+          dst[0] = make_uint4(bf[0], bf[1], bf[2], bf[3]);
+          dst[1] = make_uint4(bf[4], bf[5], bf[6], bf[7]);
+        }
+      }
+    };
+    auto scale_o = [&](float alpha) {
+#pragma unroll 1
+      for (int c16 = 0; c16 < D; c16 += 16) {
+        uint32_t r[16];
+        tc::tmem_ld16(tq + C::COL_O + c16, r);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * alpha);
+        tc::tmem_st16(tq + C::COL_O + c16, r);
+      }
+      tc::tmem_wait_st();
+    };
+
+    bool ok = true;
+    int item = blockIdx.x;
+    if (item < n_items && item_nqt(item) <= qt) item = next_item(item);
+    float qmul = 1.0f;  // 2^eq of the current item's row
+    if (item < n_items) {
+      if constexpr (C::STAGE_Q) stage_q(item);
+      qmul = convert_q(item);
+    }
+    int n = 0;  // tiles of this query tile so far (S/P slot counter)
+    bool epi = false;
+    int epi_item = 0;
+    float epi_l = 1.0f, epi_vmul = 1.0f;
+    bool epi_active = false;
+    while (ok && item < n_items) {
+      const int nxt = next_item(item);
+      const int gt0 = ((item - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x)) * T;
+      const bool warp_active = __any_sync(0xffffffffu, row_of(item) < p.n_q);
+      if constexpr (C::STAGE_Q) {
+        if (nxt < n_items) stage_q(nxt);
+      }
+      float up = 0.0f, vmul = 1.0f, m_ref = -INFINITY, l = 0.0f, qmul_next = qmul;
+      int kb = 0, t0 = 0;
+      for (int j = 0; j < T; ++j, ++n) {
+        const int nk = min(KT, p.blk[kb].n - t0);
+        const int nk16 = (nk + 15) & ~15;
+        const int slot = n % NS;
+        if (!(ok = mbar_wait_bounded(s_full(qt, slot), (n / NS) & 1))) break;
+        tc::fence_after_sync();
+        if (j == 0) {
+          // the unpack warpgroup's powers of two for this item (header of its first tile)
+          const int g = gt0;
+          if (!(ok = mbar_wait_bounded(&kv_full[g % NKV], (g / NKV) & 1))) break;
+          up = p.softmax_scale * qmul * hdr[(g % NKV) * 4 + 0];
+          vmul = hdr[(g % NKV) * 4 + 1];
+        }
+        // last QK^T of this item has completed: q of the next item can replace it
+        if (j == T - 1 && nxt < n_items) qmul_next = convert_q(nxt);
+        if (warp_active) {
+          const uint32_t t_s = tq + slot * 64;
+          uint32_t sr[KT];
+#pragma unroll
+          for (int c16 = 0; c16 < KT; c16 += 16)
+            if (c16 < nk16) tc::tmem_ld16(t_s + c16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c16]));
+          tc::tmem_wait_ld();
+          float smax = -INFINITY;
+#pragma unroll
+          for (int k = 0; k < KT; ++k)
+            if (k < nk) smax = fmaxf(smax, __uint_as_float(sr[k]));
+          const float mx = smax * up;
+          float alpha = 1.0f;
+          bool rescale = false;
+          if (mx > m_ref + kPipeTau) {
+            if (m_ref != -INFINITY) {
+              alpha = __expf(m_ref - mx);
+              rescale = true;
+            }
+            m_ref = mx;
+          }
+          l *= alpha;
+          if (__any_sync(0xffffffffu, rescale)) {
+            // O holds PV up to tile n-1 of this item once that PV completes
+            if (!(ok = mbar_wait_bounded(pv_done(qt, (n - 1) % NS), ((n - 1) / NS) & 1))) break;
+            tc::fence_after_sync();
+            scale_o(alpha);
+          }
+          constexpr float kLog2e = 1.4426950408889634f;
+          const float up2 = up * kLog2e;
+          const float c2 = -m_ref * kLog2e;
+          const uint64_t up2x2 = tc::f2pack(up2, up2);
+          const uint64_t c2x2 = tc::f2pack(c2, c2);
+          const bool partial = nk < nk16;
+          uint64_t rs2 = tc::f2pack(0.0f, 0.0f);
+#pragma unroll
+          for (int c8 = 0; c8 < KT; c8 += 8) {
+            if (c8 < nk16) {
+              // keys c8..c8+7: P hi -> columns (c8 / 16) * 16 + c8 % 16 / 2 + 0..3, lo 8 further
+              uint32_t hi[4], lo[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int j0 = c8 + 2 * u;
+                const uint64_t arg =
+                    tc::fma2(tc::f2pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), up2x2, c2x2);
+                float p0 = tc::ex2(tc::f2lo(arg));
+                float p1 = tc::ex2(tc::f2hi(arg));
+                if (partial) {
+                  p0 = (j0 < nk) ? p0 : 0.0f;
+                  p1 = (j0 + 1 < nk) ? p1 : 0.0f;
+                }
+                const uint64_t pp = tc::f2pack(p0, p1);
+                const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
+                const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
+                const uint64_t lo2 = tc::sub2(pp, tc::f2pack(h0, h1));
+                rs2 = tc::add2(rs2, pp);
+                hi[u] = pipe_h2(h0, h1);
+                lo[u] = pipe_h2(tc::f2lo(lo2), tc::f2hi(lo2));
+              }
+              // S of this row is in registers: P hi and lo replace it in place
+              const uint32_t col = (c8 & ~15) + (c8 & 15) / 2;
+              tc::tmem_st4(t_s + col, hi);
+              tc::tmem_st4(t_s + col + 8, lo);
+            }
+          }
+          tc::tmem_wait_st();
+          l += tc::f2lo(rs2) + tc::f2hi(rs2);
+        }
+        // the previous item's output, once its last PV is done (before this
+        // item's first PV overwrites O)
+        if (j == 0 && epi) {
+          epi = false;
+          if (epi_active) {
+            if (!(ok = mbar_wait_bounded(pv_done(qt, (n - 1) % NS), ((n - 1) / NS) & 1))) break;
+            tc::fence_after_sync();
+            epilogue(epi_item, epi_l, epi_vmul);
+          }
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(qt, slot));
+        t0 += KT;
+        if (t0 >= p.blk[kb].n) {
+          ++kb;
+          t0 = 0;
+        }
+      }
+      if (!ok) break;
+      epi = true;
+      epi_item = item;
+      epi_l = l;
+      epi_vmul = vmul;
+      epi_active = warp_active;
+      qmul = qmul_next;
+      item = nxt;
+    }
+    if (ok && epi && epi_active) {
+      if (mbar_wait_bounded(pv_done(qt, (n - 1) % NS), ((n - 1) / NS) & 1)) {
+        tc::fence_after_sync();
+        epilogue(epi_item, epi_l, epi_vmul);
+      }
+    }
+  }
+
+  // ---- teardown: every role has left its loop
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+template <int BITS, int D, int NQT>
+cudaError_t launch_attention_pipe(const AttnParams& p, cudaStream_t stream) {
+  using C = PipeCfg<BITS, D, NQT>;
+  static bool configured[kMaxDevices] = {};
+  static int ctas_per_sm[kMaxDevices] = {};
+  static int sms[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(attention_pipe_kernel<BITS, D, NQT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm[dev], attention_pipe_kernel<BITS, D, NQT>,
+                                                      C::THREADS, C::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    if (ctas_per_sm[dev] < 1) return cudaErrorInvalidConfiguration;
+    // tensor memory: at most 512 columns per SM
+    ctas_per_sm[dev] = min(ctas_per_sm[dev], 512 / C::TMEM_COLS);
+    configured[dev] = true;
+  }
+  const int n_qt = (p.n_q + 127) / 128;
+  const int64_t n_items = static_cast<int64_t>(p.B) * p.H * ((n_qt + NQT - 1) / NQT);
+  if (n_items > (int64_t(1) << 30)) return cudaErrorInvalidConfiguration;
+  const int64_t slots = static_cast<int64_t>(sms[dev]) * ctas_per_sm[dev];
+  const int grid = static_cast<int>(n_items < slots ? n_items : slots);
+  attention_pipe_kernel<BITS, D, NQT><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace vq

@@ -63,16 +63,14 @@ struct TcCfg {
   static constexpr int KB_SZ = kKT * D * 2;
   static constexpr int VB0 = KB0 + 2 * KB_SZ;             // 2 x [64][D] fp16 (read MN-major)
   static constexpr int VB_SZ = kKT * D * 2;
-  static constexpr int P_HI = VB0 + 2 * VB_SZ;            // [128][64] fp16
-  static constexpr int P_LO = P_HI + 128 * kKT * 2;
-  static constexpr int STG0 = P_LO + 128 * kKT * 2;       // 2 x {K words, V words}
+  static constexpr int STG0 = VB0 + 2 * VB_SZ;           // 2 x {K words, V words}
   static constexpr int STG_SZ = 2 * STAGE_WORDS * 4;
   static constexpr int META = STG0 + 2 * STG_SZ;          // 2 x [4][D] fp32: sk, zk, sv, zv
   static constexpr int BARS = META + 2 * 4 * D * 4;       // s[2], pv[2], stage[2]
   static constexpr int TMEM_SLOT = BARS + 6 * 8;
   static constexpr int SMEM = TMEM_SLOT + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;          // room to align the base
-  static_assert(KB0 % 1024 == 0 && VB0 % 1024 == 0 && P_HI % 1024 == 0 && P_LO % 1024 == 0, "tile alignment");
+  static_assert(KB0 % 1024 == 0 && VB0 % 1024 == 0, "tile alignment");
   static_assert(STG0 % 128 == 0 && STG_SZ % 128 == 0, "stage alignment");
   // tensor memory columns
   static constexpr int COL_S = 0;                         // 2 x 64 columns
@@ -138,7 +136,7 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
 
   // zero the K/V operand buffers once: rows past a tile's valid keys are read by
   // the MMAs (multiplied by zero probabilities) and must hold finite values
-  for (int i = C::KB0 + tid * 16; i < C::P_HI; i += kTcThreads * 16) tc::sts128(sbase + i, 0u, 0u, 0u, 0u);
+  for (int i = C::KB0 + tid * 16; i < C::STG0; i += kTcThreads * 16) tc::sts128(sbase + i, 0u, 0u, 0u, 0u);
   if (warp == 0) {
     tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
     tc::tmem_relinquish();
@@ -299,16 +297,18 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
     tc::commit(&bar_s[buf]);
   };
 
+  // PV of tile `buf`: A = P from TMEM, written in place over S[buf] (per 16-key
+  // chunk kk: 8 columns of P hi, then 8 columns of P lo), B = V codes (MN-major).
   auto issue_pv = [&](int nk16, int buf, bool first_of_block) {
     const uint32_t vbuf = sbase + C::VB0 + buf * C::VB_SZ;
     constexpr uint32_t kLbo = kKT * 128;  // 64-channel groups of the [64][D] V tile
+    const uint32_t pa = tmem + C::COL_S + buf * 64;
     for (int kk = 0; kk < nk16 / 16; ++kk) {
-      tc::mma_f16_ss(tmem + C::COL_U, tc::sw128_desc(sbase + C::P_HI + kk * 32),
-                     tc::sw128_desc_mn(vbuf + kk * 2048, kLbo), idesc_pv, (first_of_block && kk == 0) ? 0u : 1u);
+      tc::mma_f16_ts(tmem + C::COL_U, pa + 16 * kk, tc::sw128_desc_mn(vbuf + kk * 2048, kLbo), idesc_pv,
+                     (first_of_block && kk == 0) ? 0u : 1u);
     }
     for (int kk = 0; kk < nk16 / 16; ++kk) {
-      tc::mma_f16_ss(tmem + C::COL_U, tc::sw128_desc(sbase + C::P_LO + kk * 32),
-                     tc::sw128_desc_mn(vbuf + kk * 2048, kLbo), idesc_pv, 1u);
+      tc::mma_f16_ts(tmem + C::COL_U, pa + 16 * kk + 8, tc::sw128_desc_mn(vbuf + kk * 2048, kLbo), idesc_pv, 1u);
     }
     tc::commit(&bar_pv[buf]);
   };
@@ -418,23 +418,16 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
     const float up = up_q[cur.kb & 1];
     const uint32_t t_s = tmem + lane_off + C::COL_S + (g & 1) * 64;
     const bool partial = nk < nk16;  // columns [nk, nk16) are padding
+    // all of this row's S in one TMEM round trip (up to 64 columns)
+    uint32_t sr[kKT];
+#pragma unroll
+    for (int c16 = 0; c16 < kKT; c16 += 16)
+      if (c16 < nk16) tc::tmem_ld16(t_s + c16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c16]));
+    tc::tmem_wait_ld();
     float smax = -INFINITY;
 #pragma unroll
-    for (int c16 = 0; c16 < kKT; c16 += 16) {
-      if (c16 < nk16) {
-        uint32_t r[16];
-        tc::tmem_ld16(t_s + c16, r);
-        tc::tmem_wait_ld();
-        if (partial) {
-#pragma unroll
-          for (int u = 0; u < 16; ++u)
-            if (c16 + u < nk) smax = fmaxf(smax, __uint_as_float(r[u]));
-        } else {
-#pragma unroll
-          for (int u = 0; u < 16; ++u) smax = fmaxf(smax, __uint_as_float(r[u]));
-        }
-      }
-    }
+    for (int j = 0; j < kKT; ++j)
+      if (j < nk) smax = fmaxf(smax, __uint_as_float(sr[j]));
     const float mx = fmaf(smax, up, bias);
     float alpha = 1.0f;
     bool rescale = false;
@@ -482,37 +475,32 @@ __global__ void __launch_bounds__(kTcThreads, (D == 64) ? 2 : 1) attention_tc_ke
 #pragma unroll
     for (int c16 = 0; c16 < kKT; c16 += 16) {
       if (c16 < nk16) {
-        uint32_t r[16];
-        tc::tmem_ld16(t_s + c16, r);
-        tc::tmem_wait_ld();
+        uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int c8 = 0; c8 < 16; c8 += 8) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j0 = c16 + c8 + 2 * u;
-            const uint64_t arg = tc::fma2(tc::f2pack(__uint_as_float(r[c8 + 2 * u]), __uint_as_float(r[c8 + 2 * u + 1])),
-                                          up2x2, c2x2);
-            float p0 = tc::ex2(tc::f2lo(arg));
-            float p1 = tc::ex2(tc::f2hi(arg));
-            if (partial) {
-              p0 = (j0 < nk) ? p0 : 0.0f;
-              p1 = (j0 + 1 < nk) ? p1 : 0.0f;
-            }
-            const uint64_t pp = tc::f2pack(p0, p1);
-            const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
-            const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
-            const uint64_t lo2 = tc::fma2(tc::f2pack(h0, h1), neg1x2, pp);
-            rs2 = tc::add2(rs2, pp);
-            hi[u] = tc::cvt_half2(h0, h1);
-            lo[u] = tc::cvt_half2(tc::f2lo(lo2), tc::f2hi(lo2));
+        for (int u = 0; u < 8; ++u) {
+          const int j0 = c16 + 2 * u;
+          const uint64_t arg =
+              tc::fma2(tc::f2pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), up2x2, c2x2);
+          float p0 = tc::ex2(tc::f2lo(arg));
+          float p1 = tc::ex2(tc::f2hi(arg));
+          if (partial) {
+            p0 = (j0 < nk) ? p0 : 0.0f;
+            p1 = (j0 + 1 < nk) ? p1 : 0.0f;
           }
-          const uint32_t off = tc::sw128_offset(row, c16 + c8, 128);
-          tc::sts128(sbase + C::P_HI + off, hi[0], hi[1], hi[2], hi[3]);
-          tc::sts128(sbase + C::P_LO + off, lo[0], lo[1], lo[2], lo[3]);
+          const uint64_t pp = tc::f2pack(p0, p1);
+          const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
+          const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
+          const uint64_t lo2 = tc::fma2(tc::f2pack(h0, h1), neg1x2, pp);
+          rs2 = tc::add2(rs2, pp);
+          hi[u] = tc::cvt_half2(h0, h1);
+          lo[u] = tc::cvt_half2(tc::f2lo(lo2), tc::f2hi(lo2));
         }
+        // S of this row is in registers: P hi and lo replace it in place
+        tc::tmem_st8(t_s + c16, hi);
+        tc::tmem_st8(t_s + c16 + 8, lo);
       }
     }
+    tc::tmem_wait_st();
     rs += tc::f2lo(rs2) + tc::f2hi(rs2);
     }  // warp_active
     fence_proxy_async_smem();
