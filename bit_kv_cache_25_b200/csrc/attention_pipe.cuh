@@ -3,36 +3,39 @@
 //
 // The queries of block s attend to every cached token of blocks 0..s.
 //
-// Operands. Each key tile (at most 64 tokens of one block) is dequantized in
-// shared memory to the cache's own fp32 values x^ = fma(code, scale, zero),
-// times a power of two 2^-e chosen per (batch, head) so that the largest |x^|
-// over blocks 0..s lies in [2^14, 2^15), and split into two fp16 parts:
-// hi = x^ with its mantissa cut to 10 bits (exact in fp16), lo = x^ - hi
-// rounded to fp16, so hi + lo = x^ (1 + O(2^-21)). The bf16 queries are exact
-// in fp16 after a power-of-two scale per row. Per tile and query tile of 128
-// rows, all accumulation in fp32:
+// Operands. The cached tokens of blocks 0..s are walked as one sequence, in
+// key tiles of KT = 8192 / D tokens (128 at head_dim 64, 64 at 128) that may
+// span several blocks (at most MAXSEG block segments per tile). Each tile is
+// dequantized in shared memory to the cache's own fp32 values
+// x^ = fma(code, scale, zero) of each token's block, times a power of two 2^-e
+// chosen per (batch, head) so that the largest |x^| over blocks 0..s lies in
+// [2^14, 2^15), and split into two fp16 parts: hi = x^ with its mantissa cut to
+// 10 bits (exact in fp16), lo = x^ - hi rounded to fp16, so
+// hi + lo = x^ (1 + O(2^-21)). The bf16 queries are exact in fp16 after a
+// power-of-two scale per row. Per tile, for the 128 query rows of a work item,
+// all accumulation in fp32:
 //   S  = q . (K^hi + K^lo)^T                      2 MMAs per 16-wide k-step
 //   O += Phi . V^hi + Plo . V^hi + Phi . V^lo     3 MMAs per 16-key step
 // with P = exp(logit - m) split the same way into fp16 hi/lo and written to
-// tensor memory over S. The dropped Plo . V^lo term is below 2^-20 of O. No
-// per-block state is needed: the scales live in the operands, so O collects
-// every block directly.
+// tensor memory over S. The dropped Plo . V^lo term is below 2^-20 of O. The
+// scales live in the operands, so O collects every block directly.
 //
-// Roles of one CTA (NQT query tiles of 128 rows of one (batch, head)):
-//   control warp, one thread: bulk copies of each tile's packed K/V words and
-//     of its block's four scale/zero vectors into a stage ring, and every
-//     tcgen05.mma: QK^T of tile g, then PV of tile g-1;
-//   unpack warpgroup: stage -> dequantized fp16 hi/lo K and V tiles (ring of
-//     NKV slots), plus the per-(batch, head) powers of two;
-//   one softmax warpgroup per query tile (one row per thread): query load and
-//     conversion, online softmax with a lazy reference maximum (O is rescaled
-//     in tensor memory only when a row maximum grows by more than kPipeTau),
-//     normalisation and output.
-// The CTA is persistent: it walks work items (batch*head, group of NQT query
-// tiles) with a stride of gridDim.x. Every ring runs on across items, so the
-// next item's copies, unpacking and first QK^T overlap this item's last tiles,
-// and a query tile's output is written while its next item's first softmax
-// is already done.
+// Roles of one CTA (one CTA per SM, 448 threads):
+//   softmax warps 0-3 (one query row per thread, tensor-memory lanes 0-127):
+//     query load and conversion, online softmax with a lazy reference maximum
+//     (O is rescaled in tensor memory only when a row maximum grows by more
+//     than kPipeTau), normalisation and output;
+//   unpack warps 4-11: staged packed words -> dequantized fp16 hi/lo K and V
+//     tiles (ring of NKV slots), and the per-(batch, head) powers of two;
+//   producer warp 12, one thread: bulk copies of each tile's packed K/V word
+//     rows and of its blocks' scale/zero vectors into a stage ring;
+//   MMA warp 13, one thread: every tcgen05.mma, with shared-memory descriptors
+//     built once and advanced by constant offsets: QK^T of tile g, then PV of
+//     tile g-1.
+// The CTA is persistent: it walks work items (batch*head, 128-query tile)
+// with a stride of gridDim.x. Every ring runs on across items, so the next
+// item's copies, unpacking and first QK^T overlap this item's last tiles, and
+// an item's output is written while the next item's first softmax is done.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -49,52 +52,53 @@ namespace {
 
 constexpr float kPipeTau = 8.0f;  // lazy-rescale threshold (natural-log units); p <= e^8 fits fp16
 
-template <int BITS, int D, int NQT>
+template <int BITS, int D>
 struct PipeCfg {
-  static constexpr int KT = 64;                            // keys per tile
+  static constexpr int KT = 8192 / D;                      // keys per tile
   static constexpr int CPW = 32 / BITS;
   static constexpr uint32_t MASK = (1u << BITS) - 1u;
-  static constexpr int MAXW = (KT + CPW - 1) / CPW + 1;    // packed word-rows one tile can touch
-  static constexpr int STAGE_WORDS = MAXW * D;             // per tensor
-  static constexpr int NS = (D == 64) ? 3 : 2;             // S slots per query tile (tensor memory)
-  static constexpr int NKV = (D == 64) ? 3 : 2;            // dequantized K/V tile slots
-  static constexpr int NSTG = (D == 64) ? 4 : 2;           // packed-word stages
+  static constexpr int MAXSEG = (D == 64) ? 8 : 4;         // block segments per tile
+  static constexpr int MAXROWS = (KT + CPW - 1) / CPW + 2 * MAXSEG;  // staged word rows per tensor
+  static constexpr int NS = (D == 64) ? 3 : 4;             // S slots (tensor memory)
+  static constexpr int NKV = 2;                            // dequantized K/V tile slots
+  static constexpr int NSTG = 2;                           // packed-word stages
   static constexpr bool STAGE_Q = (D == 64);               // next item's queries prefetched by cp.async
-  // one CTA per SM (416 threads, 128 registers each); with a single query
-  // tile the unpacking gets twice the warps, since it then bounds the tile rate
-  static constexpr int UNPACK_WARPS = (NQT == 2) ? 4 : 8;
+  static constexpr int UNPACK_WARPS = 8;
   static constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
-  static constexpr int KSPLIT = UNPACK_THREADS / 128;      // unpack threads per (tensor, word-row, octet)
-  static constexpr int UNPACK_T0 = NQT * 128;
-  static constexpr int CTRL_WARP = (NQT * 128 + UNPACK_THREADS) / 32;
-  static constexpr int THREADS = NQT * 128 + UNPACK_THREADS + 32;
-  static_assert(CPW % KSPLIT == 0, "key slots per word split evenly");
+  static constexpr int UNPACK_T0 = 128;
+  static constexpr int PROD_WARP = 12;
+  static constexpr int MMA_WARP = 13;
+  static constexpr int THREADS = 448;
   // ---- shared memory (byte offsets from a 1024-aligned base)
   static constexpr int Q_SZ = 128 * D * 2;                 // fp16 q [128][D], K-major SW128
   static constexpr int Q0 = 0;
-  static constexpr int TILE_SZ = KT * D * 2;               // fp16 [64][D], K-major SW128
-  static constexpr int KV0 = Q0 + NQT * Q_SZ;              // NKV x {K hi, K lo, V hi, V lo}
+  static constexpr int TILE_SZ = KT * D * 2;               // fp16 [KT][D], K-major SW128
+  static constexpr int KV0 = Q0 + Q_SZ;                    // NKV x {K hi, K lo, V hi, V lo}
   static constexpr int KV_SZ = 4 * TILE_SZ;
-  static constexpr int QST0 = KV0 + NKV * KV_SZ;           // bf16 [128][D] query staging per query tile
+  static constexpr int QST0 = KV0 + NKV * KV_SZ;           // bf16 [128][D] query staging
   static constexpr int QST_SZ = STAGE_Q ? 128 * D * 2 : 0;
-  static constexpr int STG0 = QST0 + NQT * QST_SZ;         // NSTG x {K words, V words, [4][D] fp32 meta}
-  static constexpr int STG_META = 2 * STAGE_WORDS * 4;
-  static constexpr int STG_SZ = STG_META + 4 * D * 4;
+  static constexpr int STG0 = QST0 + QST_SZ;               // NSTG x {K rows, V rows, meta, segment table}
+  static constexpr int STG_V = MAXROWS * D * 4;
+  static constexpr int STG_META = 2 * STG_V;               // MAXSEG x [4][D] fp32: sk, zk, sv, zv
+  static constexpr int STG_SEG = STG_META + MAXSEG * 4 * D * 4;  // MAXSEG x int4 {block, u0, take, key0}
+  static constexpr int STG_ROWS = STG_SEG + MAXSEG * 16;   // MAXSEG x {first staged row, rows}, segment count
+  static constexpr int STG_SZ = STG_ROWS + (2 * MAXSEG + 4) * 4;
   static constexpr int HDR0 = STG0 + NSTG * STG_SZ;        // NKV x {2^eK, 2^eV, -, -}
   static constexpr int NRED = 4;                           // exponent reduction slots (> NKV)
   static constexpr int RED0 = HDR0 + NKV * 16;             // NRED x {K, V} x UNPACK_WARPS floats
   static constexpr int BARS = RED0 + NRED * 2 * UNPACK_WARPS * 4;
-  static constexpr int NBARS = 2 * NSTG + 2 * NKV + NRED + NQT * (1 + 3 * NS);
+  static constexpr int NBARS = 2 * NSTG + 2 * NKV + NRED + 1 + 3 * NS;
   static constexpr int TMEM_SLOT = BARS + NBARS * 8;
   static constexpr int SMEM = TMEM_SLOT + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;           // room to align the base
   static_assert(KV0 % 1024 == 0 && TILE_SZ % 1024 == 0 && Q_SZ % 1024 == 0, "operand alignment");
-  static_assert(STG0 % 16 == 0 && STG_SZ % 16 == 0 && STG_META % 16 == 0, "stage alignment");
+  static_assert(STG0 % 16 == 0 && STG_SZ % 16 == 0 && STG_V % 16 == 0 && STG_META % 16 == 0, "stage alignment");
+  static_assert(HDR0 % 16 == 0 && BARS % 8 == 0, "header alignment");
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
-  // ---- tensor memory: query tile qt owns columns [256 qt, 256 qt + 256): S slots, then O
-  static constexpr int COL_O = NS * 64;
-  static constexpr int TMEM_COLS = NQT * 256;
-  static_assert(NS * 64 + D <= 256, "tensor memory per query tile");
+  // ---- tensor memory: NS S slots of KT columns, then O (D columns)
+  static constexpr int COL_O = NS * KT;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(NS * KT + D <= TMEM_COLS, "tensor memory");
 };
 
 // 16-byte asynchronous copy global -> shared (L2 only); src_bytes = 0 fills zeros.
@@ -115,18 +119,44 @@ __device__ __forceinline__ void pipe_pow2(float amax, float& mul, float& inv) {
   inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
 }
 
-// fp32 pair -> fp16x2 (lo half = a), round to nearest even
-__device__ __forceinline__ uint32_t pipe_h2(float a, float b) { return tc::cvt_half2(a, b); }
+// Key-tile walker over the tokens of blocks 0..s: a tile takes up to KT tokens
+// and at most MAXSEG block segments. (kb, u): the block and the block-relative
+// token where the next tile starts.
+template <int KT, int MAXSEG>
+struct PipeWalk {
+  int kb, u;
+  __device__ __forceinline__ void reset() { kb = 0, u = 0; }
+  // Advances over one tile and returns its key count; seg(i, kb, u0, take,
+  // key0) is called for each of its block segments.
+  template <typename F>
+  __device__ __forceinline__ int next(const AttnParams& p, F&& seg) {
+    int nk = 0;
+    for (int i = 0; i < MAXSEG && nk < KT && kb <= p.s; ++i) {
+      const int take = min(KT - nk, p.blk[kb].n - u);
+      seg(i, kb, u, take, nk);
+      nk += take;
+      u += take;
+      if (u >= p.blk[kb].n) {
+        ++kb;
+        u = 0;
+      }
+    }
+    return nk;
+  }
+  __device__ __forceinline__ int next(const AttnParams& p) {
+    return next(p, [](int, int, int, int, int) {});
+  }
+};
 
-template <int BITS, int D, int NQT>
-__global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
-    attention_pipe_kernel(const __grid_constant__ AttnParams p) {
-  using C = PipeCfg<BITS, D, NQT>;
+template <int BITS, int D>
+__global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_kernel(const __grid_constant__ AttnParams p) {
+  using C = PipeCfg<BITS, D>;
   constexpr int CPW = C::CPW;
   constexpr int KT = C::KT;
   constexpr int NS = C::NS;
   constexpr int NKV = C::NKV;
   constexpr int NSTG = C::NSTG;
+  using Walk = PipeWalk<KT, C::MAXSEG>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -137,12 +167,10 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   uint64_t* kv_full = stg_empty + NSTG;
   uint64_t* kv_empty = kv_full + NKV;
   uint64_t* red_bar = kv_empty + NKV;
-  uint64_t* qbars = red_bar + C::NRED;  // per query tile: q_full, s_full[NS], p_full[NS], pv_done[NS]
-  constexpr int QB = 1 + 3 * NS;
-  auto q_full = [&](int qt) { return qbars + qt * QB; };
-  auto s_full = [&](int qt, int i) { return qbars + qt * QB + 1 + i; };
-  auto p_full = [&](int qt, int i) { return qbars + qt * QB + 1 + NS + i; };
-  auto pv_done = [&](int qt, int i) { return qbars + qt * QB + 1 + 2 * NS + i; };
+  uint64_t* q_full = red_bar + C::NRED;
+  uint64_t* s_full = q_full + 1;
+  uint64_t* p_full = s_full + NS;
+  uint64_t* pv_done = p_full + NS;
   float* hdr = reinterpret_cast<float*>(sm + C::HDR0);
   float* red = reinterpret_cast<float*>(sm + C::RED0);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::TMEM_SLOT);
@@ -152,13 +180,18 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   const int lane = tid & 31;
   const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
   const int n_qt = (p.n_q + 127) / 128;
-  const int n_groups = (n_qt + NQT - 1) / NQT;
-  const int n_items = p.B * p.H * n_groups;
+  const int n_items = p.B * p.H * n_qt;
   int T = 0;  // key tiles per item
-  for (int kb = 0; kb <= p.s; ++kb) T += (p.blk[kb].n + KT - 1) / KT;
-  auto item_nqt = [&](int item) { return min(NQT, n_qt - (item % n_groups) * NQT); };
+  {
+    Walk w;
+    w.reset();
+    while (w.kb <= p.s) {
+      w.next(p);
+      ++T;
+    }
+  }
 
-  // ---- set-up: TMEM (warp 0), barriers (thread 0), zeroed K/V slots (unpack warpgroup)
+  // ---- set-up: TMEM (warp 0), barriers (thread 0), zeroed K/V slots (unpack warps)
   if (warp == 0) {
     tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
     tc::tmem_relinquish();
@@ -173,13 +206,11 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < C::NRED; ++i) mbar_init(&red_bar[i], C::UNPACK_WARPS);
-    for (int qt = 0; qt < NQT; ++qt) {
-      mbar_init(q_full(qt), 4);
-      for (int i = 0; i < NS; ++i) {
-        mbar_init(s_full(qt, i), 1);
-        mbar_init(p_full(qt, i), 4);
-        mbar_init(pv_done(qt, i), 1);
-      }
+    mbar_init(q_full, 4);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
     }
     fence_barrier_init();
   }
@@ -195,145 +226,138 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == C::CTRL_WARP) {
-    // =========================================================== control warp
+  if (warp == C::PROD_WARP) {
+    // =========================================================== producer thread
     if (lane == 0) {
-      // -- copies: walker over (item, block, first key); `copies` = tiles issued
-      int c_item = blockIdx.x, c_kb = 0, c_t0 = 0, copies = 0;
       bool ok = true;
-      auto copy_next = [&]() -> bool {
-        const int st = copies % NSTG;
-        if (copies >= NSTG && !mbar_wait_bounded(&stg_empty[st], ((copies / NSTG) - 1) & 1)) return false;
-        const int bh = c_item / n_groups;
-        const AttnBlockInfo& bi = p.blk[c_kb];
-        const int wa = c_t0 / CPW;
-        const int wb = min(bi.W - 1, (c_t0 + KT - 1) / CPW);
-        const uint32_t bytes = static_cast<uint32_t>(wb - wa + 1) * D * 4;
-        const int64_t off = bi.word_off + static_cast<int64_t>(bh) * bi.W * D + static_cast<int64_t>(wa) * D;
-        const int64_t mo = c_kb * BHD + static_cast<int64_t>(bh) * D;
-        unsigned char* dst = sm + C::STG0 + st * C::STG_SZ;
-        constexpr uint32_t kMetaBytes = D * 4;
-        mbar_arrive_expect_tx(&stg_full[st], 2 * bytes + 4 * kMetaBytes);
-        bulk_copy_g2s(dst, p.packed_k + off, bytes, &stg_full[st]);
-        bulk_copy_g2s(dst + C::STAGE_WORDS * 4, p.packed_v + off, bytes, &stg_full[st]);
-        bulk_copy_g2s(dst + C::STG_META, p.scale_k + mo, kMetaBytes, &stg_full[st]);
-        bulk_copy_g2s(dst + C::STG_META + kMetaBytes, p.zero_k + mo, kMetaBytes, &stg_full[st]);
-        bulk_copy_g2s(dst + C::STG_META + 2 * kMetaBytes, p.scale_v + mo, kMetaBytes, &stg_full[st]);
-        bulk_copy_g2s(dst + C::STG_META + 3 * kMetaBytes, p.zero_v + mo, kMetaBytes, &stg_full[st]);
-        ++copies;
-        c_t0 += KT;
-        if (c_t0 >= bi.n) {
-          c_t0 = 0;
-          if (++c_kb > p.s) {
-            c_kb = 0;
-            c_item += gridDim.x;
+      int g = 0;
+      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        const int bh = item / n_qt;
+        Walk w;
+        w.reset();
+        for (int j = 0; j < T; ++j, ++g) {
+          const int st = g % NSTG;
+          if (g >= NSTG && !(ok = mbar_wait_bounded(&stg_empty[st], ((g / NSTG) - 1) & 1))) break;
+          unsigned char* stage = sm + C::STG0 + st * C::STG_SZ;
+          int4* segt = reinterpret_cast<int4*>(stage + C::STG_SEG);
+          int* rows = reinterpret_cast<int*>(stage + C::STG_ROWS);
+          // segment table (generic stores, published by the arrive below) and byte count
+          int nseg = 0, row0 = 0;
+          w.next(p, [&](int i, int kb, int u0, int take, int key0) {
+            const int wa = u0 / CPW, wb = (u0 + take - 1) / CPW;
+            segt[i] = make_int4(kb, u0, take, key0);
+            rows[2 * i] = row0;
+            rows[2 * i + 1] = wb - wa + 1;
+            row0 += wb - wa + 1;
+            nseg = i + 1;
+          });
+          rows[2 * C::MAXSEG] = nseg;
+          constexpr uint32_t kMetaBytes = D * 4;
+          mbar_arrive_expect_tx(&stg_full[st],
+                                static_cast<uint32_t>(row0) * D * 4 * 2 + static_cast<uint32_t>(nseg) * 4 * kMetaBytes);
+          for (int i = 0; i < nseg; ++i) {
+            const int4 sg = segt[i];
+            const AttnBlockInfo& bi = p.blk[sg.x];
+            const int wa = sg.y / CPW;
+            const uint32_t bytes = static_cast<uint32_t>(rows[2 * i + 1]) * D * 4;
+            const int64_t off = bi.word_off + static_cast<int64_t>(bh) * bi.W * D + static_cast<int64_t>(wa) * D;
+            const int64_t mo = sg.x * BHD + static_cast<int64_t>(bh) * D;
+            unsigned char* dst = stage + rows[2 * i] * D * 4;
+            bulk_copy_g2s(dst, p.packed_k + off, bytes, &stg_full[st]);
+            bulk_copy_g2s(dst + C::STG_V, p.packed_v + off, bytes, &stg_full[st]);
+            unsigned char* md = stage + C::STG_META + i * 4 * kMetaBytes;
+            bulk_copy_g2s(md, p.scale_k + mo, kMetaBytes, &stg_full[st]);
+            bulk_copy_g2s(md + kMetaBytes, p.zero_k + mo, kMetaBytes, &stg_full[st]);
+            bulk_copy_g2s(md + 2 * kMetaBytes, p.scale_v + mo, kMetaBytes, &stg_full[st]);
+            bulk_copy_g2s(md + 3 * kMetaBytes, p.zero_v + mo, kMetaBytes, &stg_full[st]);
           }
         }
-        return true;
-      };
-      for (int k = 0; k < NSTG && c_item < n_items; ++k) copy_next();
-
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // =========================================================== MMA thread
+    if (lane == 0) {
+      constexpr uint32_t kLbo = KT * 128;  // 64-channel groups of a [KT][D] V tile read MN-major
       const uint32_t idesc_pv = tc::idesc_f16_f32(128, D, /*b_mn_major=*/true);
-      constexpr uint32_t kLbo = KT * 128;  // 64-channel groups of a [64][D] V tile read MN-major
-      auto issue_qk = [&](int qt, int slot, int kvs, int nk16) {
+      const uint64_t qdesc = tc::sw128_desc(sbase + C::Q0);
+      const uint64_t kdesc0 = tc::sw128_desc(sbase + C::KV0);
+      const uint64_t vdesc0 = tc::sw128_desc_mn(sbase + C::KV0 + 2 * C::TILE_SZ, kLbo);
+      auto issue_qk = [&](int slot, int kvs, int nk16) {
         const uint32_t idesc = tc::idesc_f16_f32(128, nk16);
-        const uint32_t qa = sbase + C::Q0 + qt * C::Q_SZ;
-        const uint32_t kh = sbase + C::KV0 + kvs * C::KV_SZ;
-        const uint32_t d = tmem + qt * 256 + slot * 64;
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>((kvs * C::KV_SZ) >> 4);
+        const uint32_t d = tmem + slot * KT;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-            const uint32_t boff = part * C::TILE_SZ + (kk >> 2) * KT * 128 + (kk & 3) * 32;
-            tc::mma_f16_ss(d, tc::sw128_desc(qa + koff), tc::sw128_desc(kh + boff), idesc,
-                           (part == 0 && kk == 0) ? 0u : 1u);
+            constexpr int kSlabA = 128 * 128, kSlabB = KT * 128;
+            const uint32_t aoff = ((kk >> 2) * kSlabA + (kk & 3) * 32) >> 4;
+            const uint32_t boff = (part * C::TILE_SZ + (kk >> 2) * kSlabB + (kk & 3) * 32) >> 4;
+            tc::mma_f16_ss(d, qdesc + aoff, kd + boff, idesc, (part == 0 && kk == 0) ? 0u : 1u);
           }
         }
-        tc::commit(s_full(qt, slot));
+        tc::commit(&s_full[slot]);
       };
-      auto issue_pv = [&](int qt, int slot, int kvs, int nk16, bool first) {
-        const uint32_t vh = sbase + C::KV0 + kvs * C::KV_SZ + 2 * C::TILE_SZ;
-        const uint32_t pa = tmem + qt * 256 + slot * 64;
-        const uint32_t o = tmem + qt * 256 + C::COL_O;
+      auto issue_pv = [&](int slot, int kvs, int nk16, bool first) {
+        const uint64_t vd = vdesc0 + static_cast<uint64_t>((kvs * C::KV_SZ) >> 4);
+        const uint32_t pa = tmem + slot * KT;
+        const uint32_t o = tmem + C::COL_O;
+        const int nkk = nk16 / 16;
         // (A part, B part): (P hi, V hi), (P lo, V hi), (P hi, V lo)
 #pragma unroll
         for (int part = 0; part < 3; ++part) {
           const uint32_t acol = (part == 1) ? 8u : 0u;
-          const uint32_t vb = vh + ((part == 2) ? C::TILE_SZ : 0);
-          for (int kk = 0; kk < nk16 / 16; ++kk)
-            tc::mma_f16_ts(o, pa + 16 * kk + acol, tc::sw128_desc_mn(vb + kk * 2048, kLbo), idesc_pv,
-                           (first && part == 0 && kk == 0) ? 0u : 1u);
+          const uint32_t vpart = (part == 2) ? (C::TILE_SZ >> 4) : 0u;
+#pragma unroll
+          for (int kk = 0; kk < KT / 16; ++kk) {
+            if (kk < nkk)
+              tc::mma_f16_ts(o, pa + 16 * kk + acol, vd + vpart + ((kk * 2048) >> 4), idesc_pv,
+                             (first && part == 0 && kk == 0) ? 0u : 1u);
+          }
         }
-        tc::commit(pv_done(qt, slot));
+        tc::commit(&pv_done[slot]);
       };
 
-      int nq[NQT], iq[NQT], prev_n[NQT];
-#pragma unroll
-      for (int qt = 0; qt < NQT; ++qt) nq[qt] = iq[qt] = prev_n[qt] = 0;
+      bool ok = true;
       bool prev = false, prev_first = false;
-      int prev_nqt = 0, prev_kvs = 0, prev_nk16 = 0;
-      int gt = 0;
+      int prev_nk16 = 0;
+      int g = 0, iq = 0;
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-        const int nqt = item_nqt(item);
-        int kb = 0, t0 = 0;
-        for (int j = 0; j < T; ++j, ++gt) {
-          const int nk = min(KT, p.blk[kb].n - t0);
+        Walk w;
+        w.reset();
+        for (int j = 0; j < T; ++j, ++g) {
+          const int nk = w.next(p);
           const int nk16 = (nk + 15) & ~15;
-          const int kvs = gt % NKV;
-          if (!(ok = mbar_wait_bounded(&kv_full[kvs], (gt / NKV) & 1))) break;
-          // tile gt is unpacked, so its stage is free: refill it NSTG tiles ahead
-          if (c_item < n_items && !(ok = copy_next())) break;
-          if (j == 0) {
-            for (int qt = 0; qt < nqt && ok; ++qt) ok = mbar_wait_bounded(q_full(qt), iq[qt]++ & 1);
-            if (!ok) break;
-          }
+          const int kvs = g % NKV;
+          const int slot = g % NS;
+          if (!(ok = mbar_wait_bounded(&kv_full[kvs], (g / NKV) & 1))) break;
+          if (j == 0 && !(ok = mbar_wait_bounded(q_full, iq++ & 1))) break;
+          if (g >= NS && !(ok = mbar_wait_bounded(&pv_done[slot], ((g / NS) - 1) & 1))) break;
           tc::fence_after_sync();
-          // ---- QK^T of tile gt for every query tile
-          for (int qt = 0; qt < nqt && ok; ++qt) {
-            const int n = nq[qt];
-            const int slot = n % NS;
-            if (n >= NS && !(ok = mbar_wait_bounded(pv_done(qt, slot), ((n / NS) - 1) & 1))) break;
-            tc::fence_after_sync();
-            issue_qk(qt, slot, kvs, nk16);
-          }
-          if (!ok) break;
-          // ---- PV of the previous tile
+          issue_qk(slot, kvs, nk16);
           if (prev) {
-            for (int qt = 0; qt < prev_nqt && ok; ++qt) {
-              const int n = prev_n[qt];
-              if (!(ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1))) break;
-              tc::fence_after_sync();
-              issue_pv(qt, n % NS, prev_kvs, prev_nk16, prev_first);
-            }
-            if (!ok) break;
-            tc::commit(&kv_empty[prev_kvs]);
+            const int gp = g - 1;
+            if (!(ok = mbar_wait_bounded(&p_full[gp % NS], (gp / NS) & 1))) break;
+            tc::fence_after_sync();
+            issue_pv(gp % NS, gp % NKV, prev_nk16, prev_first);
+            tc::commit(&kv_empty[gp % NKV]);
           }
           prev = true;
           prev_first = (j == 0);
-          prev_nqt = nqt;
-          prev_kvs = kvs;
           prev_nk16 = nk16;
-          for (int qt = 0; qt < nqt; ++qt) prev_n[qt] = nq[qt]++;
-          t0 += KT;
-          if (t0 >= p.blk[kb].n) {
-            ++kb;
-            t0 = 0;
-          }
         }
       }
       if (ok && prev) {
-        for (int qt = 0; qt < prev_nqt && ok; ++qt) {
-          const int n = prev_n[qt];
-          if (!(ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1))) break;
+        const int gp = g - 1;
+        if (mbar_wait_bounded(&p_full[gp % NS], (gp / NS) & 1)) {
           tc::fence_after_sync();
-          issue_pv(qt, n % NS, prev_kvs, prev_nk16, prev_first);
+          issue_pv(gp % NS, gp % NKV, prev_nk16, prev_first);
+          tc::commit(&kv_empty[gp % NKV]);
         }
-        if (ok) tc::commit(&kv_empty[prev_kvs]);
       }
     }
   } else if (tid >= C::UNPACK_T0) {
-    // =========================================================== unpack warpgroup
+    // =========================================================== unpack warps
     const int ut = tid - C::UNPACK_T0;
     const float cmax = static_cast<float>(C::MASK);
     // Powers of two of the k-th item of this CTA: max |x^| over blocks 0..s.
@@ -342,7 +366,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     // runs at most NKV - 1 tiles ahead of another, so NRED > NKV slots never
     // alias a slot that is still to be read.
     auto pow2_post = [&](int item, int k) {
-      const int bh = item / n_groups;
+      const int bh = item / n_qt;
       float ak = 0.0f, av = 0.0f;
       for (int idx = ut; idx < (p.s + 1) * D; idx += C::UNPACK_THREADS) {
         const int kb = idx / D;
@@ -382,36 +406,36 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
 
     float kmul = 1.0f, kinv = 1.0f, vmul = 1.0f, vinv = 1.0f;
     if (static_cast<int>(blockIdx.x) < n_items) pow2_post(blockIdx.x, 0);
-    int gt = 0;
+    int g = 0;
     bool ok = true;
     for (int item = blockIdx.x, k = 0; ok && item < n_items; item += gridDim.x, ++k) {
       if (!(ok = pow2_take(k, kmul, kinv, vmul, vinv))) break;
-      int kb = 0, t0 = 0;
-      for (int j = 0; j < T; ++j, ++gt) {
-        const int st = gt % NSTG;
-        const int kvs = gt % NKV;
-        if (!(ok = mbar_wait_bounded(&stg_full[st], (gt / NSTG) & 1))) break;
-        if (!(ok = mbar_wait_bounded(&kv_empty[kvs], ((gt / NKV) & 1) ^ 1))) break;
+      for (int j = 0; j < T; ++j, ++g) {
+        const int st = g % NSTG;
+        const int kvs = g % NKV;
+        if (!(ok = mbar_wait_bounded(&stg_full[st], (g / NSTG) & 1))) break;
+        if (!(ok = mbar_wait_bounded(&kv_empty[kvs], ((g / NKV) & 1) ^ 1))) break;
         if (j == 0 && ut == 0) {
           hdr[kvs * 4 + 0] = kmul;
           hdr[kvs * 4 + 1] = vmul;
         }
-        const AttnBlockInfo& bi = p.blk[kb];
-        const int wa = t0 / CPW;
-        const int wb = min(bi.W - 1, (t0 + KT - 1) / CPW);
-        const int nw = wb - wa + 1;
         const unsigned char* stage = sm + C::STG0 + st * C::STG_SZ;
+        const int4* segt = reinterpret_cast<const int4*>(stage + C::STG_SEG);
+        const int* rows = reinterpret_cast<const int*>(stage + C::STG_ROWS);
+        const int nseg = rows[2 * C::MAXSEG];
+        const int R = rows[2 * (nseg - 1)] + rows[2 * (nseg - 1) + 1];  // staged word rows
         const uint32_t kvbase = sbase + C::KV0 + kvs * C::KV_SZ;
-        const int per = nw * (D / 8);
-        for (int task = ut; task < 2 * per * C::KSPLIT; task += C::UNPACK_THREADS) {
-          const int ks = task / (2 * per);  // which CPW / KSPLIT key slots of the word
-          const int tt = task - ks * (2 * per);
-          const int tsel = tt >= per ? 1 : 0;
-          const int r = tt - tsel * per;
-          const int wl = r / (D / 8);
-          const int jj = r - wl * (D / 8);
-          const uint32_t* src =
-              reinterpret_cast<const uint32_t*>(stage) + tsel * C::STAGE_WORDS + wl * D + 8 * jj;
+        constexpr int OCT = D / 8;
+        for (int task = ut; task < 2 * R * OCT; task += C::UNPACK_THREADS) {
+          const int tsel = task >= R * OCT ? 1 : 0;
+          const int r = task - tsel * R * OCT;
+          const int sr = r / OCT;
+          const int jj = r - sr * OCT;
+          // the segment of staged row sr
+          int i = 0;
+          while (i + 1 < nseg && rows[2 * (i + 1)] <= sr) ++i;
+          const int4 sg = segt[i];  // {block, u0, take, key0}
+          const uint32_t* src = reinterpret_cast<const uint32_t*>(stage + tsel * C::STG_V) + sr * D + 8 * jj;
           // lanes jj and jj+4 of a quarter-warp would hit the same banks with
           // 32-byte strided 16-byte loads; odd quads read their halves swapped
           const int sw = (jj >> 2) & 1;
@@ -419,11 +443,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           const uint4 a1 = *reinterpret_cast<const uint4*>(src + 4 * (sw ^ 1));
           const uint4 a = sw ? a1 : a0;
           const uint4 bq = sw ? a0 : a1;
-          constexpr int SLOTS = CPW / C::KSPLIT;
-          const int i0 = ks * SLOTS;
-          const uint32_t wd[8] = {a.x >> (BITS * i0), a.y >> (BITS * i0), a.z >> (BITS * i0), a.w >> (BITS * i0),
-                                  bq.x >> (BITS * i0), bq.y >> (BITS * i0), bq.z >> (BITS * i0), bq.w >> (BITS * i0)};
-          const float* meta = reinterpret_cast<const float*>(stage + C::STG_META) + 2 * tsel * D + 8 * jj;
+          const uint32_t wd[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+          const float* meta =
+              reinterpret_cast<const float*>(stage + C::STG_META) + (i * 4 + 2 * tsel) * D + 8 * jj;
           const float mul = tsel ? vinv : kinv;
           uint64_t sc2[4], ze2[4];
 #pragma unroll
@@ -432,28 +454,30 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             ze2[u] = tc::f2pack(meta[D + 2 * u] * mul, meta[D + 2 * u + 1] * mul);
           }
           const uint32_t dst = kvbase + tsel * 2 * C::TILE_SZ;
-          const int kbase = (wa + wl) * CPW + i0 - t0;  // tile-local key of slot i0
+          // block token of slot 0 of this word row, and its tile key
+          const int ub = (sg.y / CPW + (sr - rows[2 * i])) * CPW;
+          const int kbase = sg.w + ub - sg.y;
+          const int ulo = sg.y - ub, uhi = sg.y + sg.z - ub;  // valid slots [ulo, uhi)
           const uint64_t magic2 = tc::f2pack(-8388608.0f, -8388608.0f);
 #pragma unroll
-          for (int i = 0; i < SLOTS; ++i) {
-            const int key = kbase + i;
-            if (key < 0 || key >= KT) continue;
+          for (int s = 0; s < CPW; ++s) {
+            if (s < ulo || s >= uhi) continue;
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               // code c as the float 2^23 + c, minus 2^23: exact
-              const uint32_t c0 = ((wd[2 * u] >> (BITS * i)) & C::MASK) | 0x4B000000u;
-              const uint32_t c1 = ((wd[2 * u + 1] >> (BITS * i)) & C::MASK) | 0x4B000000u;
+              const uint32_t c0 = ((wd[2 * u] >> (BITS * s)) & C::MASK) | 0x4B000000u;
+              const uint32_t c1 = ((wd[2 * u + 1] >> (BITS * s)) & C::MASK) | 0x4B000000u;
               const uint64_t cf = tc::add2(tc::f2pack(__uint_as_float(c0), __uint_as_float(c1)), magic2);
               const uint64_t x = tc::fma2(cf, sc2[u], ze2[u]);  // fma(code, scale, zero) * 2^-e
               const float x0 = tc::f2lo(x), x1 = tc::f2hi(x);
               const float h0 = __uint_as_float(__float_as_uint(x0) & 0xffffe000u);
               const float h1 = __uint_as_float(__float_as_uint(x1) & 0xffffe000u);
               const uint64_t l2 = tc::sub2(x, tc::f2pack(h0, h1));
-              hi[u] = pipe_h2(h0, h1);
-              lo[u] = pipe_h2(tc::f2lo(l2), tc::f2hi(l2));
+              hi[u] = tc::cvt_half2(h0, h1);
+              lo[u] = tc::cvt_half2(tc::f2lo(l2), tc::f2hi(l2));
             }
-            const uint32_t off = tc::sw128_offset(key, 8 * jj, KT);
+            const uint32_t off = tc::sw128_offset(kbase + s, 8 * jj, KT);
             tc::sts128(dst + off, hi[0], hi[1], hi[2], hi[3]);
             tc::sts128(dst + C::TILE_SZ + off, lo[0], lo[1], lo[2], lo[3]);
           }
@@ -463,29 +487,18 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         mbar_arrive(&kv_full[kvs]);
         // the next item's maxima, while this item's tiles run
         if (j == 0 && item + static_cast<int>(gridDim.x) < n_items) pow2_post(item + gridDim.x, k + 1);
-        t0 += KT;
-        if (t0 >= bi.n) {
-          ++kb;
-          t0 = 0;
-        }
       }
     }
-  } else if ((tid >> 7) < NQT) {
-    // =========================================================== softmax warpgroup qt
-    const int qt = tid >> 7;
-    const int row = tid & 127;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tq = tmem + lane_off + qt * 256;
-    const uint32_t qs = sbase + C::Q0 + qt * C::Q_SZ;
-    const uint32_t qst = sbase + C::QST0 + qt * C::QST_SZ;
-    auto next_item = [&](int item) {
-      for (item += gridDim.x; item < n_items && item_nqt(item) <= qt; item += gridDim.x) {
-      }
-      return item;
-    };
-    auto row_of = [&](int item) { return (item % n_groups) * NQT * 128 + qt * 128 + row; };
+  } else {
+    // =========================================================== softmax warps
+    const int row = tid;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tq = tmem + lane_off;
+    const uint32_t qs = sbase + C::Q0;
+    const uint32_t qst = sbase + C::QST0;
+    auto row_of = [&](int item) { return (item % n_qt) * 128 + row; };
     auto q_ptr = [&](int item) -> const uint16_t* {
-      const int bh = item / n_groups;
+      const int bh = item / n_qt;
       const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
       return p.q + b * p.q_sb + h * p.q_sh + static_cast<int64_t>(row_of(item)) * p.q_st;
     };
@@ -502,7 +515,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     // Two passes over the row (maximum, then conversion), 8 values at a time.
     auto q_chunk = [&](int item, int c) -> uint4 {
       if constexpr (C::STAGE_Q) {
-        return lds128(sm + C::QST0 + qt * C::QST_SZ + (row * (D / 8) + (c ^ (row & 7))) * 16);
+        return lds128(sm + C::QST0 + (row * (D / 8) + (c ^ (row & 7))) * 16);
       } else {
         uint4 v = make_uint4(0, 0, 0, 0);
         if (row_of(item) < p.n_q) v = *reinterpret_cast<const uint4*>(q_ptr(item) + 8 * c);
@@ -529,18 +542,18 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         uint32_t h[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          h[k] = pipe_h2(__uint_as_float(w[k] << 16) * inv, __uint_as_float(w[k] & 0xffff0000u) * inv);
+          h[k] = tc::cvt_half2(__uint_as_float(w[k] << 16) * inv, __uint_as_float(w[k] & 0xffff0000u) * inv);
         tc::sts128(qs + tc::sw128_offset(row, 8 * c, 128), h[0], h[1], h[2], h[3]);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(q_full(qt));
+      if (lane == 0) mbar_arrive(q_full);
       return mul;
     };
     auto epilogue = [&](int item, float l, float vmul) {
       const int r = row_of(item);
       const bool valid = r < p.n_q;
-      const int bh = item / n_groups;
+      const int bh = item / n_qt;
       const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
       const int64_t obase = b * p.o_sb + h * p.o_sh + static_cast<int64_t>(r) * p.o_st;
       const float scl = vmul / l;
@@ -587,38 +600,44 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       }
       tc::tmem_wait_st();
     };
+    // S columns [c0, c0 + 64) of slot t_s into sr (only 16-column chunks below nk16)
+    auto load_s64 = [&](uint32_t t_s, int c0, int nk16, uint32_t (&sr)[64]) {
+#pragma unroll
+      for (int c16 = 0; c16 < 64; c16 += 16)
+        if (c0 + c16 < nk16) tc::tmem_ld16(t_s + c0 + c16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c16]));
+      tc::tmem_wait_ld();
+    };
 
     bool ok = true;
     int item = blockIdx.x;
-    if (item < n_items && item_nqt(item) <= qt) item = next_item(item);
     float qmul = 1.0f;  // 2^eq of the current item's row
     if (item < n_items) {
       if constexpr (C::STAGE_Q) stage_q(item);
       qmul = convert_q(item);
     }
-    int n = 0;  // tiles of this query tile so far (S/P slot counter)
+    int g = 0;  // tiles so far (S/P slot counter)
     bool epi = false;
     int epi_item = 0;
     float epi_l = 1.0f, epi_vmul = 1.0f;
     bool epi_active = false;
+    constexpr float kLog2e = 1.4426950408889634f;
     while (ok && item < n_items) {
-      const int nxt = next_item(item);
-      const int gt0 = ((item - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x)) * T;
+      const int nxt = item + gridDim.x;
       const bool warp_active = __any_sync(0xffffffffu, row_of(item) < p.n_q);
       if constexpr (C::STAGE_Q) {
         if (nxt < n_items) stage_q(nxt);
       }
       float up = 0.0f, vmul = 1.0f, m_ref = -INFINITY, l = 0.0f, qmul_next = qmul;
-      int kb = 0, t0 = 0;
-      for (int j = 0; j < T; ++j, ++n) {
-        const int nk = min(KT, p.blk[kb].n - t0);
+      Walk w;
+      w.reset();
+      for (int j = 0; j < T; ++j, ++g) {
+        const int nk = w.next(p);
         const int nk16 = (nk + 15) & ~15;
-        const int slot = n % NS;
-        if (!(ok = mbar_wait_bounded(s_full(qt, slot), (n / NS) & 1))) break;
+        const int slot = g % NS;
+        if (!(ok = mbar_wait_bounded(&s_full[slot], (g / NS) & 1))) break;
         tc::fence_after_sync();
         if (j == 0) {
-          // the unpack warpgroup's powers of two for this item (header of its first tile)
-          const int g = gt0;
+          // the unpack warps' powers of two for this item (header of its first tile)
           if (!(ok = mbar_wait_bounded(&kv_full[g % NKV], (g / NKV) & 1))) break;
           up = p.softmax_scale * qmul * hdr[(g % NKV) * 4 + 0];
           vmul = hdr[(g % NKV) * 4 + 1];
@@ -626,16 +645,19 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         // last QK^T of this item has completed: q of the next item can replace it
         if (j == T - 1 && nxt < n_items) qmul_next = convert_q(nxt);
         if (warp_active) {
-          const uint32_t t_s = tq + slot * 64;
-          uint32_t sr[KT];
-#pragma unroll
-          for (int c16 = 0; c16 < KT; c16 += 16)
-            if (c16 < nk16) tc::tmem_ld16(t_s + c16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c16]));
-          tc::tmem_wait_ld();
+          const uint32_t t_s = tq + slot * KT;
+          uint32_t sr[64];
+          // pass 1: the tile's row maximum
           float smax = -INFINITY;
 #pragma unroll
-          for (int k = 0; k < KT; ++k)
-            if (k < nk) smax = fmaxf(smax, __uint_as_float(sr[k]));
+          for (int c0 = 0; c0 < KT; c0 += 64) {
+            if (c0 < nk16) {
+              load_s64(t_s, c0, nk16, sr);
+#pragma unroll
+              for (int k = 0; k < 64; ++k)
+                if (c0 + k < nk) smax = fmaxf(smax, __uint_as_float(sr[k]));
+            }
+          }
           const float mx = smax * up;
           float alpha = 1.0f;
           bool rescale = false;
@@ -648,46 +670,52 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           }
           l *= alpha;
           if (__any_sync(0xffffffffu, rescale)) {
-            // O holds PV up to tile n-1 of this item once that PV completes
-            if (!(ok = mbar_wait_bounded(pv_done(qt, (n - 1) % NS), ((n - 1) / NS) & 1))) break;
+            // O holds PV up to tile g-1 once that PV completes
+            if (!(ok = mbar_wait_bounded(&pv_done[(g - 1) % NS], ((g - 1) / NS) & 1))) break;
             tc::fence_after_sync();
             scale_o(alpha);
           }
-          constexpr float kLog2e = 1.4426950408889634f;
           const float up2 = up * kLog2e;
           const float c2 = -m_ref * kLog2e;
           const uint64_t up2x2 = tc::f2pack(up2, up2);
           const uint64_t c2x2 = tc::f2pack(c2, c2);
-          const bool partial = nk < nk16;
           uint64_t rs2 = tc::f2pack(0.0f, 0.0f);
+          // pass 2: P = 2^(S up log2e - m log2e), hi/lo in place over S, 64 keys at a time
 #pragma unroll
-          for (int c8 = 0; c8 < KT; c8 += 8) {
-            if (c8 < nk16) {
-              // keys c8..c8+7: P hi -> columns (c8 / 16) * 16 + c8 % 16 / 2 + 0..3, lo 8 further
-              uint32_t hi[4], lo[4];
+          for (int c0 = 0; c0 < KT; c0 += 64) {
+            if (c0 < nk16) {
+              if (KT > 64) load_s64(t_s, c0, nk16, sr);  // (KT == 64: still in sr from pass 1)
+              const bool partial = c0 + 64 > nk;
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int j0 = c8 + 2 * u;
-                const uint64_t arg =
-                    tc::fma2(tc::f2pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), up2x2, c2x2);
-                float p0 = tc::ex2(tc::f2lo(arg));
-                float p1 = tc::ex2(tc::f2hi(arg));
-                if (partial) {
-                  p0 = (j0 < nk) ? p0 : 0.0f;
-                  p1 = (j0 + 1 < nk) ? p1 : 0.0f;
+              for (int c8 = 0; c8 < 64; c8 += 8) {
+                if (c0 + c8 < nk16) {
+                  uint32_t hi[4], lo[4];
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    const int j0 = c8 + 2 * u;
+                    const uint64_t arg = tc::fma2(
+                        tc::f2pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), up2x2, c2x2);
+                    float p0 = tc::ex2(tc::f2lo(arg));
+                    float p1 = tc::ex2(tc::f2hi(arg));
+                    if (partial) {
+                      p0 = (c0 + j0 < nk) ? p0 : 0.0f;
+                      p1 = (c0 + j0 + 1 < nk) ? p1 : 0.0f;
+                    }
+                    const uint64_t pp = tc::f2pack(p0, p1);
+                    const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
+                    const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
+                    const uint64_t lo2 = tc::sub2(pp, tc::f2pack(h0, h1));
+                    rs2 = tc::add2(rs2, pp);
+                    hi[u] = tc::cvt_half2(h0, h1);
+                    lo[u] = tc::cvt_half2(tc::f2lo(lo2), tc::f2hi(lo2));
+                  }
+                  // keys c0+c8..+7: P hi at columns (key / 16) * 16 + (key % 16) / 2, lo 8 further
+                  const int key = c0 + c8;
+                  const uint32_t col = (key & ~15) + (key & 15) / 2;
+                  tc::tmem_st4(t_s + col, hi);
+                  tc::tmem_st4(t_s + col + 8, lo);
                 }
-                const uint64_t pp = tc::f2pack(p0, p1);
-                const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
-                const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
-                const uint64_t lo2 = tc::sub2(pp, tc::f2pack(h0, h1));
-                rs2 = tc::add2(rs2, pp);
-                hi[u] = pipe_h2(h0, h1);
-                lo[u] = pipe_h2(tc::f2lo(lo2), tc::f2hi(lo2));
               }
-              // S of this row is in registers: P hi and lo replace it in place
-              const uint32_t col = (c8 & ~15) + (c8 & 15) / 2;
-              tc::tmem_st4(t_s + col, hi);
-              tc::tmem_st4(t_s + col + 8, lo);
             }
           }
           tc::tmem_wait_st();
@@ -698,19 +726,14 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         if (j == 0 && epi) {
           epi = false;
           if (epi_active) {
-            if (!(ok = mbar_wait_bounded(pv_done(qt, (n - 1) % NS), ((n - 1) / NS) & 1))) break;
+            if (!(ok = mbar_wait_bounded(&pv_done[(g - 1) % NS], ((g - 1) / NS) & 1))) break;
             tc::fence_after_sync();
             epilogue(epi_item, epi_l, epi_vmul);
           }
         }
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full(qt, slot));
-        t0 += KT;
-        if (t0 >= p.blk[kb].n) {
-          ++kb;
-          t0 = 0;
-        }
+        if (lane == 0) mbar_arrive(&p_full[slot]);
       }
       if (!ok) break;
       epi = true;
@@ -722,7 +745,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       item = nxt;
     }
     if (ok && epi && epi_active) {
-      if (mbar_wait_bounded(pv_done(qt, (n - 1) % NS), ((n - 1) / NS) & 1)) {
+      if (mbar_wait_bounded(&pv_done[(g - 1) % NS], ((g - 1) / NS) & 1)) {
         tc::fence_after_sync();
         epilogue(epi_item, epi_l, epi_vmul);
       }
@@ -736,36 +759,33 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   if (warp == 0) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int BITS, int D, int NQT>
+template <int BITS, int D>
 cudaError_t launch_attention_pipe(const AttnParams& p, cudaStream_t stream) {
-  using C = PipeCfg<BITS, D, NQT>;
+  using C = PipeCfg<BITS, D>;
   static bool configured[kMaxDevices] = {};
-  static int ctas_per_sm[kMaxDevices] = {};
   static int sms[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(attention_pipe_kernel<BITS, D, NQT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(attention_pipe_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm[dev], attention_pipe_kernel<BITS, D, NQT>,
-                                                      C::THREADS, C::SMEM_ALLOC);
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attention_pipe_kernel<BITS, D>, C::THREADS,
+                                                      C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    if (ctas_per_sm[dev] < 1) return cudaErrorInvalidConfiguration;
-    // tensor memory: at most 512 columns per SM
-    ctas_per_sm[dev] = min(ctas_per_sm[dev], 512 / C::TMEM_COLS);
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
     configured[dev] = true;
   }
-  const int n_qt = (p.n_q + 127) / 128;
-  const int64_t n_items = static_cast<int64_t>(p.B) * p.H * ((n_qt + NQT - 1) / NQT);
+  const int64_t n_items = static_cast<int64_t>(p.B) * p.H * ((p.n_q + 127) / 128);
   if (n_items > (int64_t(1) << 30)) return cudaErrorInvalidConfiguration;
-  const int64_t slots = static_cast<int64_t>(sms[dev]) * ctas_per_sm[dev];
-  const int grid = static_cast<int>(n_items < slots ? n_items : slots);
-  attention_pipe_kernel<BITS, D, NQT><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(p);
+  // one CTA per SM: all 512 tensor-memory columns are this CTA's
+  const int grid = static_cast<int>(n_items < sms[dev] ? n_items : sms[dev]);
+  attention_pipe_kernel<BITS, D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(p);
   return cudaGetLastError();
 }
 
