@@ -447,37 +447,49 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
           const float* meta =
               reinterpret_cast<const float*>(stage + C::STG_META) + (i * 4 + 2 * tsel) * D + 8 * jj;
           const float mul = tsel ? vinv : kinv;
-          uint64_t sc2[4], ze2[4];
+          float sc[8], ze[8];  // scale and zero of the 8 channels, times 2^-e (exact)
+          {
+            const uint4 s0 = *reinterpret_cast<const uint4*>(meta + 4 * sw);
+            const uint4 s1 = *reinterpret_cast<const uint4*>(meta + 4 * (sw ^ 1));
+            const uint4 z0 = *reinterpret_cast<const uint4*>(meta + D + 4 * sw);
+            const uint4 z1 = *reinterpret_cast<const uint4*>(meta + D + 4 * (sw ^ 1));
+            const uint4 sa = sw ? s1 : s0, sb = sw ? s0 : s1;
+            const uint4 za = sw ? z1 : z0, zb = sw ? z0 : z1;
+            const uint32_t sv8[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+            const uint32_t zv8[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            sc2[u] = tc::f2pack(meta[2 * u] * mul, meta[2 * u + 1] * mul);
-            ze2[u] = tc::f2pack(meta[D + 2 * u] * mul, meta[D + 2 * u + 1] * mul);
+            for (int u = 0; u < 8; ++u) {
+              sc[u] = __uint_as_float(sv8[u]) * mul;
+              ze[u] = __uint_as_float(zv8[u]) * mul;
+            }
           }
-          const uint32_t dst = kvbase + tsel * 2 * C::TILE_SZ;
           // block token of slot 0 of this word row, and its tile key
           const int ub = (sg.y / CPW + (sr - rows[2 * i])) * CPW;
           const int kbase = sg.w + ub - sg.y;
-          const int ulo = sg.y - ub, uhi = sg.y + sg.z - ub;  // valid slots [ulo, uhi)
-          const uint64_t magic2 = tc::f2pack(-8388608.0f, -8388608.0f);
+          const int s_lo = max(0, sg.y - ub), s_hi = min(CPW, sg.y + sg.z - ub);  // valid slots
+          // key row r of the [KT][D] tile: byte r * 128 + ((octet ^ (r & 7)) << 4) in its 64-channel slab
+          const uint32_t dst = kvbase + tsel * 2 * C::TILE_SZ + (jj >> 3) * KT * 128;
+          const uint32_t oct = jj & 7;
+#pragma unroll 1
+          for (int s = s_lo; s < s_hi; ++s) {
+            const int sh = BITS * s;
+            const uint32_t row = static_cast<uint32_t>(kbase + s);
+            float h[8], l[8];
 #pragma unroll
-          for (int s = 0; s < CPW; ++s) {
-            if (s < ulo || s >= uhi) continue;
+            for (int u = 0; u < 8; ++u) {
+              // code c as the float 2^23 + c, minus 2^23: exact; then fma(c, scale, zero) * 2^-e
+              const float c = __uint_as_float(((wd[u] >> sh) & C::MASK) | 0x4B000000u) - 8388608.0f;
+              const float x = fmaf(c, sc[u], ze[u]);
+              h[u] = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
+              l[u] = x - h[u];
+            }
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              // code c as the float 2^23 + c, minus 2^23: exact
-              const uint32_t c0 = ((wd[2 * u] >> (BITS * s)) & C::MASK) | 0x4B000000u;
-              const uint32_t c1 = ((wd[2 * u + 1] >> (BITS * s)) & C::MASK) | 0x4B000000u;
-              const uint64_t cf = tc::add2(tc::f2pack(__uint_as_float(c0), __uint_as_float(c1)), magic2);
-              const uint64_t x = tc::fma2(cf, sc2[u], ze2[u]);  // fma(code, scale, zero) * 2^-e
-              const float x0 = tc::f2lo(x), x1 = tc::f2hi(x);
-              const float h0 = __uint_as_float(__float_as_uint(x0) & 0xffffe000u);
-              const float h1 = __uint_as_float(__float_as_uint(x1) & 0xffffe000u);
-              const uint64_t l2 = tc::sub2(x, tc::f2pack(h0, h1));
-              hi[u] = tc::cvt_half2(h0, h1);
-              lo[u] = tc::cvt_half2(tc::f2lo(l2), tc::f2hi(l2));
+              hi[u] = tc::cvt_half2(h[2 * u], h[2 * u + 1]);
+              lo[u] = tc::cvt_half2(l[2 * u], l[2 * u + 1]);
             }
-            const uint32_t off = tc::sw128_offset(kbase + s, 8 * jj, KT);
+            const uint32_t off = row * 128 + ((oct ^ (row & 7)) << 4);
             tc::sts128(dst + off, hi[0], hi[1], hi[2], hi[3]);
             tc::sts128(dst + C::TILE_SZ + off, lo[0], lo[1], lo[2], lo[3]);
           }
@@ -600,12 +612,18 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
       }
       tc::tmem_wait_st();
     };
-    // S columns [c0, c0 + 64) of slot t_s into sr (only 16-column chunks below nk16)
-    auto load_s64 = [&](uint32_t t_s, int c0, int nk16, uint32_t (&sr)[64]) {
+    // S columns [c0, c0 + 64) of slot t_s into sr: 16-column chunks below nk16
+    // are loaded, columns from nk on read as -inf
+    auto load_s64 = [&](uint32_t t_s, int c0, int nk16, uint32_t (&sr)[64], int nk) {
 #pragma unroll
       for (int c16 = 0; c16 < 64; c16 += 16)
         if (c0 + c16 < nk16) tc::tmem_ld16(t_s + c0 + c16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c16]));
       tc::tmem_wait_ld();
+      if (c0 + 64 > nk) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if (c0 + k >= nk) sr[k] = 0xff800000u;
+      }
     };
 
     bool ok = true;
@@ -647,15 +665,19 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
         if (warp_active) {
           const uint32_t t_s = tq + slot * KT;
           uint32_t sr[64];
-          // pass 1: the tile's row maximum
+          // pass 1: the tile's row maximum. Columns past nk (within the last
+          // 16-column chunk) are set to -inf, which the maximum ignores and
+          // pass 2 turns into p = 0.
           float smax = -INFINITY;
-#pragma unroll
+#pragma unroll 1
           for (int c0 = 0; c0 < KT; c0 += 64) {
             if (c0 < nk16) {
-              load_s64(t_s, c0, nk16, sr);
+              load_s64(t_s, c0, nk16, sr, nk);
 #pragma unroll
-              for (int k = 0; k < 64; ++k)
-                if (c0 + k < nk) smax = fmaxf(smax, __uint_as_float(sr[k]));
+              for (int k = 0; k < 64; k += 4)
+                smax = tc::max3(smax, tc::max3(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1]),
+                                               __uint_as_float(sr[k + 2])),
+                                __uint_as_float(sr[k + 3]));
             }
           }
           const float mx = smax * up;
@@ -677,37 +699,29 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
           }
           const float up2 = up * kLog2e;
           const float c2 = -m_ref * kLog2e;
-          const uint64_t up2x2 = tc::f2pack(up2, up2);
-          const uint64_t c2x2 = tc::f2pack(c2, c2);
-          uint64_t rs2 = tc::f2pack(0.0f, 0.0f);
-          // pass 2: P = 2^(S up log2e - m log2e), hi/lo in place over S, 64 keys at a time
-#pragma unroll
+          float rs = 0.0f;
+          // pass 2: p = 2^(S up log2e - m log2e); hi = p cut to 10 mantissa bits,
+          // lo = p - hi; both as fp16 pairs in place over S, 64 keys at a time
+#pragma unroll 1
           for (int c0 = 0; c0 < KT; c0 += 64) {
             if (c0 < nk16) {
-              if (KT > 64) load_s64(t_s, c0, nk16, sr);  // (KT == 64: still in sr from pass 1)
-              const bool partial = c0 + 64 > nk;
+              if (KT > 64) load_s64(t_s, c0, nk16, sr, nk);  // (KT == 64: still in sr from pass 1)
 #pragma unroll
               for (int c8 = 0; c8 < 64; c8 += 8) {
                 if (c0 + c8 < nk16) {
+                  float ph[8], pl[8];
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) {
+                    const float pv = tc::ex2(fmaf(__uint_as_float(sr[c8 + u]), up2, c2));
+                    ph[u] = __uint_as_float(__float_as_uint(pv) & 0xffffe000u);
+                    pl[u] = pv - ph[u];
+                    rs += pv;
+                  }
                   uint32_t hi[4], lo[4];
 #pragma unroll
                   for (int u = 0; u < 4; ++u) {
-                    const int j0 = c8 + 2 * u;
-                    const uint64_t arg = tc::fma2(
-                        tc::f2pack(__uint_as_float(sr[j0]), __uint_as_float(sr[j0 + 1])), up2x2, c2x2);
-                    float p0 = tc::ex2(tc::f2lo(arg));
-                    float p1 = tc::ex2(tc::f2hi(arg));
-                    if (partial) {
-                      p0 = (c0 + j0 < nk) ? p0 : 0.0f;
-                      p1 = (c0 + j0 + 1 < nk) ? p1 : 0.0f;
-                    }
-                    const uint64_t pp = tc::f2pack(p0, p1);
-                    const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
-                    const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
-                    const uint64_t lo2 = tc::sub2(pp, tc::f2pack(h0, h1));
-                    rs2 = tc::add2(rs2, pp);
-                    hi[u] = tc::cvt_half2(h0, h1);
-                    lo[u] = tc::cvt_half2(tc::f2lo(lo2), tc::f2hi(lo2));
+                    hi[u] = tc::cvt_half2(ph[2 * u], ph[2 * u + 1]);
+                    lo[u] = tc::cvt_half2(pl[2 * u], pl[2 * u + 1]);
                   }
                   // keys c0+c8..+7: P hi at columns (key / 16) * 16 + (key % 16) / 2, lo 8 further
                   const int key = c0 + c8;
@@ -719,7 +733,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
             }
           }
           tc::tmem_wait_st();
-          l += tc::f2lo(rs2) + tc::f2hi(rs2);
+          l += rs;
         }
         // the previous item's output, once its last PV is done (before this
         // item's first PV overwrites O)
