@@ -4,7 +4,7 @@
 // The queries of block s attend to every cached token of blocks 0..s.
 //
 // Operands. The cached tokens of blocks 0..s are walked as one sequence, in
-// key tiles of KT = 8192 / D tokens (128 at head_dim 64, 64 at 128) that may
+// key tiles of KT tokens (64 at head_dim 64, 48 at 128) that may
 // span several blocks (at most MAXSEG block segments per tile). Each tile is
 // dequantized in shared memory to the cache's own fp32 values
 // x^ = fma(code, scale, zero) of each token's block, times a power of two 2^-e
@@ -20,22 +20,26 @@
 // tensor memory over S. The dropped Plo . V^lo term is below 2^-20 of O. The
 // scales live in the operands, so O collects every block directly.
 //
-// Roles of one CTA (one CTA per SM, 448 threads):
-//   softmax warps 0-3 (one query row per thread, tensor-memory lanes 0-127):
-//     query load and conversion, online softmax with a lazy reference maximum
-//     (O is rescaled in tensor memory only when a row maximum grows by more
-//     than kPipeTau), normalisation and output;
-//   unpack warps 4-11: staged packed words -> dequantized fp16 hi/lo K and V
-//     tiles (ring of NKV slots), and the per-(batch, head) powers of two;
-//   producer warp 12, one thread: bulk copies of each tile's packed K/V word
+// Roles of one CTA (one CTA per SM, 448 threads, NQT = 1 or 2 query tiles of
+// 128 rows of one (batch, head) per work item):
+//   one softmax warpgroup per query tile (one query row per thread,
+//     tensor-memory lanes 0-127 of that tile's columns): query load and
+//     conversion, online softmax with a lazy reference maximum (O is rescaled
+//     in tensor memory only when a row maximum grows by more than kPipeTau),
+//     normalisation and output. With two query tiles the two warpgroups take
+//     turns on the tensor cores and hide each other's tensor-memory latency;
+//   unpack warps (8 with one query tile, 4 with two): staged packed words ->
+//     dequantized fp16 hi/lo K and V tiles (ring of NKV slots) shared by the
+//     item's query tiles, and the per-(batch, head) powers of two;
+//   producer warp, one thread: bulk copies of each tile's packed K/V word
 //     rows and of its blocks' scale/zero vectors into a stage ring;
-//   MMA warp 13, one thread: every tcgen05.mma, with shared-memory descriptors
-//     built once and advanced by constant offsets: QK^T of tile g, then PV of
-//     tile g-1.
-// The CTA is persistent: it walks work items (batch*head, 128-query tile)
-// with a stride of gridDim.x. Every ring runs on across items, so the next
-// item's copies, unpacking and first QK^T overlap this item's last tiles, and
-// an item's output is written while the next item's first softmax is done.
+//   MMA warp, one thread: every tcgen05.mma, with shared-memory descriptors
+//     built once and advanced by constant offsets: QK^T of tile g for each
+//     query tile, then PV of tile g-1 for each.
+// The CTA is persistent: it walks work items (batch*head, group of NQT query
+// tiles) with a stride of gridDim.x. Every ring runs on across items, so the
+// next item's copies, unpacking and first QK^T overlap this item's last tiles,
+// and an item's output is written while the next item's first softmax is done.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -52,53 +56,57 @@ namespace {
 
 constexpr float kPipeTau = 8.0f;  // lazy-rescale threshold (natural-log units); p <= e^8 fits fp16
 
-template <int BITS, int D>
+template <int BITS, int D, int NQT>
 struct PipeCfg {
-  static constexpr int KT = 8192 / D;                      // keys per tile
+  static constexpr int KT = (D == 64) ? 64 : 48;           // keys per tile: S of a row fits in registers
   static constexpr int CPW = 32 / BITS;
   static constexpr uint32_t MASK = (1u << BITS) - 1u;
   static constexpr int MAXSEG = (D == 64) ? 8 : 4;         // block segments per tile
   static constexpr int MAXROWS = (KT + CPW - 1) / CPW + 2 * MAXSEG;  // staged word rows per tensor
-  static constexpr int NS = (D == 64) ? 3 : 4;             // S slots (tensor memory)
-  static constexpr int NKV = 2;                            // dequantized K/V tile slots
+  static constexpr int TM_QT = 512 / NQT;                  // tensor-memory columns per query tile
+  static constexpr int NS = (NQT == 1) ? 4 : ((D == 64) ? 3 : 2);  // S slots per query tile
+  static constexpr int NKV = (D == 64) ? (NQT == 1 ? 4 : 3) : (NQT == 1 ? 3 : 2);  // K/V tile slots
   static constexpr int NSTG = 2;                           // packed-word stages
   static constexpr bool STAGE_Q = (D == 64);               // next item's queries prefetched by cp.async
-  static constexpr int UNPACK_WARPS = 8;
+  static constexpr int UNPACK_WARPS = (NQT == 1) ? 8 : 4;
   static constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
-  static constexpr int UNPACK_T0 = 128;
-  static constexpr int PROD_WARP = 12;
-  static constexpr int MMA_WARP = 13;
-  static constexpr int THREADS = 448;
+  static constexpr int UNPACK_T0 = NQT * 128;
+  static constexpr int PROD_WARP = (NQT * 128 + UNPACK_THREADS) / 32;
+  static constexpr int MMA_WARP = PROD_WARP + 1;
+  static constexpr int THREADS = (MMA_WARP + 1) * 32;
   // ---- shared memory (byte offsets from a 1024-aligned base)
-  static constexpr int Q_SZ = 128 * D * 2;                 // fp16 q [128][D], K-major SW128
+  static constexpr int Q_SZ = 128 * D * 2;                 // fp16 q [128][D] per query tile, K-major SW128
   static constexpr int Q0 = 0;
   static constexpr int TILE_SZ = KT * D * 2;               // fp16 [KT][D], K-major SW128
-  static constexpr int KV0 = Q0 + Q_SZ;                    // NKV x {K hi, K lo, V hi, V lo}
+  static constexpr int KV0 = Q0 + NQT * Q_SZ;              // NKV x {K hi, K lo, V hi, V lo}
   static constexpr int KV_SZ = 4 * TILE_SZ;
-  static constexpr int QST0 = KV0 + NKV * KV_SZ;           // bf16 [128][D] query staging
+  static constexpr int QST0 = KV0 + NKV * KV_SZ;           // bf16 [128][D] query staging per query tile
   static constexpr int QST_SZ = STAGE_Q ? 128 * D * 2 : 0;
-  static constexpr int STG0 = QST0 + QST_SZ;               // NSTG x {K rows, V rows, meta, segment table}
+  static constexpr int STG0 = QST0 + NQT * QST_SZ;         // NSTG x {K rows, V rows, meta, segment table}
   static constexpr int STG_V = MAXROWS * D * 4;
   static constexpr int STG_META = 2 * STG_V;               // MAXSEG x [4][D] fp32: sk, zk, sv, zv
   static constexpr int STG_SEG = STG_META + MAXSEG * 4 * D * 4;  // MAXSEG x int4 {block, u0, take, key0}
   static constexpr int STG_ROWS = STG_SEG + MAXSEG * 16;   // MAXSEG x {first staged row, rows}, segment count
   static constexpr int STG_SZ = STG_ROWS + (2 * MAXSEG + 4) * 4;
   static constexpr int HDR0 = STG0 + NSTG * STG_SZ;        // NKV x {2^eK, 2^eV, -, -}
-  static constexpr int NRED = 4;                           // exponent reduction slots (> NKV)
+  static constexpr int NRED = 5;                           // exponent reduction slots (> NKV)
   static constexpr int RED0 = HDR0 + NKV * 16;             // NRED x {K, V} x UNPACK_WARPS floats
   static constexpr int BARS = RED0 + NRED * 2 * UNPACK_WARPS * 4;
-  static constexpr int NBARS = 2 * NSTG + 2 * NKV + NRED + 1 + 3 * NS;
+  static constexpr int QBARS = 1 + 3 * NS;                 // per query tile: q_full, s_full, p_full, pv_done
+  static constexpr int NBARS = 2 * NSTG + 2 * NKV + NRED + NQT * QBARS;
   static constexpr int TMEM_SLOT = BARS + NBARS * 8;
   static constexpr int SMEM = TMEM_SLOT + 16;
   static constexpr int SMEM_ALLOC = SMEM + 1024;           // room to align the base
+  static_assert(THREADS == 448, "one CTA per SM at 128 registers per thread");
   static_assert(KV0 % 1024 == 0 && TILE_SZ % 1024 == 0 && Q_SZ % 1024 == 0, "operand alignment");
   static_assert(STG0 % 16 == 0 && STG_SZ % 16 == 0 && STG_V % 16 == 0 && STG_META % 16 == 0, "stage alignment");
   static_assert(HDR0 % 16 == 0 && BARS % 8 == 0, "header alignment");
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
-  // ---- tensor memory: NS S slots of KT columns, then O (D columns)
+  static_assert(NRED > NKV, "exponent slots");
+  // ---- tensor memory: query tile qt owns columns [qt * TM_QT, +TM_QT): NS S slots of KT columns, then O
   static constexpr int COL_O = NS * KT;
   static constexpr int TMEM_COLS = 512;
-  static_assert(NS * KT + D <= TMEM_COLS, "tensor memory");
+  static_assert(NS * KT + D <= TM_QT, "tensor memory");
 };
 
 // 16-byte asynchronous copy global -> shared (L2 only); src_bytes = 0 fills zeros.
@@ -148,9 +156,10 @@ struct PipeWalk {
   }
 };
 
-template <int BITS, int D>
-__global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_kernel(const __grid_constant__ AttnParams p) {
-  using C = PipeCfg<BITS, D>;
+template <int BITS, int D, int NQT>
+__global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
+    attention_pipe_kernel(const __grid_constant__ AttnParams p) {
+  using C = PipeCfg<BITS, D, NQT>;
   constexpr int CPW = C::CPW;
   constexpr int KT = C::KT;
   constexpr int NS = C::NS;
@@ -167,10 +176,11 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
   uint64_t* kv_full = stg_empty + NSTG;
   uint64_t* kv_empty = kv_full + NKV;
   uint64_t* red_bar = kv_empty + NKV;
-  uint64_t* q_full = red_bar + C::NRED;
-  uint64_t* s_full = q_full + 1;
-  uint64_t* p_full = s_full + NS;
-  uint64_t* pv_done = p_full + NS;
+  uint64_t* qbars = red_bar + C::NRED;
+  auto q_full = [&](int qt) { return qbars + qt * C::QBARS; };
+  auto s_full = [&](int qt, int i) { return qbars + qt * C::QBARS + 1 + i; };
+  auto p_full = [&](int qt, int i) { return qbars + qt * C::QBARS + 1 + NS + i; };
+  auto pv_done = [&](int qt, int i) { return qbars + qt * C::QBARS + 1 + 2 * NS + i; };
   float* hdr = reinterpret_cast<float*>(sm + C::HDR0);
   float* red = reinterpret_cast<float*>(sm + C::RED0);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::TMEM_SLOT);
@@ -180,7 +190,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
   const int lane = tid & 31;
   const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
   const int n_qt = (p.n_q + 127) / 128;
-  const int n_items = p.B * p.H * n_qt;
+  const int n_groups = (n_qt + NQT - 1) / NQT;
+  const int n_items = p.B * p.H * n_groups;
+  auto item_nqt = [&](int item) { return min(NQT, n_qt - (item % n_groups) * NQT); };
   int T = 0;  // key tiles per item
   {
     Walk w;
@@ -206,11 +218,13 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
       mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < C::NRED; ++i) mbar_init(&red_bar[i], C::UNPACK_WARPS);
-    mbar_init(q_full, 4);
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&pv_done[i], 1);
+    for (int qt = 0; qt < NQT; ++qt) {
+      mbar_init(q_full(qt), 4);
+      for (int i = 0; i < NS; ++i) {
+        mbar_init(s_full(qt, i), 1);
+        mbar_init(p_full(qt, i), 4);
+        mbar_init(pv_done(qt, i), 1);
+      }
     }
     fence_barrier_init();
   }
@@ -232,7 +246,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
       bool ok = true;
       int g = 0;
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-        const int bh = item / n_qt;
+        const int bh = item / n_groups;
         Walk w;
         w.reset();
         for (int j = 0; j < T; ++j, ++g) {
@@ -282,10 +296,11 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
       const uint64_t qdesc = tc::sw128_desc(sbase + C::Q0);
       const uint64_t kdesc0 = tc::sw128_desc(sbase + C::KV0);
       const uint64_t vdesc0 = tc::sw128_desc_mn(sbase + C::KV0 + 2 * C::TILE_SZ, kLbo);
-      auto issue_qk = [&](int slot, int kvs, int nk16) {
+      auto issue_qk = [&](int qt, int slot, int kvs, int nk16) {
         const uint32_t idesc = tc::idesc_f16_f32(128, nk16);
+        const uint64_t qd = qdesc + static_cast<uint64_t>((qt * C::Q_SZ) >> 4);
         const uint64_t kd = kdesc0 + static_cast<uint64_t>((kvs * C::KV_SZ) >> 4);
-        const uint32_t d = tmem + slot * KT;
+        const uint32_t d = tmem + qt * C::TM_QT + slot * KT;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
 #pragma unroll
@@ -293,15 +308,15 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
             constexpr int kSlabA = 128 * 128, kSlabB = KT * 128;
             const uint32_t aoff = ((kk >> 2) * kSlabA + (kk & 3) * 32) >> 4;
             const uint32_t boff = (part * C::TILE_SZ + (kk >> 2) * kSlabB + (kk & 3) * 32) >> 4;
-            tc::mma_f16_ss(d, qdesc + aoff, kd + boff, idesc, (part == 0 && kk == 0) ? 0u : 1u);
+            tc::mma_f16_ss(d, qd + aoff, kd + boff, idesc, (part == 0 && kk == 0) ? 0u : 1u);
           }
         }
-        tc::commit(&s_full[slot]);
+        tc::commit(s_full(qt, slot));
       };
-      auto issue_pv = [&](int slot, int kvs, int nk16, bool first) {
+      auto issue_pv = [&](int qt, int slot, int kvs, int nk16, bool first) {
         const uint64_t vd = vdesc0 + static_cast<uint64_t>((kvs * C::KV_SZ) >> 4);
-        const uint32_t pa = tmem + slot * KT;
-        const uint32_t o = tmem + C::COL_O;
+        const uint32_t pa = tmem + qt * C::TM_QT + slot * KT;
+        const uint32_t o = tmem + qt * C::TM_QT + C::COL_O;
         const int nkk = nk16 / 16;
         // (A part, B part): (P hi, V hi), (P lo, V hi), (P hi, V lo)
 #pragma unroll
@@ -315,45 +330,82 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
                              (first && part == 0 && kk == 0) ? 0u : 1u);
           }
         }
-        tc::commit(&pv_done[slot]);
+        tc::commit(pv_done(qt, slot));
       };
 
       bool ok = true;
       bool prev = false, prev_first = false;
-      int prev_nk16 = 0;
-      int g = 0, iq = 0;
+      int prev_nk16 = 0, prev_nqt = 0, prev_kvs = 0;
+      int nq[NQT], iq[NQT], prev_n[NQT];  // per query tile: tiles so far, items so far, last tile
+#pragma unroll
+      for (int qt = 0; qt < NQT; ++qt) nq[qt] = iq[qt] = prev_n[qt] = 0;
+      int g = 0;
       for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        const int nqt = item_nqt(item);
         Walk w;
         w.reset();
         for (int j = 0; j < T; ++j, ++g) {
           const int nk = w.next(p);
           const int nk16 = (nk + 15) & ~15;
           const int kvs = g % NKV;
-          const int slot = g % NS;
           if (!(ok = mbar_wait_bounded(&kv_full[kvs], (g / NKV) & 1))) break;
-          if (j == 0 && !(ok = mbar_wait_bounded(q_full, iq++ & 1))) break;
-          if (g >= NS && !(ok = mbar_wait_bounded(&pv_done[slot], ((g / NS) - 1) & 1))) break;
-          tc::fence_after_sync();
-          issue_qk(slot, kvs, nk16);
+          if (j == 0) {
+#pragma unroll
+            for (int qt = 0; qt < NQT; ++qt)
+              if (qt < nqt && ok) ok = mbar_wait_bounded(q_full(qt), iq[qt]++ & 1);
+            if (!ok) break;
+          }
+#pragma unroll
+          for (int qt = 0; qt < NQT; ++qt) {
+            if (qt < nqt && ok) {
+              const int n = nq[qt];
+              const int slot = n % NS;
+              if (n >= NS) ok = mbar_wait_bounded(pv_done(qt, slot), ((n / NS) - 1) & 1);
+              if (ok) {
+                tc::fence_after_sync();
+                issue_qk(qt, slot, kvs, nk16);
+              }
+            }
+          }
+          if (!ok) break;
           if (prev) {
-            const int gp = g - 1;
-            if (!(ok = mbar_wait_bounded(&p_full[gp % NS], (gp / NS) & 1))) break;
-            tc::fence_after_sync();
-            issue_pv(gp % NS, gp % NKV, prev_nk16, prev_first);
-            tc::commit(&kv_empty[gp % NKV]);
+#pragma unroll
+            for (int qt = 0; qt < NQT; ++qt) {
+              if (qt < prev_nqt && ok) {
+                const int n = prev_n[qt];
+                ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1);
+                if (ok) {
+                  tc::fence_after_sync();
+                  issue_pv(qt, n % NS, prev_kvs, prev_nk16, prev_first);
+                }
+              }
+            }
+            if (!ok) break;
+            tc::commit(&kv_empty[prev_kvs]);
           }
           prev = true;
           prev_first = (j == 0);
           prev_nk16 = nk16;
+          prev_nqt = nqt;
+          prev_kvs = kvs;
+#pragma unroll
+          for (int qt = 0; qt < NQT; ++qt)
+            if (qt < nqt) prev_n[qt] = nq[qt]++;
         }
       }
       if (ok && prev) {
-        const int gp = g - 1;
-        if (mbar_wait_bounded(&p_full[gp % NS], (gp / NS) & 1)) {
-          tc::fence_after_sync();
-          issue_pv(gp % NS, gp % NKV, prev_nk16, prev_first);
-          tc::commit(&kv_empty[gp % NKV]);
+#pragma unroll
+        for (int qt = 0; qt < NQT; ++qt) {
+          if (qt < prev_nqt && ok) {
+            const int n = prev_n[qt];
+            ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1);
+            if (ok) {
+              tc::fence_after_sync();
+              issue_pv(qt, n % NS, prev_kvs, prev_nk16, prev_first);
+            }
+          }
         }
+        if (ok) tc::commit(&kv_empty[prev_kvs]);
       }
     }
   } else if (tid >= C::UNPACK_T0) {
@@ -366,7 +418,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
     // runs at most NKV - 1 tiles ahead of another, so NRED > NKV slots never
     // alias a slot that is still to be read.
     auto pow2_post = [&](int item, int k) {
-      const int bh = item / n_qt;
+      const int bh = item / n_groups;
       float ak = 0.0f, av = 0.0f;
       for (int idx = ut; idx < (p.s + 1) * D; idx += C::UNPACK_THREADS) {
         const int kb = idx / D;
@@ -502,15 +554,22 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
       }
     }
   } else {
-    // =========================================================== softmax warps
-    const int row = tid;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tq = tmem + lane_off;
-    const uint32_t qs = sbase + C::Q0;
-    const uint32_t qst = sbase + C::QST0;
-    auto row_of = [&](int item) { return (item % n_qt) * 128 + row; };
+    // =========================================================== softmax warpgroup qt
+    const int qt = tid >> 7;
+    const int row = tid & 127;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tq = tmem + lane_off + qt * C::TM_QT;
+    const uint32_t qs = sbase + C::Q0 + qt * C::Q_SZ;
+    const uint32_t qst = sbase + C::QST0 + qt * C::QST_SZ;
+    auto row_of = [&](int item) { return (item % n_groups) * NQT * 128 + qt * 128 + row; };
+    // next item of this CTA in which query tile qt holds queries
+    auto next_item = [&](int item) {
+      for (item += gridDim.x; item < n_items && item_nqt(item) <= qt; item += gridDim.x) {
+      }
+      return item;
+    };
     auto q_ptr = [&](int item) -> const uint16_t* {
-      const int bh = item / n_qt;
+      const int bh = item / n_groups;
       const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
       return p.q + b * p.q_sb + h * p.q_sh + static_cast<int64_t>(row_of(item)) * p.q_st;
     };
@@ -527,7 +586,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
     // Two passes over the row (maximum, then conversion), 8 values at a time.
     auto q_chunk = [&](int item, int c) -> uint4 {
       if constexpr (C::STAGE_Q) {
-        return lds128(sm + C::QST0 + (row * (D / 8) + (c ^ (row & 7))) * 16);
+        return lds128(sm + C::QST0 + qt * C::QST_SZ + (row * (D / 8) + (c ^ (row & 7))) * 16);
       } else {
         uint4 v = make_uint4(0, 0, 0, 0);
         if (row_of(item) < p.n_q) v = *reinterpret_cast<const uint4*>(q_ptr(item) + 8 * c);
@@ -559,13 +618,13 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(q_full);
+      if (lane == 0) mbar_arrive(q_full(qt));
       return mul;
     };
     auto epilogue = [&](int item, float l, float vmul) {
       const int r = row_of(item);
       const bool valid = r < p.n_q;
-      const int bh = item / n_qt;
+      const int bh = item / n_groups;
       const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
       const int64_t obase = b * p.o_sb + h * p.o_sh + static_cast<int64_t>(r) * p.o_st;
       const float scl = vmul / l;
@@ -628,19 +687,22 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
 
     bool ok = true;
     int item = blockIdx.x;
+    if (item < n_items && item_nqt(item) <= qt) item = next_item(item);
     float qmul = 1.0f;  // 2^eq of the current item's row
     if (item < n_items) {
       if constexpr (C::STAGE_Q) stage_q(item);
       qmul = convert_q(item);
     }
-    int g = 0;  // tiles so far (S/P slot counter)
+    int g = 0;  // tiles of this query tile so far (S/P slot counter)
     bool epi = false;
     int epi_item = 0;
     float epi_l = 1.0f, epi_vmul = 1.0f;
     bool epi_active = false;
     constexpr float kLog2e = 1.4426950408889634f;
     while (ok && item < n_items) {
-      const int nxt = item + gridDim.x;
+      const int nxt = next_item(item);
+      // this item's first tile in the CTA-wide tile sequence (K/V slot and header)
+      const int gt0 = ((item - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x)) * T;
       const bool warp_active = __any_sync(0xffffffffu, row_of(item) < p.n_q);
       if constexpr (C::STAGE_Q) {
         if (nxt < n_items) stage_q(nxt);
@@ -652,13 +714,13 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
         const int nk = w.next(p);
         const int nk16 = (nk + 15) & ~15;
         const int slot = g % NS;
-        if (!(ok = mbar_wait_bounded(&s_full[slot], (g / NS) & 1))) break;
+        if (!(ok = mbar_wait_bounded(s_full(qt, slot), (g / NS) & 1))) break;
         tc::fence_after_sync();
         if (j == 0) {
           // the unpack warps' powers of two for this item (header of its first tile)
-          if (!(ok = mbar_wait_bounded(&kv_full[g % NKV], (g / NKV) & 1))) break;
-          up = p.softmax_scale * qmul * hdr[(g % NKV) * 4 + 0];
-          vmul = hdr[(g % NKV) * 4 + 1];
+          if (!(ok = mbar_wait_bounded(&kv_full[gt0 % NKV], (gt0 / NKV) & 1))) break;
+          up = p.softmax_scale * qmul * hdr[(gt0 % NKV) * 4 + 0];
+          vmul = hdr[(gt0 % NKV) * 4 + 1];
         }
         // last QK^T of this item has completed: q of the next item can replace it
         if (j == T - 1 && nxt < n_items) qmul_next = convert_q(nxt);
@@ -693,7 +755,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
           l *= alpha;
           if (__any_sync(0xffffffffu, rescale)) {
             // O holds PV up to tile g-1 once that PV completes
-            if (!(ok = mbar_wait_bounded(&pv_done[(g - 1) % NS], ((g - 1) / NS) & 1))) break;
+            if (!(ok = mbar_wait_bounded(pv_done(qt, (g - 1) % NS), ((g - 1) / NS) & 1))) break;
             tc::fence_after_sync();
             scale_o(alpha);
           }
@@ -740,14 +802,14 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
         if (j == 0 && epi) {
           epi = false;
           if (epi_active) {
-            if (!(ok = mbar_wait_bounded(&pv_done[(g - 1) % NS], ((g - 1) / NS) & 1))) break;
+            if (!(ok = mbar_wait_bounded(pv_done(qt, (g - 1) % NS), ((g - 1) / NS) & 1))) break;
             tc::fence_after_sync();
             epilogue(epi_item, epi_l, epi_vmul);
           }
         }
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[slot]);
+        if (lane == 0) mbar_arrive(p_full(qt, slot));
       }
       if (!ok) break;
       epi = true;
@@ -759,7 +821,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
       item = nxt;
     }
     if (ok && epi && epi_active) {
-      if (mbar_wait_bounded(&pv_done[(g - 1) % NS], ((g - 1) / NS) & 1)) {
+      if (mbar_wait_bounded(pv_done(qt, (g - 1) % NS), ((g - 1) / NS) & 1)) {
         tc::fence_after_sync();
         epilogue(epi_item, epi_l, epi_vmul);
       }
@@ -773,9 +835,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D>::THREADS, 1) attention_pipe_k
   if (warp == 0) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int BITS, int D>
+template <int BITS, int D, int NQT>
 cudaError_t launch_attention_pipe(const AttnParams& p, cudaStream_t stream) {
-  using C = PipeCfg<BITS, D>;
+  using C = PipeCfg<BITS, D, NQT>;
   static bool configured[kMaxDevices] = {};
   static int sms[kMaxDevices] = {};
   int dev = 0;
@@ -783,23 +845,24 @@ cudaError_t launch_attention_pipe(const AttnParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(attention_pipe_kernel<BITS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(attention_pipe_kernel<BITS, D, NQT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attention_pipe_kernel<BITS, D>, C::THREADS,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attention_pipe_kernel<BITS, D, NQT>, C::THREADS,
                                                       C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     configured[dev] = true;
   }
-  const int64_t n_items = static_cast<int64_t>(p.B) * p.H * ((p.n_q + 127) / 128);
+  const int n_qt = (p.n_q + 127) / 128;
+  const int64_t n_items = static_cast<int64_t>(p.B) * p.H * ((n_qt + NQT - 1) / NQT);
   if (n_items > (int64_t(1) << 30)) return cudaErrorInvalidConfiguration;
   // one CTA per SM: all 512 tensor-memory columns are this CTA's
   const int grid = static_cast<int>(n_items < sms[dev] ? n_items : sms[dev]);
-  attention_pipe_kernel<BITS, D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(p);
+  attention_pipe_kernel<BITS, D, NQT><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(p);
   return cudaGetLastError();
 }
 
