@@ -192,7 +192,7 @@ def blas_threads():
         return 1
 
 
-def cpu_sample(w, bits, budget_s=15.0, max_units=64):
+def cpu_sample(w, bits, budget_s=15.0, max_units=4096):
     """Time the oracle on (b, h) units of layer 0 until ~budget_s; return
     (tokens_per_s scaled to the whole step, units, seconds)."""
     k, v = _small_kv(w)

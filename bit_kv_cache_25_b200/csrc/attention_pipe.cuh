@@ -54,7 +54,9 @@
 namespace vq {
 namespace {
 
-constexpr float kPipeTau = 8.0f;  // lazy-rescale threshold (natural-log units); p <= e^8 fits fp16
+constexpr float kPipeTau = 10.5f;  // lazy-rescale threshold (natural-log units): p <= e^10.5 < 2^16 fits fp16
+constexpr float kPipeHead = 2.5f;  // an item's first reference maximum sits this far above its first tile's
+constexpr int kPipeMaxTable = 4096;  // tiles per item whose key counts are tabled in shared memory
 
 template <int BITS, int D, int NQT>
 struct PipeCfg {
@@ -95,7 +97,8 @@ struct PipeCfg {
   static constexpr int QBARS = 1 + 3 * NS;                 // per query tile: q_full, s_full, p_full, pv_done
   static constexpr int NBARS = 2 * NSTG + 2 * NKV + NRED + NQT * QBARS;
   static constexpr int TMEM_SLOT = BARS + NBARS * 8;
-  static constexpr int SMEM = TMEM_SLOT + 16;
+  static constexpr int NKTAB = TMEM_SLOT + 16;             // kPipeMaxTable x uint8: keys of each tile of an item
+  static constexpr int SMEM = NKTAB + kPipeMaxTable;
   static constexpr int SMEM_ALLOC = SMEM + 1024;           // room to align the base
   static_assert(THREADS == 448, "one CTA per SM at 128 registers per thread");
   static_assert(KV0 % 1024 == 0 && TILE_SZ % 1024 == 0 && Q_SZ % 1024 == 0, "operand alignment");
@@ -193,15 +196,21 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   const int n_groups = (n_qt + NQT - 1) / NQT;
   const int n_items = p.B * p.H * n_groups;
   auto item_nqt = [&](int item) { return min(NQT, n_qt - (item % n_groups) * NQT); };
-  int T = 0;  // key tiles per item
+  // key tiles per item (the same for every item), and the key count of each
+  // of the first kPipeMaxTable tiles in shared memory (thread 0 writes it; the
+  // set-up barrier below publishes it)
+  uint8_t* nktab = sm + C::NKTAB;
+  int T = 0;
   {
     Walk w;
     w.reset();
     while (w.kb <= p.s) {
-      w.next(p);
+      const int nk = w.next(p);
+      if (tid == 0 && T < kPipeMaxTable) nktab[T] = static_cast<uint8_t>(nk);
       ++T;
     }
   }
+  const bool tabled = T <= kPipeMaxTable;
 
   // ---- set-up: TMEM (warp 0), barriers (thread 0), zeroed K/V slots (unpack warps)
   if (warp == 0) {
@@ -327,7 +336,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           for (int kk = 0; kk < KT / 16; ++kk) {
             if (kk < nkk)
               tc::mma_f16_ts(o, pa + 16 * kk + acol, vd + vpart + ((kk * 2048) >> 4), idesc_pv,
-                             (first && part == 0 && kk == 0) ? 0u : 1u);
+                                (first && part == 0 && kk == 0) ? 0u : 1u);
           }
         }
         tc::commit(pv_done(qt, slot));
@@ -345,7 +354,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         Walk w;
         w.reset();
         for (int j = 0; j < T; ++j, ++g) {
-          const int nk = w.next(p);
+          const int nk = tabled ? nktab[j] : w.next(p);
           const int nk16 = (nk + 15) & ~15;
           const int kvs = g % NKV;
           if (!(ok = mbar_wait_bounded(&kv_full[kvs], (g / NKV) & 1))) break;
@@ -420,13 +429,28 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     auto pow2_post = [&](int item, int k) {
       const int bh = item / n_groups;
       float ak = 0.0f, av = 0.0f;
-      for (int idx = ut; idx < (p.s + 1) * D; idx += C::UNPACK_THREADS) {
-        const int kb = idx / D;
-        const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + (idx - kb * D);
-        const float sk = __ldg(p.scale_k + mo), zk = __ldg(p.zero_k + mo);
-        const float sv = __ldg(p.scale_v + mo), zv = __ldg(p.zero_v + mo);
-        ak = fmaxf(ak, fmaxf(fabsf(zk), fabsf(fmaf(cmax, sk, zk))));
-        av = fmaxf(av, fmaxf(fabsf(zv), fabsf(fmaf(cmax, sv, zv))));
+      // up to kPow2Batch (block, channel) pairs per thread in flight at once
+      constexpr int kPow2Batch = 8;
+      for (int base = 0; base < (p.s + 1) * D; base += kPow2Batch * C::UNPACK_THREADS) {
+        float sk[kPow2Batch], zk[kPow2Batch], sv[kPow2Batch], zv[kPow2Batch];
+#pragma unroll
+        for (int u = 0; u < kPow2Batch; ++u) {
+          const int idx = base + u * C::UNPACK_THREADS + ut;
+          sk[u] = zk[u] = sv[u] = zv[u] = 0.0f;
+          if (idx < (p.s + 1) * D) {
+            const int kb = idx / D;
+            const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + (idx - kb * D);
+            sk[u] = __ldg(p.scale_k + mo);
+            zk[u] = __ldg(p.zero_k + mo);
+            sv[u] = __ldg(p.scale_v + mo);
+            zv[u] = __ldg(p.zero_v + mo);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kPow2Batch; ++u) {
+          ak = fmaxf(ak, fmaxf(fabsf(zk[u]), fabsf(fmaf(cmax, sk[u], zk[u]))));
+          av = fmaxf(av, fmaxf(fabsf(zv[u]), fabsf(fmaf(cmax, sv[u], zv[u]))));
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
@@ -711,7 +735,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       Walk w;
       w.reset();
       for (int j = 0; j < T; ++j, ++g) {
-        const int nk = w.next(p);
+        const int nk = tabled ? nktab[j] : w.next(p);
         const int nk16 = (nk + 15) & ~15;
         const int slot = g % NS;
         if (!(ok = mbar_wait_bounded(s_full(qt, slot), (g / NS) & 1))) break;
@@ -745,11 +769,13 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           const float mx = smax * up;
           float alpha = 1.0f;
           bool rescale = false;
-          if (mx > m_ref + kPipeTau) {
-            if (m_ref != -INFINITY) {
-              alpha = __expf(m_ref - mx);
-              rescale = true;
-            }
+          if (m_ref == -INFINITY) {
+            // first tile of the item: start the reference above its maximum so
+            // that later tiles rarely need a rescale (p >= e^-kPipeHead here)
+            m_ref = mx + kPipeHead;
+          } else if (mx > m_ref + kPipeTau) {
+            alpha = __expf(m_ref - mx);
+            rescale = true;
             m_ref = mx;
           }
           l *= alpha;

@@ -108,8 +108,8 @@ bool plan_quant(vq::QuantParams& p) {
     while (G > 1 && int64_t(G) * slab > kSingle) --G;
     if (G > p.units) G = p.units;
     p.G = G;
-    // three staging buffers (two groups in flight) while they fit in ~100 KB
-    p.stages = (3 * int64_t(G) * slab <= 100 * 1024) ? 3 : 2;
+    // two staging buffers (one group in flight): smaller CTAs, more of them per SM
+    p.stages = 2;
     return true;
   }
   p.G = 1;
