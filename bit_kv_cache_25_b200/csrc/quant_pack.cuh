@@ -10,25 +10,27 @@
 // implies).
 //
 // Design (HBM-bound; ~2 B read + ~0.5 B written per bf16 element):
-//   * work unit = (tensor, b, h): an n_s x D slab. A CTA stages whole slabs
-//     (several small ones) or a chunk of word-rows of one large slab in shared
-//     memory with 1-D bulk async copies (one per slab chunk when tokens are
-//     contiguous). Large slabs are split over a thread-block cluster of up to
-//     16 CTAs. The partial per-channel min/max are exchanged through
-//     distributed shared memory, so HBM is read exactly once.
-//   * task = (word-row w, 16-byte vector j of a row): a thread reads the cpw
-//     rows of word-row w at vector j, i.e. 8 bf16 (or 4 fp32) channels.
-//     Shared-memory reads are 128-bit, each quarter-warp on one contiguous
-//     128-byte span, which is bank-conflict free.
-//   * pass 1: per-task min/max (packed bf16x2 min/max for bf16), then integer
-//     atomics on order-preserving keys into per-(unit, channel) shared slots.
-//     Min/max is exact, so the order of reduction does not matter.
-//   * scale/inv: one IEEE division and one IEEE reciprocal per group.
-//   * pass 2: d = x - min and t = d * inv, each correctly rounded (no FMA
-//     contraction), then round half to even by adding 1.5*2^23. The rounded
-//     value's low mantissa bits are the code (t <= 2^bits - 1 + tiny, so no
-//     clamp is needed). The codes are summed into the word with shifts and a
-//     final constant correction, then stored with 128-bit coalesced stores.
+//   * work unit = (tensor, b, h): an n_s x D slab. A group of P warps (P = 1
+//     when the block has thousands of units, up to 16 for a few large ones)
+//     owns a unit at a time; groups walk the units with a grid-wide stride.
+//     Nothing is staged and no CTA-wide barrier is taken: warp `part` of a
+//     group streams its whole word-rows of the slab through registers with
+//     16-byte loads (32/V rows per warp load, V = 16-byte vectors per row).
+//   * pass 1: packed bf16x2 (or fp32) min/max per lane, kQuantUnroll loads in
+//     flight (row indices past the part's end are clamped to its last row,
+//     which min/max ignore), then shuffles across the lanes that share a
+//     channel vector; with P > 1 the P partials meet in shared memory behind a
+//     named barrier of the group. Min/max is exact, so the order of reduction
+//     does not matter.
+//   * scale/inv: one IEEE division and one IEEE reciprocal per group (every
+//     lane computes its own channels' values).
+//   * pass 2: the warp re-reads its rows (now in L2), one word-row per lane and
+//     vector, all cpw row loads issued first: d = x - min and t = d * inv, each
+//     correctly rounded (no FMA contraction), then round half to even by adding
+//     1.5*2^23. The rounded value's low mantissa bits are the code
+//     (t <= 2^bits - 1 + tiny, so no clamp is needed). The codes are summed
+//     into the word with shifts and a final constant correction, then stored
+//     with 128-bit coalesced stores.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -42,35 +44,16 @@ namespace vq {
 
 namespace {
 
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 512;  // 16 warps
+constexpr int kQuantWarps = kQuantThreads / 32;
+constexpr int kQuantUnroll = 8;  // pass-1 loads in flight per lane
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kRoundMagic = 12582912.0f;
-
-struct QuantSmem {
-  // layout inside dynamic shared memory (byte offsets)
-  uint32_t bar, mnk, mxk, mn, inv, stage, stage_bytes;
-  uint32_t total;
-};
-
-__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
-
-// `stages` staging buffers of G slabs of rows_chunk rows each.
-__host__ __device__ inline QuantSmem quant_smem_layout(int G, int D, int rows_chunk, int rowbytes, int stages) {
-  QuantSmem L;
-  L.bar = 0;    // up to 4 mbarriers
-  L.mnk = 32;
-  L.mxk = L.mnk + 4u * G * D;
-  L.mn = L.mxk + 4u * G * D;
-  L.inv = L.mn + 4u * G * D;
-  L.stage = align_up(L.inv + 4u * G * D, 128);
-  L.stage_bytes = align_up(static_cast<uint32_t>(G) * rows_chunk * rowbytes, 128);
-  L.total = L.stage + stages * L.stage_bytes;
-  return L;
-}
 
 // 8 bf16 channels of one 16-byte vector.
 struct Bf16Vec {
   static constexpr int kCh = 8;
+  static constexpr uint32_t kMnInit = 0x7F807F80u, kMxInit = 0xFF80FF80u;
   __device__ static void minmax_init(uint32_t (&mn)[4], uint32_t (&mx)[4], const uint4& v) {
     mn[0] = mx[0] = v.x;
     mn[1] = mx[1] = v.y;
@@ -104,6 +87,7 @@ struct Bf16Vec {
 // 4 fp32 channels of one 16-byte vector.
 struct F32Vec {
   static constexpr int kCh = 4;
+  static constexpr uint32_t kMnInit = 0x7F800000u, kMxInit = 0xFF800000u;
   __device__ static void minmax_init(uint32_t (&mn)[4], uint32_t (&mx)[4], const uint4& v) {
     mn[0] = mx[0] = v.x;
     mn[1] = mx[1] = v.y;
@@ -125,378 +109,159 @@ struct F32Vec {
   }
 };
 
-// Work of one CTA-step: `units` consecutive units starting at `unit0`, each
-// restricted to the token rows [row0, row0 + rows) / word-rows [wr0, wr0 + wrs).
-struct QuantStep {
-  int unit0, units, row0, rows, wr0, wrs;
-};
-
-// Warp 0: stage the slabs of one step into `stage` (completion on `bar`).
-__device__ __forceinline__ void quant_issue_copies(const QuantParams& p, const QuantStep& st, unsigned char* stage,
-                                                   uint64_t* bar, int rowbytes) {
-  const int tid = threadIdx.x;
-  if (tid >= 32) return;
-  const uint32_t total = static_cast<uint32_t>(st.units) * st.rows * rowbytes;
-  if (tid == 0) mbar_arrive_expect_tx(bar, total);
-  __syncwarp();
-  const int BH = p.B * p.H;
-  for (int g = 0; g < st.units; ++g) {
-    const int unit = st.unit0 + g;
-    const QuantTensor& T = p.t[unit / BH];
-    const int bh = unit % BH;
-    const int64_t base = (bh / p.H) * T.sb + (bh % p.H) * T.sh;
-    const unsigned char* src = static_cast<const unsigned char*>(T.x) + (base + int64_t(st.row0) * T.st) * p.esize;
-    unsigned char* dst = stage + static_cast<size_t>(g) * p.rows_chunk * rowbytes;
-    if (T.st * p.esize == rowbytes) {
-      if (tid == 0) bulk_copy_g2s(dst, src, static_cast<uint32_t>(st.rows) * rowbytes, bar);
-    } else {
-      for (int r = tid; r < st.rows; r += 32)
-        bulk_copy_g2s(dst + r * rowbytes, src + int64_t(r) * T.st * p.esize, rowbytes, bar);
-    }
-  }
+__device__ __forceinline__ uint4 ldg128(const unsigned char* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
-// Pass 1: per-task min/max over the task's cpw rows, merged into the
-// per-(unit, channel) key slots. When a whole warp works on one unit, the
-// lanes that share a channel vector (lane % V) first combine their keys with
-// shuffles and only V lanes issue shared-memory atomics; otherwise every lane
-// issues its own. Min and max are idempotent, so any merge order is exact.
 template <class Vec, int BITS>
-__device__ __forceinline__ void quant_pass1(const QuantParams& p, const QuantStep& st, const unsigned char* stage,
-                                            int32_t* mnk, int32_t* mxk) {
+__global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __grid_constant__ QuantParams p) {
   constexpr int CPW = 32 / BITS;
   constexpr int CH = Vec::kCh;
-  const int V = p.vecs_per_row;
-  const int rowbytes = V * 16;
+  extern __shared__ __align__(16) float qred[];  // [2][groups][P][2][D]
   const int D = p.D;
-  const int tpu = st.wrs * V;
-  const int ntask = st.units * tpu;
+  const int V = p.vecs_per_row;
+  const int RW = 32 / V;
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int wbase = threadIdx.x & ~31;
-  for (int base = 0; base < ntask; base += blockDim.x) {
-    const int task = base + threadIdx.x;
-    const bool valid = task < ntask;
-    const int g = valid ? task / tpu : 0;
-    const int r = task - g * tpu;
-    const int wl = r / V;
-    const int j = r - wl * V;
-    int32_t kmn[CH], kmx[CH];
-    if (valid) {
-      const int tl0 = wl * CPW;
-      const int nvalid = min(CPW, st.rows - tl0);
-      const unsigned char* src = stage + (static_cast<size_t>(g) * p.rows_chunk + tl0) * rowbytes + j * 16;
-      uint32_t mn[4], mx[4];
-      Vec::minmax_init(mn, mx, lds128(src));
-#pragma unroll
-      for (int i = 1; i < CPW; ++i)
-        if (i < nvalid) Vec::minmax_acc(mn, mx, lds128(src + i * rowbytes));
-#pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        kmn[c] = float_key(Vec::ch(mn, c));
-        kmx[c] = float_key(Vec::ch(mx, c));
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        kmn[c] = INT32_MAX;
-        kmx[c] = INT32_MIN;
-      }
-    }
-    const int t_first = base + wbase;
-    const bool uniform = (t_first + 31 < ntask) && (t_first / tpu == (t_first + 31) / tpu);
-    if (uniform) {  // warp-uniform branch
-      for (int off = V; off < 32; off <<= 1) {
-#pragma unroll
-        for (int c = 0; c < CH; ++c) {
-          kmn[c] = min(kmn[c], __shfl_xor_sync(0xffffffffu, kmn[c], off));
-          kmx[c] = max(kmx[c], __shfl_xor_sync(0xffffffffu, kmx[c], off));
-        }
-      }
-      if (lane < V) {
-#pragma unroll
-        for (int c = 0; c < CH; ++c) {
-          atomicMin(&mnk[g * D + j * CH + c], kmn[c]);
-          atomicMax(&mxk[g * D + j * CH + c], kmx[c]);
-        }
-      }
-    } else if (valid) {
-#pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        atomicMin(&mnk[g * D + j * CH + c], kmn[c]);
-        atomicMax(&mxk[g * D + j * CH + c], kmx[c]);
-      }
-    }
-  }
-}
-
-// Per group: scale = (max - min) / (2^b - 1) (IEEE division), zero = min + 0,
-// inv = min(1/scale, FLT_MAX) (IEEE reciprocal), written to shared memory for
-// pass 2 and (when `write`) to the output arrays.
-template <int BITS>
-__device__ __forceinline__ void quant_finalize(const QuantParams& p, const QuantStep& st, int32_t kmn, int32_t kmx,
-                                               int i, float* s_mn, float* s_inv, bool write) {
-  const int D = p.D;
-  const float mn = key_float(kmn);
-  const float mx = key_float(kmx);
-  const float diff = __fsub_rn(mx, mn);
-  const float scale = __fdiv_rn(diff, static_cast<float>((1 << BITS) - 1));
-  const float zero = __fadd_rn(mn, 0.0f);
-  const float inv = (scale > 0.0f) ? fminf(__frcp_rn(scale), FLT_MAX) : 0.0f;
-  s_mn[i] = mn;
-  s_inv[i] = inv;
-  if (write) {
-    const int BH = p.B * p.H;
-    const int g = i / D;
-    const int c = i - g * D;
-    const int unit = st.unit0 + g;
+  const int P = p.P;
+  const int gpc = kQuantWarps / P;
+  const int grp = warp / P;
+  const int part = warp - grp * P;
+  const int j = lane % V;
+  const int rsub = lane / V;
+  const int BH = p.B * p.H;
+  int par = 0;
+  for (int unit = blockIdx.x * gpc + grp; unit < p.units; unit += gridDim.x * gpc, par ^= 1) {
     const QuantTensor& T = p.t[unit / BH];
     const int bh = unit % BH;
-    T.scale[static_cast<size_t>(bh) * D + c] = scale;
-    T.zero[static_cast<size_t>(bh) * D + c] = zero;
-  }
-}
-
-// Pass 2: encode and pack. d = x - min and t = d * inv, each correctly rounded
-// (__fsub_rn / __fmul_rn are never contracted into an FMA), then round half to
-// even by adding 1.5 * 2^23: the rounded value's low mantissa bits are the code
-// (t <= 2^b - 1 + tiny, so no clamp is needed). Codes are summed into the word
-// with shifts; the magic bits are removed once. (Packed f32x2 arithmetic is
-// not used here: ptxas may fuse a packed multiply and add into one rounding.)
-template <class Vec, int BITS>
-__device__ __forceinline__ void quant_pass2(const QuantParams& p, const QuantStep& st, const unsigned char* stage,
-                                            const float* s_mn, const float* s_inv) {
-  constexpr int CPW = 32 / BITS;
-  constexpr int CH = Vec::kCh;
-  const int V = p.vecs_per_row;
-  const int rowbytes = V * 16;
-  const int D = p.D;
-  const int BH = p.B * p.H;
-  const int tpu = st.wrs * V;
-  for (int task = threadIdx.x; task < st.units * tpu; task += blockDim.x) {
-    const int g = task / tpu;
-    const int r = task - g * tpu;
-    const int wl = r / V;
-    const int j = r - wl * V;
-    const int tl0 = wl * CPW;
-    const int nvalid = min(CPW, st.rows - tl0);
-    const unsigned char* src = stage + (static_cast<size_t>(g) * p.rows_chunk + tl0) * rowbytes + j * 16;
-    float mn[CH], inv[CH];
+    const unsigned char* slab =
+        static_cast<const unsigned char*>(T.x) + ((bh / p.H) * T.sb + (bh % p.H) * T.sh) * p.esize + j * 16;
+    const int64_t rstride = T.st * p.esize;
+    const int w0 = part * p.WP, w1 = min(p.W, w0 + p.WP);
+    const int r0 = w0 * CPW, r1 = min(p.n, w1 * CPW);
+    uint32_t mn[4], mx[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      mn[k] = Vec::kMnInit;
+      mx[k] = Vec::kMxInit;
+    }
+    // pass 1: rows past r1 re-read row r1-1 (min/max are idempotent), so
+    // every load of a batch is issued before any is used
+    for (int r = r0 + rsub; r < r1; r += kQuantUnroll * RW) {
+      uint4 v[kQuantUnroll];
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) v[u] = ldg128(slab + min(r + u * RW, r1 - 1) * rstride);
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) Vec::minmax_acc(mn, mx, v[u]);
+    }
+    float fmn[CH], fmx[CH];
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-      mn[c] = s_mn[g * D + j * CH + c];
-      inv[c] = s_inv[g * D + j * CH + c];
+      fmn[c] = Vec::ch(mn, c);
+      fmx[c] = Vec::ch(mx, c);
     }
-    uint32_t acc[CH];
+    for (int off = V; off < 32; off <<= 1) {
 #pragma unroll
-    for (int c = 0; c < CH; ++c) acc[c] = 0u;
-    uint32_t corr = 0u;
-#pragma unroll
-    for (int i = 0; i < CPW; ++i) {
-      if (i < nvalid) {
-        const uint4 v = lds128(src + i * rowbytes);
-        corr += kRoundMagicBits << (BITS * i);
+      for (int c = 0; c < CH; ++c) {
+        fmn[c] = fminf(fmn[c], __shfl_xor_sync(0xffffffffu, fmn[c], off));
+        fmx[c] = fmaxf(fmx[c], __shfl_xor_sync(0xffffffffu, fmx[c], off));
+      }
+    }
+    if (P > 1) {
+      float* rb = qred + ((par * gpc + grp) * P) * 2 * D;
+      if (rsub == 0) {
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
-          const float d = __fsub_rn(Vec::elem(v, c), mn[c]);
-          const float t = __fmul_rn(d, inv[c]);
-          const float rq = __fadd_rn(t, kRoundMagic);
-          acc[c] += __float_as_uint(rq) << (BITS * i);
+          rb[part * 2 * D + CH * j + c] = fmn[c];
+          rb[part * 2 * D + D + CH * j + c] = fmx[c];
+        }
+      }
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(32 * P) : "memory");
+      for (int q = 0; q < P; ++q) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          fmn[c] = fminf(fmn[c], rb[q * 2 * D + CH * j + c]);
+          fmx[c] = fmaxf(fmx[c], rb[q * 2 * D + D + CH * j + c]);
         }
       }
     }
-    const int unit = st.unit0 + g;
-    const QuantTensor& T = p.t[unit / BH];
-    const int bh = unit % BH;
-    uint32_t* dst = T.packed + (static_cast<size_t>(bh) * p.W + st.wr0 + wl) * D + j * CH;
+    float scl[CH], zer[CH], inv[CH];
 #pragma unroll
-    for (int q = 0; q < CH / 4; ++q)
-      reinterpret_cast<uint4*>(dst)[q] =
-          make_uint4(acc[4 * q] - corr, acc[4 * q + 1] - corr, acc[4 * q + 2] - corr, acc[4 * q + 3] - corr);
-  }
-}
-
-// Blocks whose (tensor, b, h) slab fits one CTA: a persistent loop over groups
-// of G units with a p.stages-deep bulk-copy pipeline, so the next groups'
-// slabs are in flight while this group is reduced, encoded and stored.
-template <class Vec, int BITS>
-__global__ void __launch_bounds__(kQuantThreads) quant_pack_stream_kernel(const __grid_constant__ QuantParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int D = p.D;
-  const int rowbytes = p.vecs_per_row * 16;
-  const int NST = p.stages;
-  const QuantSmem L = quant_smem_layout(p.G, D, p.rows_chunk, rowbytes, NST);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);
-  int32_t* mnk = reinterpret_cast<int32_t*>(smem + L.mnk);
-  int32_t* mxk = reinterpret_cast<int32_t*>(smem + L.mxk);
-  float* s_mn = reinterpret_cast<float*>(smem + L.mn);
-  float* s_inv = reinterpret_cast<float*>(smem + L.inv);
-  const int tid = threadIdx.x;
-  const int groups = (p.units + p.G - 1) / p.G;
-
-  auto step_of = [&](int grp) {
-    QuantStep st;
-    st.unit0 = grp * p.G;
-    st.units = min(p.G, p.units - st.unit0);
-    st.row0 = 0;
-    st.rows = p.n;
-    st.wr0 = 0;
-    st.wrs = p.W;
-    return st;
-  };
-
-  if (tid == 0) {
-    for (int i = 0; i < NST; ++i) mbar_init(&bar[i], 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
-  // prologue: the first NST-1 groups of this CTA
-  for (int k = 0; k < NST - 1; ++k) {
-    const int grp = blockIdx.x + k * gridDim.x;
-    if (grp < groups) quant_issue_copies(p, step_of(grp), smem + L.stage + k * L.stage_bytes, &bar[k], rowbytes);
-  }
-  bool ok = true;
-  int it = 0;
-  for (int grp = blockIdx.x; grp < groups; ++it, grp += gridDim.x) {
-    const QuantStep st = step_of(grp);
-    const int stg = it % NST;
-    // keep NST-1 groups in flight: the stage refilled here was last read by
-    // the previous iteration, which ended with a barrier
-    const int ahead = grp + (NST - 1) * gridDim.x;
-    if (ahead < groups) {
-      const int s2 = (it + NST - 1) % NST;
-      quant_issue_copies(p, step_of(ahead), smem + L.stage + s2 * L.stage_bytes, &bar[s2], rowbytes);
+    for (int c = 0; c < CH; ++c) {
+      scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), static_cast<float>((1 << BITS) - 1));
+      zer[c] = __fadd_rn(fmn[c], 0.0f);
+      inv[c] = (scl[c] > 0.0f) ? fminf(__frcp_rn(scl[c]), FLT_MAX) : 0.0f;
     }
-    for (int i = tid; i < st.units * D; i += blockDim.x) {
-      mnk[i] = INT32_MAX;
-      mxk[i] = INT32_MIN;
+    if (part == 0 && rsub == 0) {
+      float* sd = T.scale + static_cast<size_t>(bh) * D + CH * j;
+      float* zd = T.zero + static_cast<size_t>(bh) * D + CH * j;
+#pragma unroll
+      for (int q = 0; q < CH / 4; ++q) {
+        reinterpret_cast<float4*>(sd)[q] = make_float4(scl[4 * q], scl[4 * q + 1], scl[4 * q + 2], scl[4 * q + 3]);
+        reinterpret_cast<float4*>(zd)[q] = make_float4(zer[4 * q], zer[4 * q + 1], zer[4 * q + 2], zer[4 * q + 3]);
+      }
     }
-    ok = __syncthreads_and(mbar_wait_bounded(&bar[stg], (it / NST) & 1));
-    if (!ok) break;
-    const unsigned char* stage = smem + L.stage + stg * L.stage_bytes;
-    quant_pass1<Vec, BITS>(p, st, stage, mnk, mxk);
-    __syncthreads();
-    for (int i = tid; i < st.units * D; i += blockDim.x) quant_finalize<BITS>(p, st, mnk[i], mxk[i], i, s_mn, s_inv, true);
-    __syncthreads();
-    quant_pass2<Vec, BITS>(p, st, stage, s_mn, s_inv);
-    fence_proxy_async_smem();  // generic reads of this stage before a later bulk copy overwrites it
-    __syncthreads();
-  }
-}
-
-// Blocks whose slab is split over a cluster of C CTAs: each CTA stages its
-// chunk of word-rows; the per-channel partial min/max are combined through
-// distributed shared memory, so HBM is read exactly once.
-template <class Vec, int BITS>
-__global__ void __launch_bounds__(kQuantThreads) quant_pack_cluster_kernel(const __grid_constant__ QuantParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int D = p.D;
-  const int rowbytes = p.vecs_per_row * 16;
-  const QuantSmem L = quant_smem_layout(1, D, p.rows_chunk, rowbytes, 1);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.bar);
-  int32_t* mnk = reinterpret_cast<int32_t*>(smem + L.mnk);
-  int32_t* mxk = reinterpret_cast<int32_t*>(smem + L.mxk);
-  float* s_mn = reinterpret_cast<float*>(smem + L.mn);
-  float* s_inv = reinterpret_cast<float*>(smem + L.inv);
-  constexpr int CPW = 32 / BITS;
-  const int C = p.C;
-  const uint32_t rank = cluster_ctarank();
-  const int tid = threadIdx.x;
-
-  QuantStep st;
-  st.unit0 = static_cast<int>(blockIdx.x) / C;
-  st.units = 1;
-  st.wr0 = static_cast<int>(rank) * p.wr_chunk;
-  st.wrs = max(0, min(p.wr_chunk, p.W - st.wr0));
-  st.row0 = st.wr0 * CPW;
-  st.rows = max(0, min(p.rows_chunk, p.n - st.row0));
-
-  if (tid == 0) {
-    mbar_init(bar, 1);
-    fence_barrier_init();
-  }
-  for (int i = tid; i < D; i += blockDim.x) {
-    mnk[i] = INT32_MAX;
-    mxk[i] = INT32_MIN;
-  }
-  __syncthreads();
-  quant_issue_copies(p, st, smem + L.stage, bar, rowbytes);
-  const bool staged = __syncthreads_and(mbar_wait_bounded(bar, 0));
-  if (staged) quant_pass1<Vec, BITS>(p, st, smem + L.stage, mnk, mxk);
-  __syncthreads();
-
-  cluster_sync();  // every CTA's partials are complete and visible
-  int32_t fmn = INT32_MAX, fmx = INT32_MIN;
-  if (tid < D) {
-    for (int r = 0; r < C; ++r) {
-      fmn = min(fmn, dsmem_ld_s32(&mnk[tid], r));
-      fmx = max(fmx, dsmem_ld_s32(&mxk[tid], r));
+    // pass 2: one word-row per lane and vector; every row load issued first
+    for (int w = w0 + rsub; w < w1; w += RW) {
+      const int tl0 = w * CPW;
+      const int nvalid = min(CPW, p.n - tl0);
+      uint4 v[CPW];
+#pragma unroll
+      for (int i = 0; i < CPW; ++i) v[i] = ldg128(slab + (tl0 + min(i, nvalid - 1)) * rstride);
+      uint32_t acc[CH];
+#pragma unroll
+      for (int c = 0; c < CH; ++c) acc[c] = 0u;
+      uint32_t corr = 0u;
+#pragma unroll
+      for (int i = 0; i < CPW; ++i) {
+        if (i < nvalid) {
+          corr += kRoundMagicBits << (BITS * i);
+#pragma unroll
+          for (int c = 0; c < CH; ++c) {
+            const float d = __fsub_rn(Vec::elem(v[i], c), fmn[c]);
+            const float t = __fmul_rn(d, inv[c]);
+            const float rq = __fadd_rn(t, kRoundMagic);
+            acc[c] += __float_as_uint(rq) << (BITS * i);
+          }
+        }
+      }
+      uint32_t* dst = T.packed + (static_cast<size_t>(bh) * p.W + w) * D + CH * j;
+#pragma unroll
+      for (int q = 0; q < CH / 4; ++q)
+        reinterpret_cast<uint4*>(dst)[q] =
+            make_uint4(acc[4 * q] - corr, acc[4 * q + 1] - corr, acc[4 * q + 2] - corr, acc[4 * q + 3] - corr);
     }
   }
-  cluster_arrive();  // done reading peers; the matching wait is at the end
-  if (tid < D) quant_finalize<BITS>(p, st, fmn, fmx, tid, s_mn, s_inv, rank == 0 && staged);
-  __syncthreads();
-  if (staged) quant_pass2<Vec, BITS>(p, st, smem + L.stage, s_mn, s_inv);
-  cluster_wait();  // peers may still read this CTA's partials until here
 }
 
 template <class Vec, int BITS>
 cudaError_t launch_typed(const QuantParams& p, cudaStream_t stream) {
-  const bool cluster = p.C > 1;
-  auto kern = cluster ? quant_pack_cluster_kernel<Vec, BITS> : quant_pack_stream_kernel<Vec, BITS>;
-  const int rowbytes = p.vecs_per_row * 16;
-  const QuantSmem L = quant_smem_layout(cluster ? 1 : p.G, p.D, p.rows_chunk, rowbytes, cluster ? 1 : p.stages);
-  // Function attributes are set once per device and size, outside any stream
-  // work, so launches can be captured into CUDA graphs.
-  static int configured_smem[2][kMaxDevices] = {};
-  static bool configured_cluster[kMaxDevices] = {};
+  auto kern = quant_pack_kernel<Vec, BITS>;
   static int sm_count[kMaxDevices] = {};
+  static bool configured[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (static_cast<int>(L.total) > configured_smem[cluster][dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(quant_smem_bytes(128)));
     if (e != cudaSuccess) return e;
-    configured_smem[cluster][dev] = static_cast<int>(L.total);
-  }
-  if (sm_count[dev] == 0) {
     e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
+    configured[dev] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.blockDim = dim3(kQuantThreads);
-  cfg.dynamicSmemBytes = L.total;
-  cfg.stream = stream;
-  if (cluster) {
-    if (p.C > 8 && !configured_cluster[dev]) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-      configured_cluster[dev] = true;
-    }
-    cfg.gridDim = dim3(p.units * p.C);
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  } else {
-    // persistent: enough CTAs to fill every SM at the residency shared memory allows
-    const int groups = (p.units + p.G - 1) / p.G;
-    const int per_sm = max(1, min(8, static_cast<int>((227u * 1024u) / (L.total + 1024u))));
-    cfg.gridDim = dim3(min(groups, sm_count[dev] * per_sm));
-  }
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  const int gpc = kQuantWarps / p.P;
+  const int ctas = (p.units + gpc - 1) / gpc;
+  const int grid = ctas < sm_count[dev] ? ctas : sm_count[dev];
+  kern<<<grid, kQuantThreads, p.P > 1 ? quant_smem_bytes(p.D) : 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t quant_smem_bytes(int G, int D, int rows_chunk, int rowbytes, int stages) {
-  return quant_smem_layout(G, D, rows_chunk, rowbytes, stages).total;
-}
+size_t quant_smem_bytes(int D) { return static_cast<size_t>(2) * kQuantWarps * 2 * D * sizeof(float); }
 
-int quant_threads() { return kQuantThreads; }
+int quant_warps() { return kQuantWarps; }
 
 cudaError_t launch_quant_pack(const QuantParams& p, cudaStream_t stream) {
   const bool bf16 = (p.esize == 2);

@@ -92,41 +92,12 @@ vq_status check_strides(const int64_t st[3], int esize, const char* name) {
 // Choose units per CTA (G), CTAs per unit (cluster size C) and word-rows per CTA
 // for one quantize launch. Returns false if one slab is too large.
 bool plan_quant(vq::QuantParams& p) {
-  const int cpw = codes_per_word(p.bits);
-  const int rowbytes = p.vecs_per_row * 16;
-  const int64_t slab = int64_t(p.n) * rowbytes;
-  const int64_t kSingle = 64 * 1024;
-  if (slab <= kSingle) {
-    p.C = 1;
-    p.wr_chunk = p.W;
-    p.rows_chunk = p.n;
-    // several small slabs per CTA step, so a step has about one task per thread
-    const int tasks = p.W * p.vecs_per_row;
-    int G = vq::quant_threads() / tasks;
-    if (G < 1) G = 1;
-    if (G > 8) G = 8;
-    while (G > 1 && int64_t(G) * slab > kSingle) --G;
-    if (G > p.units) G = p.units;
-    p.G = G;
-    // two staging buffers (one group in flight): smaller CTAs, more of them per SM
-    p.stages = 2;
-    return true;
-  }
-  p.G = 1;
-  for (int64_t budget : {72 * 1024, 100 * 1024, 144 * 1024, 200 * 1024}) {
-    const int wr_max = static_cast<int>(budget / (int64_t(cpw) * rowbytes));
-    if (wr_max < 1) continue;
-    int C = (p.W + wr_max - 1) / wr_max;
-    if (C > 16) continue;
-    const int wr = (p.W + C - 1) / C;
-    C = (p.W + wr - 1) / wr;
-    p.C = C;
-    p.wr_chunk = wr;
-    p.rows_chunk = wr * cpw;
-    p.stages = 1;
-    return true;
-  }
-  return false;
+  constexpr int64_t kTargetWarps = 2048;
+  int P = 1;
+  while (P < vq::quant_warps() && int64_t(p.units) * P < kTargetWarps && 2 * P <= p.W) P *= 2;
+  p.P = P;
+  p.WP = (p.W + P - 1) / P;
+  return true;
 }
 
 vq_status launch_quant(const vq_cache_desc* d, int32_t block, vq_dtype dt, int ntensors, const void* const x[2],
@@ -159,9 +130,7 @@ vq_status launch_quant(const vq_cache_desc* d, int32_t block, vq_dtype dt, int n
     p.t[i].scale = scale[i];
     p.t[i].zero = zero[i];
   }
-  if (!plan_quant(p))
-    return fail(VQ_ERR_UNSUPPORTED, "block of %d tokens x %d bytes per row exceeds the 16-CTA cluster limit", p.n,
-                p.D * esize);
+  plan_quant(p);
   cudaError_t e = vq::launch_quant_pack(p, static_cast<cudaStream_t>(stream));
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "quantize+pack launch");

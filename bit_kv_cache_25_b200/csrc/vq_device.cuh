@@ -1,6 +1,6 @@
 // Device-side helpers shared by the libvq kernels: shared-memory addresses,
 // mbarriers with bounded waits, 1-D bulk async copies (TMA engine, no tensor
-// map, never multicast), cluster barriers and distributed shared memory.
+// map, never multicast) and 128-bit shared-memory loads.
 #pragma once
 
 #include <cstdint>
@@ -84,50 +84,12 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  cluster_arrive();
-  cluster_wait();
-}
-
-// Load a 32-bit word from the shared memory of CTA `rank` in this cluster.
-__device__ __forceinline__ int32_t dsmem_ld_s32(const void* local_ptr, uint32_t rank) {
-  uint32_t remote;
-  int32_t v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local_ptr)), "r"(rank));
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
-  return v;
-}
-
 __device__ __forceinline__ uint4 lds128(const void* p) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(smem_addr(p)));
   return v;
-}
-
-// Order-preserving map float -> int32 (involution): integer order of the keys
-// equals float order of finite values, with -0 < +0.
-__device__ __forceinline__ int32_t float_key(float f) {
-  int32_t i = __float_as_int(f);
-  return i ^ ((i >> 31) & 0x7fffffff);
-}
-__device__ __forceinline__ float key_float(int32_t k) {
-  return __int_as_float(k ^ ((k >> 31) & 0x7fffffff));
 }
 
 }  // namespace vq

@@ -27,15 +27,12 @@ struct QuantParams {
   int esize;            // 2 (bf16) or 4 (fp32)
   int vecs_per_row;     // D * esize / 16
   int units;            // tensors * B * H
-  int G;                // units per CTA (C == 1)
-  int C;                // CTAs per unit (cluster size); G == 1 when C > 1
-  int wr_chunk;         // word-rows per CTA
-  int rows_chunk;       // staged token rows per unit per CTA (n when C == 1)
-  int stages;           // staging buffers of the single-CTA (C == 1) pipeline
+  int P;                // warps per unit (1, 2, 4, 8 or 16)
+  int WP;               // word-rows per warp of a unit (ceil(W / P))
 };
 
-size_t quant_smem_bytes(int G, int D, int rows_chunk, int rowbytes, int stages);
-int quant_threads();
+size_t quant_smem_bytes(int D);
+int quant_warps();
 cudaError_t launch_quant_pack(const QuantParams& p, cudaStream_t stream);
 
 struct DequantParams {
