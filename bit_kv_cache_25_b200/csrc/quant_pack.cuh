@@ -46,7 +46,7 @@ namespace {
 
 constexpr int kQuantThreads = 512;  // 16 warps
 constexpr int kQuantWarps = kQuantThreads / 32;
-constexpr int kQuantUnroll = 8;  // pass-1 loads in flight per lane
+constexpr int kQuantUnroll = 16;  // pass-1 loads in flight per lane
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kRoundMagic = 12582912.0f;
 
@@ -120,24 +120,32 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
   extern __shared__ __align__(16) float qred[];  // [2][groups][P][2][D]
   const int D = p.D;
   const int V = p.vecs_per_row;
-  const int RW = 32 / V;
+  const int TL = p.TL;            // lanes per unit (team): a warp takes 32/TL units at once when P == 1
+  const int RW = TL / V;          // rows per team load
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int P = p.P;
   const int gpc = kQuantWarps / P;
   const int grp = warp / P;
   const int part = warp - grp * P;
-  const int j = lane % V;
-  const int rsub = lane / V;
+  const int team = lane / TL;
+  const int tl = lane - team * TL;
+  const int j = tl % V;
+  const int rsub = tl / V;
+  const int upw = 32 / TL;        // units per group step
   const int BH = p.B * p.H;
   int par = 0;
-  for (int unit = blockIdx.x * gpc + grp; unit < p.units; unit += gridDim.x * gpc, par ^= 1) {
-    const QuantTensor& T = p.t[unit / BH];
-    const int bh = unit % BH;
+  // every lane of a warp runs the same rounds (shuffles below use the full
+  // warp); a team whose unit is past the end only skips its loads and stores
+  for (int u0 = (blockIdx.x * gpc + grp) * upw; u0 < p.units; u0 += gridDim.x * gpc * upw, par ^= 1) {
+    const int unit = u0 + team;
+    const bool live = unit < p.units;
+    const QuantTensor& T = p.t[(live ? unit : u0) / BH];
+    const int bh = (live ? unit : u0) % BH;
     const unsigned char* slab =
         static_cast<const unsigned char*>(T.x) + ((bh / p.H) * T.sb + (bh % p.H) * T.sh) * p.esize + j * 16;
     const int64_t rstride = T.st * p.esize;
-    const int w0 = part * p.WP, w1 = min(p.W, w0 + p.WP);
+    const int w0 = part * p.WP, w1 = live ? min(p.W, w0 + p.WP) : w0;
     const int r0 = w0 * CPW, r1 = min(p.n, w1 * CPW);
     uint32_t mn[4], mx[4];
 #pragma unroll
@@ -160,7 +168,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
       fmn[c] = Vec::ch(mn, c);
       fmx[c] = Vec::ch(mx, c);
     }
-    for (int off = V; off < 32; off <<= 1) {
+    for (int off = V; off < TL; off <<= 1) {
 #pragma unroll
       for (int c = 0; c < CH; ++c) {
         fmn[c] = fminf(fmn[c], __shfl_xor_sync(0xffffffffu, fmn[c], off));
@@ -192,7 +200,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
       zer[c] = __fadd_rn(fmn[c], 0.0f);
       inv[c] = (scl[c] > 0.0f) ? fminf(__frcp_rn(scl[c]), FLT_MAX) : 0.0f;
     }
-    if (part == 0 && rsub == 0) {
+    if (live && part == 0 && rsub == 0) {
       float* sd = T.scale + static_cast<size_t>(bh) * D + CH * j;
       float* zd = T.zero + static_cast<size_t>(bh) * D + CH * j;
 #pragma unroll
@@ -251,7 +259,8 @@ cudaError_t launch_typed(const QuantParams& p, cudaStream_t stream) {
     configured[dev] = true;
   }
   const int gpc = kQuantWarps / p.P;
-  const int ctas = (p.units + gpc - 1) / gpc;
+  const int per_cta = gpc * (32 / p.TL);
+  const int ctas = (p.units + per_cta - 1) / per_cta;
   const int grid = ctas < sm_count[dev] ? ctas : sm_count[dev];
   kern<<<grid, kQuantThreads, p.P > 1 ? quant_smem_bytes(p.D) : 0, stream>>>(p);
   return cudaGetLastError();

@@ -97,6 +97,11 @@ bool plan_quant(vq::QuantParams& p) {
   while (P < vq::quant_warps() && int64_t(p.units) * P < kTargetWarps && 2 * P <= p.W) P *= 2;
   p.P = P;
   p.WP = (p.W + P - 1) / P;
+  // tiny blocks: a warp takes several units, each on vecs_per_row * rows lanes
+  int rows = 1;
+  while (rows * p.vecs_per_row < 32 && rows < p.n) rows *= 2;
+  p.TL = (P == 1) ? rows * p.vecs_per_row : 32;
+  if (p.TL > 32) p.TL = 32;
   return true;
 }
 

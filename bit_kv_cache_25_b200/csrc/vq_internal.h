@@ -29,6 +29,7 @@ struct QuantParams {
   int units;            // tensors * B * H
   int P;                // warps per unit (1, 2, 4, 8 or 16)
   int WP;               // word-rows per warp of a unit (ceil(W / P))
+  int TL;               // lanes per unit when P == 1 (vecs_per_row * rows per load; 32 / TL units per warp)
 };
 
 size_t quant_smem_bytes(int D);
