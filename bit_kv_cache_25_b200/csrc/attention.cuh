@@ -152,17 +152,18 @@ constexpr int kTcMinQueries = 16;
 
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
   if (p.n_q >= kTcMinQueries) {
-    // two query tiles per work item (sharing every dequantized K/V tile) once
-    // the block has more than 128 queries
+    // more than 128 queries: two query tiles per work item sharing every
+    // dequantized K/V tile; otherwise one query tile per item, the two
+    // softmax warpgroups taking the items in turn
     const bool pair = p.n_q > 128;
     if (p.bits == 4 && p.D == 64)
-      return pair ? launch_attention_pipe<4, 64, 2>(p, stream) : launch_attention_pipe<4, 64, 1>(p, stream);
+      return pair ? launch_attention_pipe<4, 64, 2, false>(p, stream) : launch_attention_pipe<4, 64, 2, true>(p, stream);
     if (p.bits == 4 && p.D == 128)
-      return pair ? launch_attention_pipe<4, 128, 2>(p, stream) : launch_attention_pipe<4, 128, 1>(p, stream);
+      return pair ? launch_attention_pipe<4, 128, 2, false>(p, stream) : launch_attention_pipe<4, 128, 2, true>(p, stream);
     if (p.bits == 3 && p.D == 64)
-      return pair ? launch_attention_pipe<3, 64, 2>(p, stream) : launch_attention_pipe<3, 64, 1>(p, stream);
+      return pair ? launch_attention_pipe<3, 64, 2, false>(p, stream) : launch_attention_pipe<3, 64, 2, true>(p, stream);
     if (p.bits == 3 && p.D == 128)
-      return pair ? launch_attention_pipe<3, 128, 2>(p, stream) : launch_attention_pipe<3, 128, 1>(p, stream);
+      return pair ? launch_attention_pipe<3, 128, 2, false>(p, stream) : launch_attention_pipe<3, 128, 2, true>(p, stream);
   }
   if (p.bits == 4 && p.D == 64) return launch_attention_small<4, 64>(p, stream);
   if (p.bits == 4 && p.D == 128) return launch_attention_small<4, 128>(p, stream);

@@ -69,7 +69,8 @@ struct PipeCfg {
   static constexpr int NS = (NQT == 1) ? 4 : ((D == 64) ? 3 : 2);  // S slots per query tile
   static constexpr int NKV = (D == 64) ? (NQT == 1 ? 4 : 3) : (NQT == 1 ? 3 : 2);  // K/V tile slots
   static constexpr int NSTG = 2;                           // packed-word stages
-  static constexpr bool STAGE_Q = (D == 64);               // next item's queries prefetched by cp.async
+  static constexpr bool STAGE_Q = (D == 64);               // queries of later items prefetched by cp.async
+  static constexpr int QPF = (STAGE_Q && NQT == 1) ? 2 : 1;  // items ahead the query staging runs
   static constexpr int UNPACK_WARPS = (NQT == 1) ? 8 : 4;
   static constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
   static constexpr int UNPACK_T0 = NQT * 128;
@@ -82,9 +83,9 @@ struct PipeCfg {
   static constexpr int TILE_SZ = KT * D * 2;               // fp16 [KT][D], K-major SW128
   static constexpr int KV0 = Q0 + NQT * Q_SZ;              // NKV x {K hi, K lo, V hi, V lo}
   static constexpr int KV_SZ = 4 * TILE_SZ;
-  static constexpr int QST0 = KV0 + NKV * KV_SZ;           // bf16 [128][D] query staging per query tile
+  static constexpr int QST0 = KV0 + NKV * KV_SZ;           // QPF x bf16 [128][D] query staging per query tile
   static constexpr int QST_SZ = STAGE_Q ? 128 * D * 2 : 0;
-  static constexpr int STG0 = QST0 + NQT * QST_SZ;         // NSTG x {K rows, V rows, meta, segment table}
+  static constexpr int STG0 = QST0 + NQT * QPF * QST_SZ;         // NSTG x {K rows, V rows, meta, segment table}
   static constexpr int STG_V = MAXROWS * D * 4;
   static constexpr int STG_META = 2 * STG_V;               // MAXSEG x [4][D] fp32: sk, zk, sv, zv
   static constexpr int STG_SEG = STG_META + MAXSEG * 4 * D * 4;  // MAXSEG x int4 {block, u0, take, key0}
@@ -159,9 +160,13 @@ struct PipeWalk {
   }
 };
 
-template <int BITS, int D, int NQT>
+// ALT (with NQT == 2): every work item is one query tile and the two softmax
+// warpgroups take the CTA's items in turn (even, odd), so one item's softmax
+// overlaps the other's query conversion, epilogue and tensor-core round trips.
+template <int BITS, int D, int NQT, bool ALT>
 __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     attention_pipe_kernel(const __grid_constant__ AttnParams p) {
+  static_assert(!ALT || NQT == 2, "alternating items need two softmax warpgroups");
   using C = PipeCfg<BITS, D, NQT>;
   constexpr int CPW = C::CPW;
   constexpr int KT = C::KT;
@@ -193,9 +198,12 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   const int lane = tid & 31;
   const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
   const int n_qt = (p.n_q + 127) / 128;
-  const int n_groups = (n_qt + NQT - 1) / NQT;
+  const int n_groups = ALT ? n_qt : (n_qt + NQT - 1) / NQT;
   const int n_items = p.B * p.H * n_groups;
-  auto item_nqt = [&](int item) { return min(NQT, n_qt - (item % n_groups) * NQT); };
+  auto item_nqt = [&](int item) { return ALT ? 1 : min(NQT, n_qt - (item % n_groups) * NQT); };
+  // query tiles [qlo, qhi) of the k-th item of this CTA
+  auto item_qlo = [&](int k) { return ALT ? (k & 1) : 0; };
+  auto item_qhi = [&](int k, int item) { return ALT ? (k & 1) + 1 : item_nqt(item); };
   // key tiles per item (the same for every item), and the key count of each
   // of the first kPipeMaxTable tiles in shared memory (thread 0 writes it; the
   // set-up barrier below publishes it)
@@ -344,13 +352,13 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
 
       bool ok = true;
       bool prev = false, prev_first = false;
-      int prev_nk16 = 0, prev_nqt = 0, prev_kvs = 0;
+      int prev_nk16 = 0, prev_qlo = 0, prev_qhi = 0, prev_kvs = 0;
       int nq[NQT], iq[NQT], prev_n[NQT];  // per query tile: tiles so far, items so far, last tile
 #pragma unroll
       for (int qt = 0; qt < NQT; ++qt) nq[qt] = iq[qt] = prev_n[qt] = 0;
       int g = 0;
-      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-        const int nqt = item_nqt(item);
+      for (int item = blockIdx.x, k = 0; ok && item < n_items; item += gridDim.x, ++k) {
+        const int qlo = item_qlo(k), qhi = item_qhi(k, item);
         Walk w;
         w.reset();
         for (int j = 0; j < T; ++j, ++g) {
@@ -361,12 +369,12 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           if (j == 0) {
 #pragma unroll
             for (int qt = 0; qt < NQT; ++qt)
-              if (qt < nqt && ok) ok = mbar_wait_bounded(q_full(qt), iq[qt]++ & 1);
+              if (qt >= qlo && qt < qhi && ok) ok = mbar_wait_bounded(q_full(qt), iq[qt]++ & 1);
             if (!ok) break;
           }
 #pragma unroll
           for (int qt = 0; qt < NQT; ++qt) {
-            if (qt < nqt && ok) {
+            if (qt >= qlo && qt < qhi && ok) {
               const int n = nq[qt];
               const int slot = n % NS;
               if (n >= NS) ok = mbar_wait_bounded(pv_done(qt, slot), ((n / NS) - 1) & 1);
@@ -380,7 +388,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           if (prev) {
 #pragma unroll
             for (int qt = 0; qt < NQT; ++qt) {
-              if (qt < prev_nqt && ok) {
+              if (qt >= prev_qlo && qt < prev_qhi && ok) {
                 const int n = prev_n[qt];
                 ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1);
                 if (ok) {
@@ -395,17 +403,18 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           prev = true;
           prev_first = (j == 0);
           prev_nk16 = nk16;
-          prev_nqt = nqt;
+          prev_qlo = qlo;
+          prev_qhi = qhi;
           prev_kvs = kvs;
 #pragma unroll
           for (int qt = 0; qt < NQT; ++qt)
-            if (qt < nqt) prev_n[qt] = nq[qt]++;
+            if (qt >= qlo && qt < qhi) prev_n[qt] = nq[qt]++;
         }
       }
       if (ok && prev) {
 #pragma unroll
         for (int qt = 0; qt < NQT; ++qt) {
-          if (qt < prev_nqt && ok) {
+          if (qt >= prev_qlo && qt < prev_qhi && ok) {
             const int n = prev_n[qt];
             ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1);
             if (ok) {
@@ -584,10 +593,22 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tq = tmem + lane_off + qt * C::TM_QT;
     const uint32_t qs = sbase + C::Q0 + qt * C::Q_SZ;
-    const uint32_t qst = sbase + C::QST0 + qt * C::QST_SZ;
-    auto row_of = [&](int item) { return (item % n_groups) * NQT * 128 + qt * 128 + row; };
+    const uint32_t qst = sbase + C::QST0 + qt * C::QPF * C::QST_SZ;
+    // query row held by this thread's tensor-memory lane. With alternating
+    // items (one tile of n_q <= 128 queries) the second warpgroup puts its
+    // rows at the top of the tile, so the two groups' busy warps sit on
+    // different SM sub-partitions when n_q is small.
+    const int roff = (ALT && qt == 1) ? 128 - p.n_q : 0;
+    auto row_of = [&](int item) {
+      return ALT ? row - roff : (item % n_groups) * NQT * 128 + qt * 128 + row;
+    };
+    auto row_ok = [&](int item) {
+      const int r = row_of(item);
+      return r >= 0 && r < p.n_q;
+    };
     // next item of this CTA in which query tile qt holds queries
     auto next_item = [&](int item) {
+      if (ALT) return item + 2 * static_cast<int>(gridDim.x);
       for (item += gridDim.x; item < n_items && item_nqt(item) <= qt; item += gridDim.x) {
       }
       return item;
@@ -597,42 +618,56 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
       return p.q + b * p.q_sb + h * p.q_sh + static_cast<int64_t>(row_of(item)) * p.q_st;
     };
-    // the next item's query row -> staging (chunk c of the row at c ^ (row & 7))
-    auto stage_q = [&](int item) {
-      const bool valid = row_of(item) < p.n_q;
-      const uint16_t* src = valid ? q_ptr(item) : p.q;
+    // a later item's query row -> staging buffer `buf` (chunk c of the row at
+    // c ^ (row & 7)); one commit group per call, empty when there is no item
+    auto stage_q = [&](int item, int buf) {
+      if (item < n_items) {
+        const bool valid = row_ok(item);
+        const uint16_t* src = valid ? q_ptr(item) : p.q;
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c)
-        cp_async16(qst + (row * (D / 8) + (c ^ (row & 7))) * 16, src + 8 * c, valid ? 16u : 0u);
+        for (int c = 0; c < D / 8; ++c)
+          cp_async16(qst + buf * C::QST_SZ + (row * (D / 8) + (c ^ (row & 7))) * 16, src + 8 * c, valid ? 16u : 0u);
+      }
       cp_async_commit();
     };
     // query row of `item` -> fp16 q * 2^-eq in the K-major SW128 A tile; returns 2^eq.
     // Two passes over the row (maximum, then conversion), 8 values at a time.
-    auto q_chunk = [&](int item, int c) -> uint4 {
+    auto q_chunk = [&](int item, int buf, int c) -> uint4 {
       if constexpr (C::STAGE_Q) {
-        return lds128(sm + C::QST0 + qt * C::QST_SZ + (row * (D / 8) + (c ^ (row & 7))) * 16);
+        return lds128(sm + C::QST0 + (qt * C::QPF + buf) * C::QST_SZ + (row * (D / 8) + (c ^ (row & 7))) * 16);
       } else {
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (row_of(item) < p.n_q) v = *reinterpret_cast<const uint4*>(q_ptr(item) + 8 * c);
+        if (row_ok(item)) v = *reinterpret_cast<const uint4*>(q_ptr(item) + 8 * c);
         return v;
       }
     };
-    auto convert_q = [&](int item) -> float {
-      if constexpr (C::STAGE_Q) cp_async_wait_all();
-      float amax = 0.0f;
-#pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 v = q_chunk(item, c);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[k] << 16)), fabsf(__uint_as_float(w[k] & 0xffff0000u))));
+    auto convert_q = [&](int item, int buf) -> float {
+      // the staging group of `item` is complete once at most QPF - 1 newer ones are pending
+      if constexpr (C::STAGE_Q) {
+        if constexpr (C::QPF == 2) {
+          asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+          cp_async_wait_all();
+        }
       }
+      // two passes over the row (8 values per 16-byte chunk): the maximum |q|
+      // on the magnitudes as packed 16-bit integers (same order as the values)
+      // in four independent accumulators, then the conversion
+      uint32_t am[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = q_chunk(item, buf, c);
+        am[0] = __vmaxu2(am[0], v.x & 0x7fff7fffu);
+        am[1] = __vmaxu2(am[1], v.y & 0x7fff7fffu);
+        am[2] = __vmaxu2(am[2], v.z & 0x7fff7fffu);
+        am[3] = __vmaxu2(am[3], v.w & 0x7fff7fffu);
+      }
+      const uint32_t a2 = __vmaxu2(__vmaxu2(am[0], am[1]), __vmaxu2(am[2], am[3]));
       float mul, inv;
-      pipe_pow2(amax, mul, inv);
+      pipe_pow2(__uint_as_float(max(a2 & 0xffffu, a2 >> 16) << 16), mul, inv);
 #pragma unroll 4
       for (int c = 0; c < D / 8; ++c) {
-        const uint4 v = q_chunk(item, c);
+        const uint4 v = q_chunk(item, buf, c);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t h[4];
 #pragma unroll
@@ -647,7 +682,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     };
     auto epilogue = [&](int item, float l, float vmul) {
       const int r = row_of(item);
-      const bool valid = r < p.n_q;
+      const bool valid = row_ok(item);
       const int bh = item / n_groups;
       const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
       const int64_t obase = b * p.o_sb + h * p.o_sh + static_cast<int64_t>(r) * p.o_st;
@@ -658,13 +693,12 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         tc::tmem_ld16(tq + C::COL_O + c16, o);
         tc::tmem_wait_ld();
         if (!valid) continue;
-        float* v = reinterpret_cast<float*>(o);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(o[k]) * scl;
         if (p.out_f32) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + c16);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_float4(__uint_as_float(o[4 * k]) * scl, __uint_as_float(o[4 * k + 1]) * scl,
+                                 __uint_as_float(o[4 * k + 2]) * scl, __uint_as_float(o[4 * k + 3]) * scl);
         } else {
           uint32_t bf[8];
 #pragma unroll
@@ -672,7 +706,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             uint32_t pair = 0;
 #pragma unroll
             for (int uu = 0; uu < 2; ++uu) {
-              const uint32_t x = __float_as_uint(v[2 * k + uu]);
+              const uint32_t x = __float_as_uint(__uint_as_float(o[2 * k + uu]) * scl);
               pair |= ((x + 0x7fffu + ((x >> 16) & 1u)) >> 16) << (16 * uu);
             }
             bf[k] = pair;
@@ -710,12 +744,16 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     };
 
     bool ok = true;
-    int item = blockIdx.x;
-    if (item < n_items && item_nqt(item) <= qt) item = next_item(item);
+    int item = blockIdx.x + (ALT ? qt * static_cast<int>(gridDim.x) : 0);
+    if (!ALT && item < n_items && item_nqt(item) <= qt) item = next_item(item);
     float qmul = 1.0f;  // 2^eq of the current item's row
+    int kq = 0;         // items of this query tile so far (staging buffer of item k: k % QPF)
     if (item < n_items) {
-      if constexpr (C::STAGE_Q) stage_q(item);
-      qmul = convert_q(item);
+      if constexpr (C::STAGE_Q) {
+        stage_q(item, 0);
+        if constexpr (C::QPF == 2) stage_q(next_item(item), 1);
+      }
+      qmul = convert_q(item, 0);
     }
     int g = 0;  // tiles of this query tile so far (S/P slot counter)
     bool epi = false;
@@ -727,10 +765,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       const int nxt = next_item(item);
       // this item's first tile in the CTA-wide tile sequence (K/V slot and header)
       const int gt0 = ((item - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x)) * T;
-      const bool warp_active = __any_sync(0xffffffffu, row_of(item) < p.n_q);
-      if constexpr (C::STAGE_Q) {
-        if (nxt < n_items) stage_q(nxt);
-      }
+      const bool warp_active = __any_sync(0xffffffffu, row_ok(item));
+      // queries of the item QPF ahead, into the buffer item kq just freed
+      if constexpr (C::STAGE_Q) stage_q(C::QPF == 2 ? (nxt < n_items ? next_item(nxt) : n_items) : nxt, kq % C::QPF);
       float up = 0.0f, vmul = 1.0f, m_ref = -INFINITY, l = 0.0f, qmul_next = qmul;
       Walk w;
       w.reset();
@@ -747,7 +784,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           vmul = hdr[(gt0 % NKV) * 4 + 1];
         }
         // last QK^T of this item has completed: q of the next item can replace it
-        if (j == T - 1 && nxt < n_items) qmul_next = convert_q(nxt);
+        if (j == T - 1 && nxt < n_items) qmul_next = convert_q(nxt, (kq + 1) % C::QPF);
         if (warp_active) {
           const uint32_t t_s = tq + slot * KT;
           uint32_t sr[64];
@@ -845,6 +882,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       epi_active = warp_active;
       qmul = qmul_next;
       item = nxt;
+      ++kq;
     }
     if (ok && epi && epi_active) {
       if (mbar_wait_bounded(pv_done(qt, (g - 1) % NS), ((g - 1) / NS) & 1)) {
@@ -861,7 +899,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   if (warp == 0) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int BITS, int D, int NQT>
+template <int BITS, int D, int NQT, bool ALT>
 cudaError_t launch_attention_pipe(const AttnParams& p, cudaStream_t stream) {
   using C = PipeCfg<BITS, D, NQT>;
   static bool configured[kMaxDevices] = {};
@@ -871,24 +909,24 @@ cudaError_t launch_attention_pipe(const AttnParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(attention_pipe_kernel<BITS, D, NQT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(attention_pipe_kernel<BITS, D, NQT, ALT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attention_pipe_kernel<BITS, D, NQT>, C::THREADS,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attention_pipe_kernel<BITS, D, NQT, ALT>, C::THREADS,
                                                       C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     configured[dev] = true;
   }
   const int n_qt = (p.n_q + 127) / 128;
-  const int64_t n_items = static_cast<int64_t>(p.B) * p.H * ((n_qt + NQT - 1) / NQT);
+  const int64_t n_items = static_cast<int64_t>(p.B) * p.H * (ALT ? n_qt : (n_qt + NQT - 1) / NQT);
   if (n_items > (int64_t(1) << 30)) return cudaErrorInvalidConfiguration;
   // one CTA per SM: all 512 tensor-memory columns are this CTA's
   const int grid = static_cast<int>(n_items < sms[dev] ? n_items : sms[dev]);
-  attention_pipe_kernel<BITS, D, NQT><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(p);
+  attention_pipe_kernel<BITS, D, NQT, ALT><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(p);
   return cudaGetLastError();
 }
 
