@@ -30,12 +30,15 @@
 //     turns on the tensor cores and hide each other's tensor-memory latency;
 //   unpack warps (8 with one query tile, 4 with two): staged packed words ->
 //     dequantized fp16 hi/lo K and V tiles (ring of NKV slots) shared by the
-//     item's query tiles, and the per-(batch, head) powers of two;
+//     item's query tiles, and the per-(batch, head) powers of two. With a
+//     two-slot ring (head_dim 128) K and V of a slot are released and refilled
+//     separately: the next K overlaps the PV that still reads this slot's V;
 //   producer warp, one thread: bulk copies of each tile's packed K/V word
 //     rows and of its blocks' scale/zero vectors into a stage ring;
 //   MMA warp, one thread: every tcgen05.mma, with shared-memory descriptors
 //     built once and advanced by constant offsets: QK^T of tile g for each
-//     query tile, then PV of tile g-1 for each.
+//     query tile, then PV of tile g-1 for each (the hi/lo parts of one k-step
+//     back to back).
 // The CTA is persistent: it walks work items (batch*head, group of NQT query
 // tiles) with a stride of gridDim.x. Every ring runs on across items, so the
 // next item's copies, unpacking and first QK^T overlap this item's last tiles,
@@ -69,6 +72,10 @@ struct PipeCfg {
   static constexpr int NS = (NQT == 1) ? 4 : ((D == 64) ? 3 : 2);  // S slots per query tile
   static constexpr int NKV = (D == 64) ? (NQT == 1 ? 4 : 3) : (NQT == 1 ? 3 : 2);  // K/V tile slots
   static constexpr int NSTG = 2;                           // packed-word stages
+  // K and V of a tile are unpacked as two phases, each announced on its own,
+  // when the K/V ring is short (K of a later tile then overlaps the PV that
+  // still holds the slot's V); otherwise as one
+  static constexpr bool SPLIT_KV = (NKV <= 2);
   static constexpr bool STAGE_Q = (D == 64);               // queries of later items prefetched by cp.async
   static constexpr int QPF = (STAGE_Q && NQT == 1) ? 2 : 1;  // items ahead the query staging runs
   static constexpr int UNPACK_WARPS = (NQT == 1) ? 8 : 4;
@@ -96,7 +103,7 @@ struct PipeCfg {
   static constexpr int RED0 = HDR0 + NKV * 16;             // NRED x {K, V} x UNPACK_WARPS floats
   static constexpr int BARS = RED0 + NRED * 2 * UNPACK_WARPS * 4;
   static constexpr int QBARS = 1 + 3 * NS;                 // per query tile: q_full, s_full, p_full, pv_done
-  static constexpr int NBARS = 2 * NSTG + 2 * NKV + NRED + NQT * QBARS;
+  static constexpr int NBARS = 2 * NSTG + 4 * NKV + NRED + NQT * QBARS;
   static constexpr int TMEM_SLOT = BARS + NBARS * 8;
   static constexpr int NKTAB = TMEM_SLOT + 16;             // kPipeMaxTable x uint8: keys of each tile of an item
   static constexpr int SMEM = NKTAB + kPipeMaxTable;
@@ -181,9 +188,11 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::BARS);
   uint64_t* stg_full = bars;
   uint64_t* stg_empty = stg_full + NSTG;
-  uint64_t* kv_full = stg_empty + NSTG;
-  uint64_t* kv_empty = kv_full + NKV;
-  uint64_t* red_bar = kv_empty + NKV;
+  uint64_t* k_full = stg_empty + NSTG;  // K (and, unsplit, V) of a slot unpacked
+  uint64_t* v_full = k_full + NKV;      // V of a slot unpacked; the slot's header written
+  uint64_t* k_empty = v_full + NKV;     // QK^T of the slot's tile complete
+  uint64_t* v_empty = k_empty + NKV;    // PV of the slot's tile complete
+  uint64_t* red_bar = v_empty + NKV;
   uint64_t* qbars = red_bar + C::NRED;
   auto q_full = [&](int qt) { return qbars + qt * C::QBARS; };
   auto s_full = [&](int qt, int i) { return qbars + qt * C::QBARS + 1 + i; };
@@ -231,8 +240,10 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       mbar_init(&stg_empty[i], C::UNPACK_THREADS);
     }
     for (int i = 0; i < NKV; ++i) {
-      mbar_init(&kv_full[i], C::UNPACK_THREADS);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_full[i], C::UNPACK_THREADS);
+      mbar_init(&v_full[i], C::UNPACK_THREADS);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < C::NRED; ++i) mbar_init(&red_bar[i], C::UNPACK_WARPS);
     for (int qt = 0; qt < NQT; ++qt) {
@@ -319,9 +330,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         const uint64_t kd = kdesc0 + static_cast<uint64_t>((kvs * C::KV_SZ) >> 4);
         const uint32_t d = tmem + qt * C::TM_QT + slot * KT;
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+        for (int kk = 0; kk < D / 16; ++kk) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int part = 0; part < 2; ++part) {
             constexpr int kSlabA = 128 * 128, kSlabB = KT * 128;
             const uint32_t aoff = ((kk >> 2) * kSlabA + (kk & 3) * 32) >> 4;
             const uint32_t boff = (part * C::TILE_SZ + (kk >> 2) * kSlabB + (kk & 3) * 32) >> 4;
@@ -337,11 +348,11 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         const int nkk = nk16 / 16;
         // (A part, B part): (P hi, V hi), (P lo, V hi), (P hi, V lo)
 #pragma unroll
-        for (int part = 0; part < 3; ++part) {
-          const uint32_t acol = (part == 1) ? 8u : 0u;
-          const uint32_t vpart = (part == 2) ? (C::TILE_SZ >> 4) : 0u;
+        for (int kk = 0; kk < KT / 16; ++kk) {
 #pragma unroll
-          for (int kk = 0; kk < KT / 16; ++kk) {
+          for (int part = 0; part < 3; ++part) {
+            const uint32_t acol = (part == 1) ? 8u : 0u;
+            const uint32_t vpart = (part == 2) ? (C::TILE_SZ >> 4) : 0u;
             if (kk < nkk)
               tc::mma_f16_ts(o, pa + 16 * kk + acol, vd + vpart + ((kk * 2048) >> 4), idesc_pv,
                                 (first && part == 0 && kk == 0) ? 0u : 1u);
@@ -352,7 +363,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
 
       bool ok = true;
       bool prev = false, prev_first = false;
-      int prev_nk16 = 0, prev_qlo = 0, prev_qhi = 0, prev_kvs = 0;
+      int prev_nk16 = 0, prev_qlo = 0, prev_qhi = 0, prev_kvs = 0, prev_g = 0;
       int nq[NQT], iq[NQT], prev_n[NQT];  // per query tile: tiles so far, items so far, last tile
 #pragma unroll
       for (int qt = 0; qt < NQT; ++qt) nq[qt] = iq[qt] = prev_n[qt] = 0;
@@ -365,7 +376,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           const int nk = tabled ? nktab[j] : w.next(p);
           const int nk16 = (nk + 15) & ~15;
           const int kvs = g % NKV;
-          if (!(ok = mbar_wait_bounded(&kv_full[kvs], (g / NKV) & 1))) break;
+          if (!(ok = mbar_wait_bounded(&k_full[kvs], (g / NKV) & 1))) break;
           if (j == 0) {
 #pragma unroll
             for (int qt = 0; qt < NQT; ++qt)
@@ -385,7 +396,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             }
           }
           if (!ok) break;
+          if constexpr (C::SPLIT_KV) tc::commit(&k_empty[kvs]);
           if (prev) {
+            if (C::SPLIT_KV && !(ok = mbar_wait_bounded(&v_full[prev_kvs], (prev_g / NKV) & 1))) break;
 #pragma unroll
             for (int qt = 0; qt < NQT; ++qt) {
               if (qt >= prev_qlo && qt < prev_qhi && ok) {
@@ -398,7 +411,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
               }
             }
             if (!ok) break;
-            tc::commit(&kv_empty[prev_kvs]);
+            tc::commit(&v_empty[prev_kvs]);
           }
           prev = true;
           prev_first = (j == 0);
@@ -406,11 +419,13 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           prev_qlo = qlo;
           prev_qhi = qhi;
           prev_kvs = kvs;
+          prev_g = g;
 #pragma unroll
           for (int qt = 0; qt < NQT; ++qt)
             if (qt >= qlo && qt < qhi) prev_n[qt] = nq[qt]++;
         }
       }
+      if (C::SPLIT_KV && ok && prev) ok = mbar_wait_bounded(&v_full[prev_kvs], (prev_g / NKV) & 1);
       if (ok && prev) {
 #pragma unroll
         for (int qt = 0; qt < NQT; ++qt) {
@@ -423,7 +438,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             }
           }
         }
-        if (ok) tc::commit(&kv_empty[prev_kvs]);
+        if (ok) tc::commit(&v_empty[prev_kvs]);
       }
     }
   } else if (tid >= C::UNPACK_T0) {
@@ -499,11 +514,8 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         const int st = g % NSTG;
         const int kvs = g % NKV;
         if (!(ok = mbar_wait_bounded(&stg_full[st], (g / NSTG) & 1))) break;
-        if (!(ok = mbar_wait_bounded(&kv_empty[kvs], ((g / NKV) & 1) ^ 1))) break;
-        if (j == 0 && ut == 0) {
-          hdr[kvs * 4 + 0] = kmul;
-          hdr[kvs * 4 + 1] = vmul;
-        }
+        // (unsplit, the slot's V release below also covers its K)
+        if (C::SPLIT_KV && !(ok = mbar_wait_bounded(&k_empty[kvs], ((g / NKV) & 1) ^ 1))) break;
         const unsigned char* stage = sm + C::STG0 + st * C::STG_SZ;
         const int4* segt = reinterpret_cast<const int4*>(stage + C::STG_SEG);
         const int* rows = reinterpret_cast<const int*>(stage + C::STG_ROWS);
@@ -511,77 +523,93 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         const int R = rows[2 * (nseg - 1)] + rows[2 * (nseg - 1) + 1];  // staged word rows
         const uint32_t kvbase = sbase + C::KV0 + kvs * C::KV_SZ;
         constexpr int OCT = D / 8;
-        for (int task = ut; task < 2 * R * OCT; task += C::UNPACK_THREADS) {
-          const int tsel = task >= R * OCT ? 1 : 0;
-          const int r = task - tsel * R * OCT;
-          const int sr = r / OCT;
-          const int jj = r - sr * OCT;
-          // the segment of staged row sr
-          int i = 0;
-          while (i + 1 < nseg && rows[2 * (i + 1)] <= sr) ++i;
-          const int4 sg = segt[i];  // {block, u0, take, key0}
-          const uint32_t* src = reinterpret_cast<const uint32_t*>(stage + tsel * C::STG_V) + sr * D + 8 * jj;
-          // lanes jj and jj+4 of a quarter-warp would hit the same banks with
-          // 32-byte strided 16-byte loads; odd quads read their halves swapped
-          const int sw = (jj >> 2) & 1;
-          const uint4 a0 = *reinterpret_cast<const uint4*>(src + 4 * sw);
-          const uint4 a1 = *reinterpret_cast<const uint4*>(src + 4 * (sw ^ 1));
-          const uint4 a = sw ? a1 : a0;
-          const uint4 bq = sw ? a0 : a1;
-          const uint32_t wd[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
-          const float* meta =
-              reinterpret_cast<const float*>(stage + C::STG_META) + (i * 4 + 2 * tsel) * D + 8 * jj;
-          const float mul = tsel ? vinv : kinv;
-          float sc[8], ze[8];  // scale and zero of the 8 channels, times 2^-e (exact)
-          {
-            const uint4 s0 = *reinterpret_cast<const uint4*>(meta + 4 * sw);
-            const uint4 s1 = *reinterpret_cast<const uint4*>(meta + 4 * (sw ^ 1));
-            const uint4 z0 = *reinterpret_cast<const uint4*>(meta + D + 4 * sw);
-            const uint4 z1 = *reinterpret_cast<const uint4*>(meta + D + 4 * (sw ^ 1));
-            const uint4 sa = sw ? s1 : s0, sb = sw ? s0 : s1;
-            const uint4 za = sw ? z1 : z0, zb = sw ? z0 : z1;
-            const uint32_t sv8[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
-            const uint32_t zv8[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+        // task t < R * OCT: K, word row t / OCT, channels 8 (t % OCT) ..; then V likewise
+        auto unpack_tasks = [&](int t0, int t1) {
+          for (int task = t0 + ut; task < t1; task += C::UNPACK_THREADS) {
+            const int tsel = task >= R * OCT ? 1 : 0;
+            const int r = task - tsel * R * OCT;
+            const int sr = r / OCT;
+            const int jj = r - sr * OCT;
+            // the segment of staged row sr
+            int i = 0;
+            while (i + 1 < nseg && rows[2 * (i + 1)] <= sr) ++i;
+            const int4 sg = segt[i];  // {block, u0, take, key0}
+            const uint32_t* src = reinterpret_cast<const uint32_t*>(stage + tsel * C::STG_V) + sr * D + 8 * jj;
+            // lanes jj and jj+4 of a quarter-warp would hit the same banks with
+            // 32-byte strided 16-byte loads; odd quads read their halves swapped
+            const int sw = (jj >> 2) & 1;
+            const uint4 a0 = *reinterpret_cast<const uint4*>(src + 4 * sw);
+            const uint4 a1 = *reinterpret_cast<const uint4*>(src + 4 * (sw ^ 1));
+            const uint4 a = sw ? a1 : a0;
+            const uint4 bq = sw ? a0 : a1;
+            const uint32_t wd[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+            const float* meta =
+                reinterpret_cast<const float*>(stage + C::STG_META) + (i * 4 + 2 * tsel) * D + 8 * jj;
+            const float mul = tsel ? vinv : kinv;
+            float sc[8], ze[8];  // scale and zero of the 8 channels, times 2^-e (exact)
+            {
+              const uint4 s0 = *reinterpret_cast<const uint4*>(meta + 4 * sw);
+              const uint4 s1 = *reinterpret_cast<const uint4*>(meta + 4 * (sw ^ 1));
+              const uint4 z0 = *reinterpret_cast<const uint4*>(meta + D + 4 * sw);
+              const uint4 z1 = *reinterpret_cast<const uint4*>(meta + D + 4 * (sw ^ 1));
+              const uint4 sa = sw ? s1 : s0, sb = sw ? s0 : s1;
+              const uint4 za = sw ? z1 : z0, zb = sw ? z0 : z1;
+              const uint32_t sv8[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+              const uint32_t zv8[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              sc[u] = __uint_as_float(sv8[u]) * mul;
-              ze[u] = __uint_as_float(zv8[u]) * mul;
+              for (int u = 0; u < 8; ++u) {
+                sc[u] = __uint_as_float(sv8[u]) * mul;
+                ze[u] = __uint_as_float(zv8[u]) * mul;
+              }
             }
-          }
-          // block token of slot 0 of this word row, and its tile key
-          const int ub = (sg.y / CPW + (sr - rows[2 * i])) * CPW;
-          const int kbase = sg.w + ub - sg.y;
-          const int s_lo = max(0, sg.y - ub), s_hi = min(CPW, sg.y + sg.z - ub);  // valid slots
-          // key row r of the [KT][D] tile: byte r * 128 + ((octet ^ (r & 7)) << 4) in its 64-channel slab
-          const uint32_t dst = kvbase + tsel * 2 * C::TILE_SZ + (jj >> 3) * KT * 128;
-          const uint32_t oct = jj & 7;
+            // block token of slot 0 of this word row, and its tile key
+            const int ub = (sg.y / CPW + (sr - rows[2 * i])) * CPW;
+            const int kbase = sg.w + ub - sg.y;
+            const int s_lo = max(0, sg.y - ub), s_hi = min(CPW, sg.y + sg.z - ub);  // valid slots
+            // key row r of the [KT][D] tile: byte r * 128 + ((octet ^ (r & 7)) << 4) in its 64-channel slab
+            const uint32_t dst = kvbase + tsel * 2 * C::TILE_SZ + (jj >> 3) * KT * 128;
+            const uint32_t oct = jj & 7;
 #pragma unroll 1
-          for (int s = s_lo; s < s_hi; ++s) {
-            const int sh = BITS * s;
-            const uint32_t row = static_cast<uint32_t>(kbase + s);
-            float h[8], l[8];
+            for (int s = s_lo; s < s_hi; ++s) {
+              const int sh = BITS * s;
+              const uint32_t row = static_cast<uint32_t>(kbase + s);
+              float h[8], l[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              // code c as the float 2^23 + c, minus 2^23: exact; then fma(c, scale, zero) * 2^-e
-              const float c = __uint_as_float(((wd[u] >> sh) & C::MASK) | 0x4B000000u) - 8388608.0f;
-              const float x = fmaf(c, sc[u], ze[u]);
-              h[u] = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
-              l[u] = x - h[u];
-            }
-            uint32_t hi[4], lo[4];
+              for (int u = 0; u < 8; ++u) {
+                // code c as the float 2^23 + c, minus 2^23: exact; then fma(c, scale, zero) * 2^-e
+                const float c = __uint_as_float(((wd[u] >> sh) & C::MASK) | 0x4B000000u) - 8388608.0f;
+                const float x = fmaf(c, sc[u], ze[u]);
+                h[u] = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
+                l[u] = x - h[u];
+              }
+              uint32_t hi[4], lo[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              hi[u] = tc::cvt_half2(h[2 * u], h[2 * u + 1]);
-              lo[u] = tc::cvt_half2(l[2 * u], l[2 * u + 1]);
+              for (int u = 0; u < 4; ++u) {
+                hi[u] = tc::cvt_half2(h[2 * u], h[2 * u + 1]);
+                lo[u] = tc::cvt_half2(l[2 * u], l[2 * u + 1]);
+              }
+              const uint32_t off = row * 128 + ((oct ^ (row & 7)) << 4);
+              tc::sts128(dst + off, hi[0], hi[1], hi[2], hi[3]);
+              tc::sts128(dst + C::TILE_SZ + off, lo[0], lo[1], lo[2], lo[3]);
             }
-            const uint32_t off = row * 128 + ((oct ^ (row & 7)) << 4);
-            tc::sts128(dst + off, hi[0], hi[1], hi[2], hi[3]);
-            tc::sts128(dst + C::TILE_SZ + off, lo[0], lo[1], lo[2], lo[3]);
           }
+        };
+        if constexpr (C::SPLIT_KV) {
+          unpack_tasks(0, R * OCT);
+          fence_proxy_async_smem();
+          mbar_arrive(&k_full[kvs]);
         }
+        // V of this slot's previous tile is free once its PV has completed
+        if (!(ok = mbar_wait_bounded(&v_empty[kvs], ((g / NKV) & 1) ^ 1))) break;
+        if (j == 0 && ut == 0) {
+          hdr[kvs * 4 + 0] = kmul;
+          hdr[kvs * 4 + 1] = vmul;
+        }
+        unpack_tasks(C::SPLIT_KV ? R * OCT : 0, 2 * R * OCT);
         fence_proxy_async_smem();
         mbar_arrive(&stg_empty[st]);
-        mbar_arrive(&kv_full[kvs]);
+        if constexpr (!C::SPLIT_KV) mbar_arrive(&k_full[kvs]);
+        mbar_arrive(&v_full[kvs]);
         // the next item's maxima, while this item's tiles run
         if (j == 0 && item + static_cast<int>(gridDim.x) < n_items) pow2_post(item + gridDim.x, k + 1);
       }
@@ -608,10 +636,13 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     };
     // next item of this CTA in which query tile qt holds queries
     auto next_item = [&](int item) {
-      if (ALT) return item + 2 * static_cast<int>(gridDim.x);
-      for (item += gridDim.x; item < n_items && item_nqt(item) <= qt; item += gridDim.x) {
+      if constexpr (ALT) {
+        return item + 2 * static_cast<int>(gridDim.x);
+      } else {
+        for (item += gridDim.x; item < n_items && item_nqt(item) <= qt; item += gridDim.x) {
+        }
+        return item;
       }
-      return item;
     };
     auto q_ptr = [&](int item) -> const uint16_t* {
       const int bh = item / n_groups;
@@ -779,7 +810,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         tc::fence_after_sync();
         if (j == 0) {
           // the unpack warps' powers of two for this item (header of its first tile)
-          if (!(ok = mbar_wait_bounded(&kv_full[gt0 % NKV], (gt0 / NKV) & 1))) break;
+          if (!(ok = mbar_wait_bounded(&v_full[gt0 % NKV], (gt0 / NKV) & 1))) break;
           up = p.softmax_scale * qmul * hdr[(gt0 % NKV) * 4 + 0];
           vmul = hdr[(gt0 % NKV) * 4 + 1];
         }
