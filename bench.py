@@ -44,6 +44,38 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
+# DRAM bytes per layer of each kernel family, from one ncu capture of layer 0
+# (profiles/dram_traffic.json); valid only while the kernels' sources are the
+# ones that capture ran.
+KERNEL_SOURCES = {
+    "attention": ("attention.cuh", "attention_pipe.cuh", "tc_ptx.cuh", "vq_device.cuh"),
+    "quant_pack": ("quant_pack.cuh", "vq_device.cuh"),
+}
+
+
+def kernel_sources_sha256(family):
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[family]:
+        with open(os.path.join(ROOT, "bit_kv_cache_25_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload, family, layers):
+    """(DRAM bytes per step, note): the captured bytes of one layer times the
+    layer count (every layer has the same shapes), or (None, why not)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None, "no capture"
+    e = json.load(open(p)).get(workload, {}).get(family)
+    if not e:
+        return None, "no capture of this workload"
+    if e.get("sources_sha256") != kernel_sources_sha256(family):
+        return None, "kernel sources changed since the capture"
+    return e["bytes_per_layer"] * layers, f"ncu capture of layer 0 ({e['launches_per_layer']} launches) x {layers} layers"
+
+
 # ------------------------------------------------------------------ algorithmic work
 def word_rows(n, bits):
     c = 32 // bits
@@ -386,12 +418,16 @@ def run_ours(args):
     a_bound = "hbm" if a_bytes / (hbm * 1e9) >= a_flops / (tc * 1e12) else "tensor"
     a_frac = (a_gbs / hbm) if a_bound == "hbm" else (a_tflops / tc)
     if a_ms >= q_ms:
+        traffic, tnote = measured_traffic(w.name, "attention", L)
         roof = {"kernel": "attention", "bound": a_bound, "achieved": a_gbs if a_bound == "hbm" else a_tflops,
                 "peak": hbm if a_bound == "hbm" else tc, "unit": "GB/s" if a_bound == "hbm" else "TFLOP/s",
-                "frac": a_frac, "traffic": None}
+                "frac": a_frac, "traffic": traffic, "algorithmic_bytes": a_bytes}
     else:
+        traffic, tnote = measured_traffic(w.name, "quant_pack", L)
         roof = {"kernel": "quant_pack", "bound": "hbm", "achieved": q_gbs, "peak": hbm, "unit": "GB/s",
-                "frac": q_gbs / hbm, "traffic": None}
+                "frac": q_gbs / hbm, "traffic": traffic, "algorithmic_bytes": q_bytes}
+    roof["traffic_unit"] = "DRAM bytes read + written per step (all launches of the kernel family in one decode)"
+    roof["traffic_source"] = tnote
     roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
 
     line = {
