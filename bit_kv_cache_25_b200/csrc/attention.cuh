@@ -6,30 +6,44 @@
 // but no attention kernel. The plainest reading: block s is appended, then its
 // queries attend to all of blocks 0..s (no mask within or across blocks).
 //
-// Scales are folded in. With k = code_k * sk + zk per (block, channel) and
-// v = code_v * sv + zv:
-//   logit(i, t) = sum_c (sigma q_ic sk_c) code_k(t, c) + sum_c sigma q_ic zk_c
-//               = q'_i . code_k(t) + bias_i       (bias is per (query, block))
-//   out_i = sum_blocks [ sv (.) (P code_v) + zv * rowsum(P) ] / l_i
-// so the integer codes enter the products exactly and the per-block scales are
-// applied once per (query, block, channel).
+// Both kernels attend over the cache's own dequantized values
+// x^ = fma(code, scale, zero) of each token's block (fp32), rebuilt on chip
+// from the packed words tile by tile; no dequantized copy is kept in HBM.
 //
-// This file holds the kernel for blocks with few queries (fewer than
-// kTcMinQueries): one CTA per (b, h), one warp per query, lanes across
-// channels. Each key's logit is a warp reduction over channels; the softmax is
-// online in fp32 (one pass over the keys). The packed words of a word-row are
-// read once per warp and serve its cpw keys from L1.
+// This file holds the two CUDA-core kernels and the dispatch between them and
+// the tensor-core kernel (attention_pipe.cuh), by measured speed on the VAR
+// and Infinity shapes: at most 4 queries -> attention_small_kernel; up to 32
+// queries whose keys fit in shared memory -> attention_cc_kernel; the rest ->
+// attention_pipe_kernel (a 128-row MMA tile is mostly padding below that).
+//
+// attention_cc_kernel: one CTA per (b, h). The cache's values of blocks 0..s
+// are dequantized once into shared memory, x^ = fma(code, scale, zero) in
+// fp32 (K^ transposed, [D][PP + 1]; V^ row-major), the queries are converted once
+// (times sigma * log2 e), and the three steps run from shared memory in fp32:
+//   S = q K^T        warp tasks of 8 rows x 32 keys (one key per lane)
+//   P = 2^(S - max)  one warp per row, row sums kept for the output
+//   O = P V^ / l     warp tasks of 8 rows x D channels (D / 32 per lane)
+// Rows are padded to a multiple of 8 and keys to a multiple of 32 with zeros
+// (padded keys are masked to p = 0), so no task needs a bounds check.
 #pragma once
 
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
+#include "tc_ptx.cuh"
 #include "vq_internal.h"
 
 namespace vq {
 namespace {
 
+// ---- blocks of at most kSmallMaxQueries queries: one CTA per (b, h), one warp
+// per query, lanes across channels; each key's logit is a warp reduction over
+// channels and the softmax is online in fp32 (one pass over the keys), with
+// the integer codes in the products and the per-block scales applied once per
+// (query, block, channel). No shared memory and no CTA barrier: the lowest
+// latency for a handful of queries.
+constexpr int kSmallMaxQueries = 4;
 constexpr int kSmallWarps = 4;
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float(static_cast<uint32_t>(h) << 16); }
@@ -136,39 +150,279 @@ cudaError_t launch_attention_small(const AttnParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+
+// ---- attention_cc_kernel
+constexpr int kCcMaxSmem = 76 * 1024;  // three CTAs per SM at most this
+constexpr int kCcMaxQueries = 64;
+
+// Shared-memory plan of one CTA (offsets in floats).
+struct CcLayout {
+  int PP, NQP;              // keys padded to 32, rows padded to 8
+  int KS;                   // row stride of K^ (PP + 1: a warp's 32 channels of one key hit 32 banks)
+  int kt, vs, qs, ps, linv; // K^ [D][KS], V^ [PP][D], q [NQP][D], S/P [NQP][PP], 1/l [NQP]
+  int floats;
+};
+
+__host__ __device__ inline CcLayout cc_layout(int n_q, int P, int D) {
+  CcLayout L;
+  L.PP = (P + 31) & ~31;
+  L.NQP = (n_q + 7) & ~7;
+  L.KS = L.PP + 1;
+  L.kt = 0;
+  L.vs = (L.kt + D * L.KS + 3) & ~3;
+  L.qs = L.vs + L.PP * D;
+  L.ps = L.qs + L.NQP * D;
+  L.linv = L.ps + L.NQP * L.PP;
+  L.floats = L.linv + L.NQP;
+  return L;
+}
+
+// THREADS: 128 for up to 16 queries, 256 above (more warps for the same
+// shared memory once there are enough row and key tasks to share)
+template <int BITS, int D, int THREADS>
+__global__ void __launch_bounds__(THREADS, 3) attention_cc_kernel(const __grid_constant__ AttnParams p, int P) {
+  constexpr int kCcThreads = THREADS;
+  constexpr int kCcWarps = THREADS / 32;
+  constexpr int kCcBatch = THREADS == 128 ? 4 : 2;  // dequantize items per thread with loads in flight together
+  constexpr int CPW = 32 / BITS;
+  constexpr uint32_t MASK = (1u << BITS) - 1u;
+  constexpr int CH = D / 32;  // output channels per lane
+  extern __shared__ __align__(16) float smc[];
+  const int n_q = p.n_q;
+  const CcLayout L = cc_layout(n_q, P, D);
+  float* kt = smc + L.kt;
+  float* vs = smc + L.vs;
+  float* qs = smc + L.qs;
+  float* ps = smc + L.ps;
+  float* linv = smc + L.linv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.x;
+  const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+  const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
+  const int PP = L.PP, NQP = L.NQP, KS = L.KS;
+
+  // ---- padding: keys [P, PP) of K^ and V^, rows [n_q, NQP) of q are zero
+  for (int e = tid; e < D * (PP - P); e += kCcThreads) {
+    const int c = e % D, j = P + e / D;
+    kt[c * KS + j] = 0.0f;
+    vs[j * D + c] = 0.0f;
+  }
+  for (int e = n_q * D + tid; e < NQP * D; e += kCcThreads) qs[e] = 0.0f;
+  // ---- queries: bf16 -> fp32 times sigma * log2(e), 8 per 16-byte load
+  const float qmul = p.softmax_scale * 1.4426950408889634f;
+  for (int e = tid; e < n_q * (D / 8); e += kCcThreads) {
+    const int i = e / (D / 8), c8 = e - i * (D / 8);
+    const uint4 v = *reinterpret_cast<const uint4*>(p.q + b * p.q_sb + h * p.q_sh + static_cast<int64_t>(i) * p.q_st + 8 * c8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float* dst = qs + i * D + 8 * c8;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      dst[2 * k] = __uint_as_float(w[k] << 16) * qmul;
+      dst[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u) * qmul;
+    }
+  }
+  // ---- dequantize blocks 0..s: one (block, word row, channel) per item, kCcBatch items per thread in flight
+  int E = 0;
+  for (int kb = 0; kb <= p.s; ++kb) E += p.blk[kb].W * D;
+  for (int e0 = tid; e0 < E; e0 += kCcBatch * kCcThreads) {
+    uint32_t wk[kCcBatch], wv[kCcBatch];
+    float sk[kCcBatch], zk[kCcBatch], sv[kCcBatch], zv[kCcBatch];
+    int j0[kCcBatch], ns[kCcBatch], ch[kCcBatch];
+#pragma unroll
+    for (int u = 0; u < kCcBatch; ++u) {
+      const int e = e0 + u * kCcThreads;
+      ns[u] = 0;
+      ch[u] = 0;
+      j0[u] = 0;
+      wk[u] = wv[u] = 0u;
+      sk[u] = zk[u] = sv[u] = zv[u] = 0.0f;
+      if (e < E) {
+        int kb = 0, base = 0, key = 0;
+        while (e >= base + p.blk[kb].W * D) {
+          base += p.blk[kb].W * D;
+          key += p.blk[kb].n;
+          ++kb;
+        }
+        const int w = (e - base) / D, c = (e - base) - w * D;
+        const AttnBlockInfo& bi = p.blk[kb];
+        const int64_t off = bi.word_off + static_cast<int64_t>(bh) * bi.W * D + static_cast<int64_t>(w) * D + c;
+        const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + c;
+        wk[u] = __ldg(p.packed_k + off);
+        wv[u] = __ldg(p.packed_v + off);
+        sk[u] = __ldg(p.scale_k + mo);
+        zk[u] = __ldg(p.zero_k + mo);
+        sv[u] = __ldg(p.scale_v + mo);
+        zv[u] = __ldg(p.zero_v + mo);
+        j0[u] = key + w * CPW;
+        ns[u] = min(CPW, bi.n - w * CPW);
+        ch[u] = c;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCcBatch; ++u) {
+#pragma unroll
+      for (int i = 0; i < CPW; ++i) {
+        if (i < ns[u]) {
+          const float ck = static_cast<float>((wk[u] >> (BITS * i)) & MASK);
+          const float cv = static_cast<float>((wv[u] >> (BITS * i)) & MASK);
+          kt[ch[u] * KS + j0[u] + i] = fmaf(ck, sk[u], zk[u]);
+          vs[(j0[u] + i) * D + ch[u]] = fmaf(cv, sv[u], zv[u]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- S = q K^T: task (8 rows, 32 keys), key j = 32 kg + lane
+  const int nkg = PP / 32;
+  for (int t = warp; t < (NQP / 8) * nkg; t += kCcWarps) {
+    const int i0 = (t / nkg) * 8, j = (t - (t / nkg) * nkg) * 32 + lane;
+    float acc[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc[r] = 0.0f;
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      const float k0 = kt[c * KS + j], k1 = kt[(c + 1) * KS + j], k2 = kt[(c + 2) * KS + j], k3 = kt[(c + 3) * KS + j];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float4 qv = *reinterpret_cast<const float4*>(qs + (i0 + r) * D + c);
+        acc[r] = fmaf(qv.x, k0, fmaf(qv.y, k1, fmaf(qv.z, k2, fmaf(qv.w, k3, acc[r]))));
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) ps[(i0 + r) * PP + j] = acc[r];
+  }
+  __syncthreads();
+
+  // ---- softmax: warp per row; keys past P get p = 0
+  for (int i = warp; i < n_q; i += kCcWarps) {
+    float m = -INFINITY;
+    for (int j = lane; j < P; j += 32) m = fmaxf(m, ps[i * PP + j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.0f;
+    for (int j = lane; j < PP; j += 32) {
+      const float e = j < P ? tc::ex2(ps[i * PP + j] - m) : 0.0f;
+      ps[i * PP + j] = e;
+      l += e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) linv[i] = 1.0f / l;
+  }
+  __syncthreads();
+
+  // ---- O = P V^ / l: task of 8 rows, channels lane + 32 k
+  for (int t = warp; t < NQP / 8; t += kCcWarps) {
+    const int i0 = 8 * t;
+    float acc[8][CH];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int k = 0; k < CH; ++k) acc[r][k] = 0.0f;
+#pragma unroll 1
+    for (int j = 0; j < PP; j += 4) {
+      float vv[4][CH];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int k = 0; k < CH; ++k) vv[u][k] = vs[(j + u) * D + lane + 32 * k];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float4 pv = *reinterpret_cast<const float4*>(ps + (i0 + r) * PP + j);
+#pragma unroll
+        for (int k = 0; k < CH; ++k)
+          acc[r][k] = fmaf(pv.x, vv[0][k], fmaf(pv.y, vv[1][k], fmaf(pv.z, vv[2][k], fmaf(pv.w, vv[3][k], acc[r][k]))));
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int i = i0 + r;
+      if (i >= n_q) break;
+      const float sc = linv[i];
+      const int64_t obase = b * p.o_sb + h * p.o_sh + static_cast<int64_t>(i) * p.o_st;
+#pragma unroll
+      for (int k = 0; k < CH; ++k) {
+        const float val = acc[r][k] * sc;
+        if (p.out_f32) {
+          static_cast<float*>(p.out)[obase + lane + 32 * k] = val;
+        } else {
+          const uint32_t x = __float_as_uint(val);
+          static_cast<uint16_t*>(p.out)[obase + lane + 32 * k] =
+              static_cast<uint16_t>((x + 0x7fffu + ((x >> 16) & 1u)) >> 16);  // round to nearest even
+        }
+      }
+    }
+  }
+}
+
+// Keys of blocks 0..s.
+inline int attn_keys(const AttnParams& p) {
+  int P = 0;
+  for (int k = 0; k <= p.s; ++k) P += p.blk[k].n;
+  return P;
+}
+
+inline bool cc_fits(const AttnParams& p) {
+  const CcLayout L = cc_layout(p.n_q, attn_keys(p), p.D);
+  return p.n_q <= kCcMaxQueries && static_cast<size_t>(L.floats) * 4 <= kCcMaxSmem;
+}
+
+template <int BITS, int D, int THREADS>
+cudaError_t launch_attention_cc(const AttnParams& p, cudaStream_t stream) {
+  static bool configured[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(attention_cc_kernel<BITS, D, THREADS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kCcMaxSmem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int P = attn_keys(p);
+  const size_t smem = static_cast<size_t>(cc_layout(p.n_q, P, D).floats) * 4;
+  attention_cc_kernel<BITS, D, THREADS><<<p.B * p.H, THREADS, smem, stream>>>(p, P);
+  return cudaGetLastError();
+}
+
 }  // namespace
 }  // namespace vq
 
 #include "attention_pipe.cuh"
 
 namespace vq {
-namespace {
-
-// Blocks with at least this many queries run on the tensor cores; smaller ones
-// (mostly padding in a 128-row MMA tile) on the CUDA-core kernel.
-constexpr int kTcMinQueries = 16;
-
-}  // namespace
 
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
-  if (p.n_q >= kTcMinQueries) {
-    // more than 128 queries: two query tiles per work item sharing every
-    // dequantized K/V tile; otherwise one query tile per item, the two
-    // softmax warpgroups taking the items in turn
-    const bool pair = p.n_q > 128;
-    if (p.bits == 4 && p.D == 64)
-      return pair ? launch_attention_pipe<4, 64, 2, false>(p, stream) : launch_attention_pipe<4, 64, 2, true>(p, stream);
-    if (p.bits == 4 && p.D == 128)
-      return pair ? launch_attention_pipe<4, 128, 2, false>(p, stream) : launch_attention_pipe<4, 128, 2, true>(p, stream);
-    if (p.bits == 3 && p.D == 64)
-      return pair ? launch_attention_pipe<3, 64, 2, false>(p, stream) : launch_attention_pipe<3, 64, 2, true>(p, stream);
-    if (p.bits == 3 && p.D == 128)
-      return pair ? launch_attention_pipe<3, 128, 2, false>(p, stream) : launch_attention_pipe<3, 128, 2, true>(p, stream);
+  // few queries over few keys: the CUDA-core kernel (a 128-row MMA tile would
+  // be mostly padding); otherwise the tensor cores. More than 128 queries: two
+  // query tiles per work item sharing every dequantized K/V tile; otherwise one
+  // query tile per item, the two softmax warpgroups taking the items in turn
+  if (p.n_q <= kSmallMaxQueries) {
+    if (p.bits == 4 && p.D == 64) return launch_attention_small<4, 64>(p, stream);
+    if (p.bits == 4 && p.D == 128) return launch_attention_small<4, 128>(p, stream);
+    if (p.bits == 3 && p.D == 64) return launch_attention_small<3, 64>(p, stream);
+    if (p.bits == 3 && p.D == 128) return launch_attention_small<3, 128>(p, stream);
+    return cudaErrorInvalidValue;
   }
-  if (p.bits == 4 && p.D == 64) return launch_attention_small<4, 64>(p, stream);
-  if (p.bits == 4 && p.D == 128) return launch_attention_small<4, 128>(p, stream);
-  if (p.bits == 3 && p.D == 64) return launch_attention_small<3, 64>(p, stream);
-  if (p.bits == 3 && p.D == 128) return launch_attention_small<3, 128>(p, stream);
+  if (cc_fits(p)) {
+    const bool wide = p.n_q > 16;
+    if (p.bits == 4 && p.D == 64) return wide ? launch_attention_cc<4, 64, 256>(p, stream) : launch_attention_cc<4, 64, 128>(p, stream);
+    if (p.bits == 4 && p.D == 128) return wide ? launch_attention_cc<4, 128, 256>(p, stream) : launch_attention_cc<4, 128, 128>(p, stream);
+    if (p.bits == 3 && p.D == 64) return wide ? launch_attention_cc<3, 64, 256>(p, stream) : launch_attention_cc<3, 64, 128>(p, stream);
+    if (p.bits == 3 && p.D == 128) return wide ? launch_attention_cc<3, 128, 256>(p, stream) : launch_attention_cc<3, 128, 128>(p, stream);
+    return cudaErrorInvalidValue;
+  }
+  const bool pair = p.n_q > 128;
+  if (p.bits == 4 && p.D == 64)
+    return pair ? launch_attention_pipe<4, 64, 2, false>(p, stream) : launch_attention_pipe<4, 64, 2, true>(p, stream);
+  if (p.bits == 4 && p.D == 128)
+    return pair ? launch_attention_pipe<4, 128, 2, false>(p, stream) : launch_attention_pipe<4, 128, 2, true>(p, stream);
+  if (p.bits == 3 && p.D == 64)
+    return pair ? launch_attention_pipe<3, 64, 2, false>(p, stream) : launch_attention_pipe<3, 64, 2, true>(p, stream);
+  if (p.bits == 3 && p.D == 128)
+    return pair ? launch_attention_pipe<3, 128, 2, false>(p, stream) : launch_attention_pipe<3, 128, 2, true>(p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -398,3 +398,69 @@ def test_barrier_simulation_finds_a_planted_hazard():
         if case["T"] == 1:
             bad += bool(simulate(seed=0, hazard=True, **case))
     assert bad > 0
+
+
+# ------------------------------------------------------------------ CUDA-core kernel (attention.cuh)
+CC_MAX_SMEM, CC_MAX_QUERIES, SMALL_MAX_QUERIES = 76 * 1024, 64, 4
+
+
+def cc_layout(n_q, P, D):
+    PP, NQP = (P + 31) & ~31, (n_q + 7) & ~7
+    KS = PP + 1
+    kt = 0
+    vs = (kt + D * KS + 3) & ~3
+    qs = vs + PP * D
+    ps = qs + NQP * D
+    linv = ps + NQP * PP
+    return dict(PP=PP, NQP=NQP, KS=KS, kt=kt, vs=vs, qs=qs, ps=ps, linv=linv, floats=linv + NQP)
+
+
+def dispatch(n_q, P, D):
+    if n_q <= SMALL_MAX_QUERIES:
+        return "small"
+    if n_q <= CC_MAX_QUERIES and cc_layout(n_q, P, D)["floats"] * 4 <= CC_MAX_SMEM:
+        return "cc"
+    return "pipe"
+
+
+def check_cc_block(sched, s, D, bits):
+    CPW = 32 // bits
+    n_q, P = sched[s], sum(sched[: s + 1])
+    L = cc_layout(n_q, P, D)
+    PP, NQP, KS = L["PP"], L["NQP"], L["KS"]
+    assert L["vs"] % 4 == 0 and L["qs"] % 4 == 0 and L["ps"] % 4 == 0  # float4 rows stay 16-byte aligned
+    kt_end, vs_end = L["kt"] + (D - 1) * KS + PP, L["vs"] + PP * D
+    assert kt_end <= L["vs"] and vs_end <= L["qs"]
+    assert L["qs"] + NQP * D <= L["ps"] and L["ps"] + NQP * PP <= L["linv"]
+    # dequantize: every (block, word row, channel) item lands on keys < P, each key once
+    keys, key = set(), 0
+    for kb in range(s + 1):
+        for w in range(-(-sched[kb] // CPW)):
+            ns = min(CPW, sched[kb] - w * CPW)
+            assert ns >= 1
+            for i in range(ns):
+                j = key + w * CPW + i
+                assert j < P and j not in keys
+                keys.add(j)
+        key += sched[kb]
+    assert keys == set(range(P))
+    # bank pattern of the dequantize stores: a warp's 32 consecutive channels of one key
+    assert len({(c * KS + 5) % 32 for c in range(32)}) == 32
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_cc_kernel_layout_and_dispatch(D):
+    rng = random.Random(D)
+    scheds = [VAR_BLOCKS, INFINITY_BLOCKS, [1, 2, 7, 11, 81, 300, 1100, 4095], [300, 200, 5, 3]]
+    scheds += [[rng.randint(1, 70) for _ in range(rng.randint(1, 10))] for _ in range(100)]
+    for sched in scheds:
+        for s in range(len(sched)):
+            if dispatch(sched[s], sum(sched[: s + 1]), D) == "cc":
+                for bits in (3, 4):
+                    check_cc_block(sched, s, D, bits)
+    # the VAR schedule at head_dim 64: blocks 0-1 warp per query, 2-5 CUDA-core, 6-9 tensor cores
+    if D == 64:
+        got = [dispatch(n, sum(VAR_BLOCKS[: s + 1]), 64) for s, n in enumerate(VAR_BLOCKS)]
+        assert got == ["small"] * 2 + ["cc"] * 4 + ["pipe"] * 4
+    # few queries over many keys fall through to the tensor cores
+    assert dispatch(5, 505, D) == "pipe"

@@ -193,8 +193,24 @@ def test_ragged_blocks_all_bit_widths(vq, D):
             _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D)
 
 
-def _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D):
-    B, H = 1, 3
+@pytest.mark.parametrize("D", [64, 128])
+def test_few_queries_over_many_keys(vq, D):
+    """Blocks of 5 and 3 queries after 500 cached tokens: too many keys for the
+    CUDA-core kernel's shared memory, so they run on the tensor-core kernel
+    with mostly empty query tiles."""
+    sched = [300, 200, 5, 3]
+    k, v, q = _ragged_kv(sched, D, H=2, B=2, seed=11)
+    for bits in (3, 4):
+        desc = vq.CacheDesc(2, 2, D, bits, sched)
+        cache = vq.LayerCache(desc)
+        p0 = 0
+        for s, n in enumerate(sched):
+            vq.vq_cache_append(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+            p0 += n
+        _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D, B=2, H=2)
+
+
+def _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D, B=1, H=3):
     sigma = 1.0 / np.sqrt(D)
     ok_, sk, zk = vo.cache_append(_host(k), sched, bits)
     ov_, sv, zv = vo.cache_append(_host(v), sched, bits)
