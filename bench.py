@@ -48,8 +48,8 @@ def load_peaks():
 # (profiles/dram_traffic.json); valid only while the kernels' sources are the
 # ones that capture ran.
 KERNEL_SOURCES = {
-    "attention": ("attention.cuh", "attention_pipe.cuh", "tc_ptx.cuh", "vq_device.cuh"),
-    "quant_pack": ("quant_pack.cuh", "vq_device.cuh"),
+    "attention": ("attention.cuh", "attention_pipe.cuh", "tc_ptx.cuh", "vq_device.cuh", "vq_api.cu"),
+    "quant_pack": ("quant_pack.cuh", "vq_device.cuh", "vq_api.cu"),
 }
 
 

@@ -89,18 +89,21 @@ vq_status check_strides(const int64_t st[3], int esize, const char* name) {
   return VQ_OK;
 }
 
-// Choose units per CTA (G), CTAs per unit (cluster size C) and word-rows per CTA
-// for one quantize launch. Returns false if one slab is too large.
+// Choose the warps per unit (P, enough units x warps to fill the GPU) and,
+// with one warp per unit, the lanes per unit (TL): the fewest rows per team
+// load that still cover the unit's rows in one batch of loads, so that small
+// blocks put several units in flight per warp. Returns false if one slab is
+// too large.
 bool plan_quant(vq::QuantParams& p) {
   constexpr int64_t kTargetWarps = 2048;
+  constexpr int kBatch = 16;  // loads in flight per lane in pass 1 (kQuantUnroll)
   int P = 1;
   while (P < vq::quant_warps() && int64_t(p.units) * P < kTargetWarps && 2 * P <= p.W) P *= 2;
   p.P = P;
   p.WP = (p.W + P - 1) / P;
-  // tiny blocks: a warp takes several units, each on vecs_per_row * rows lanes
-  int rows = 1;
-  while (rows * p.vecs_per_row < 32 && rows < p.n) rows *= 2;
-  p.TL = (P == 1) ? rows * p.vecs_per_row : 32;
+  int rw = 1;
+  while (rw * kBatch < p.n && rw * p.vecs_per_row < 32) rw *= 2;
+  p.TL = (P == 1) ? rw * p.vecs_per_row : 32;
   if (p.TL > 32) p.TL = 32;
   return true;
 }

@@ -1,0 +1,76 @@
+"""CPU model of the quantize+pack kernel's work split (csrc/quant_pack.cuh with
+the plan of csrc/vq_api.cu), no GPU: for block sizes, bit widths, row widths
+and unit counts of the workloads, every (unit, row, 16-byte vector) is read
+exactly once in pass 1, every (unit, word row, vector) is encoded exactly once
+in pass 2, and every (unit, vector) of scale/zero is written exactly once."""
+import itertools
+
+import pytest
+
+WARPS, BATCH, TARGET_WARPS = 16, 16, 2048
+
+
+def plan(units, W, n, V):
+    P = 1
+    while P < WARPS and units * P < TARGET_WARPS and 2 * P <= W:
+        P *= 2
+    rw = 1
+    while rw * BATCH < n and rw * V < 32:
+        rw *= 2
+    TL = min(32, rw * V) if P == 1 else 32
+    return P, -(-W // P), TL
+
+
+def check(n, bits, V, units, grid):
+    CPW = 32 // bits
+    W = -(-n // CPW)
+    P, WP, TL = plan(units, W, n, V)
+    assert 32 % TL == 0 and TL % V == 0
+    gpc, RW, upw = WARPS // P, TL // V, 32 // TL
+    seen1, seen2, meta = set(), set(), set()
+    for cta, warp in itertools.product(range(grid), range(WARPS)):
+        grp, part = divmod(warp, P)
+        u0 = (cta * gpc + grp) * upw
+        while u0 < units:
+            for lane in range(32):
+                team, tl = divmod(lane, TL)
+                j, rsub = tl % V, tl // V
+                unit = u0 + team
+                live = unit < units
+                w0 = part * WP
+                w1 = min(W, w0 + WP) if live else w0
+                r0, r1 = w0 * CPW, min(n, w1 * CPW)
+                r = r0 + rsub
+                while r < r1:
+                    for u in range(BATCH):
+                        if r + u * RW < r1:  # the clamped repeats re-read row r1 - 1
+                            k = (unit, r + u * RW, j)
+                            assert k not in seen1
+                            seen1.add(k)
+                    r += BATCH * RW
+                if live and part == 0 and rsub == 0:
+                    assert (unit, j) not in meta
+                    meta.add((unit, j))
+                w = w0 + rsub
+                while w < w1:
+                    assert (unit, w, j) not in seen2
+                    seen2.add((unit, w, j))
+                    w += RW
+            u0 += grid * gpc * upw
+    assert len(seen1) == units * n * V
+    assert len(seen2) == units * W * V
+    assert len(meta) == units * V
+
+
+@pytest.mark.parametrize("n", [1, 2, 4, 9, 16, 17, 25, 36, 64, 100, 256])
+def test_quant_work_split_covers_every_vector_once(n):
+    for bits, V, units, grid in itertools.product((2, 3, 4, 8), (8, 16, 32), (3, 256, 1000), (1, 148)):
+        if units * n <= 16000:
+            check(n, bits, V, units, grid)
+
+
+def test_quant_plan_small_blocks_share_warps():
+    # VAR-d30 shapes (bf16, head_dim 64: 8 vectors per row; 7680 units): blocks of up to
+    # 16 tokens take 4 units per warp, 25 tokens 2, larger blocks a whole warp
+    tl = {n: plan(7680, -(-n // 10), n, 8)[2] for n in (1, 4, 9, 16, 25, 36, 64, 256)}
+    assert tl == {1: 8, 4: 8, 9: 8, 16: 8, 25: 16, 36: 32, 64: 32, 256: 32}
