@@ -324,20 +324,22 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       const uint64_t qdesc = tc::sw128_desc(sbase + C::Q0);
       const uint64_t kdesc0 = tc::sw128_desc(sbase + C::KV0);
       const uint64_t vdesc0 = tc::sw128_desc_mn(sbase + C::KV0 + 2 * C::TILE_SZ, kLbo);
+      // The issue loops stay rolled, to keep this warp's code small: with the
+      // sequences unrolled, consecutive MMAs issued 100-190 cycles apart in the
+      // kernel (about 50 when replayed alone), the pattern of instruction-cache
+      // misses on code that no other warp shares.
       auto issue_qk = [&](int qt, int slot, int kvs, int nk16) {
         const uint32_t idesc = tc::idesc_f16_f32(128, nk16);
         const uint64_t qd = qdesc + static_cast<uint64_t>((qt * C::Q_SZ) >> 4);
         const uint64_t kd = kdesc0 + static_cast<uint64_t>((kvs * C::KV_SZ) >> 4);
         const uint32_t d = tmem + qt * C::TM_QT + slot * KT;
-#pragma unroll
+        constexpr int kSlabA = 128 * 128, kSlabB = KT * 128;
+#pragma unroll 1
         for (int kk = 0; kk < D / 16; ++kk) {
-#pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            constexpr int kSlabA = 128 * 128, kSlabB = KT * 128;
-            const uint32_t aoff = ((kk >> 2) * kSlabA + (kk & 3) * 32) >> 4;
-            const uint32_t boff = (part * C::TILE_SZ + (kk >> 2) * kSlabB + (kk & 3) * 32) >> 4;
-            tc::mma_f16_ss(d, qd + aoff, kd + boff, idesc, (part == 0 && kk == 0) ? 0u : 1u);
-          }
+          const uint64_t a = qd + static_cast<uint64_t>(((kk >> 2) * kSlabA + (kk & 3) * 32) >> 4);
+          const uint64_t b = kd + static_cast<uint64_t>(((kk >> 2) * kSlabB + (kk & 3) * 32) >> 4);
+          tc::mma_f16_ss(d, a, b, idesc, kk > 0 ? 1u : 0u);                         // q . K^hi
+          tc::mma_f16_ss(d, a, b + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc, 1u);  // q . K^lo
         }
         tc::commit(s_full(qt, slot));
       };
@@ -346,17 +348,14 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         const uint32_t pa = tmem + qt * C::TM_QT + slot * KT;
         const uint32_t o = tmem + qt * C::TM_QT + C::COL_O;
         const int nkk = nk16 / 16;
-        // (A part, B part): (P hi, V hi), (P lo, V hi), (P hi, V lo)
-#pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk) {
-#pragma unroll
-          for (int part = 0; part < 3; ++part) {
-            const uint32_t acol = (part == 1) ? 8u : 0u;
-            const uint32_t vpart = (part == 2) ? (C::TILE_SZ >> 4) : 0u;
-            if (kk < nkk)
-              tc::mma_f16_ts(o, pa + 16 * kk + acol, vd + vpart + ((kk * 2048) >> 4), idesc_pv,
-                                (first && part == 0 && kk == 0) ? 0u : 1u);
-          }
+        // per 16-key step: (P hi, V hi), (P lo, V hi), (P hi, V lo); P lo sits 8 columns after P hi
+#pragma unroll 1
+        for (int kk = 0; kk < nkk; ++kk) {
+          const uint64_t v = vd + static_cast<uint64_t>((kk * 2048) >> 4);
+          const uint32_t a = pa + 16 * kk;
+          tc::mma_f16_ts(o, a, v, idesc_pv, (first && kk == 0) ? 0u : 1u);
+          tc::mma_f16_ts(o, a + 8, v, idesc_pv, 1u);
+          tc::mma_f16_ts(o, a, v + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc_pv, 1u);
         }
         tc::commit(pv_done(qt, slot));
       };
