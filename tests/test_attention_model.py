@@ -33,7 +33,7 @@ def pipe_cfg(BITS, D, NQT):
     TM_QT = 512 // NQT
     c["NS"] = NS = 4 if NQT == 1 else (3 if D == 64 else 2)
     c["NKV"] = NKV = (4 if NQT == 1 else 3) if D == 64 else (3 if NQT == 1 else 2)
-    NSTG = 2
+    c["NSTG"] = NSTG = 3 if D == 64 else 2
     c["SPLIT"] = NKV <= 2
     STAGE_Q = D == 64
     QPF = 2 if (STAGE_Q and NQT == 1) else 1
@@ -378,7 +378,7 @@ def protocol_cases(D, ALT):
                 for bh in (1, 4, 9):
                     if cta < bh * n_groups:
                         yield dict(NQT=2, NS=c["NS"], NKV=c["NKV"], T=T, n_items=bh * n_groups, grid=grid,
-                                   n_qt=n_qt, cta=cta, ALT=ALT, SPLIT=c["SPLIT"])
+                                   n_qt=n_qt, cta=cta, ALT=ALT, SPLIT=c["SPLIT"], NSTG=c["NSTG"])
 
 
 @pytest.mark.parametrize("D,ALT", [(64, True), (64, False), (128, True), (128, False)])
