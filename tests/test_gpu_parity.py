@@ -154,7 +154,7 @@ def _ragged_kv(sched, D, H=3, B=1, dtype=torch.bfloat16, seed=5):
 
 @pytest.mark.parametrize("D", [64, 128])
 def test_ragged_blocks_all_bit_widths(vq, D):
-    """Odd block sizes (1, INT3 word-row tails, cluster-split blocks) for bits 2/3/4/8;
+    """Odd block sizes (1, INT3 word-row tails, slabs split across warp groups) for bits 2/3/4/8;
     dequantize is bit-exact too."""
     sched = [1, 2, 7, 11, 81, 300, 1100, 4095]
     k, v, q = _ragged_kv(sched, D)
