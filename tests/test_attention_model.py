@@ -464,3 +464,55 @@ def test_cc_kernel_layout_and_dispatch(D):
         assert got == ["small"] * 2 + ["cc"] * 4 + ["pipe"] * 4
     # few queries over many keys fall through to the tensor cores
     assert dispatch(5, 505, D) == "pipe"
+
+
+# ------------------------------------------------------------------ work items -> query rows
+def pipe_rows_written(n_q, BH, grid):
+    """(bh, row) -> count of softmax threads that write it, for the launch mode
+    the dispatch picks: two query tiles per item above 128 queries, otherwise
+    one tile per item with the two warpgroups taking the CTA's items in turn."""
+    ALT = n_q <= 128
+    n_qt = -(-n_q // 128)
+    n_groups = n_qt if ALT else -(-n_qt // 2)
+    n_items = BH * n_groups
+
+    def item_nqt(item):
+        return 1 if ALT else min(2, n_qt - (item % n_groups) * 2)
+
+    written = {}
+    mma_tiles = {}
+    for cta in range(min(grid, n_items)):
+        # the MMA thread: k-th item of the CTA covers query tiles [qlo, qhi)
+        for k, item in enumerate(range(cta, n_items, grid)):
+            qlo, qhi = (k & 1, (k & 1) + 1) if ALT else (0, item_nqt(item))
+            for qt in range(qlo, qhi):
+                mma_tiles[(item, qt)] = mma_tiles.get((item, qt), 0) + 1
+        for qt in range(2):
+            roff = 128 - n_q if (ALT and qt == 1) else 0
+            item = cta + (qt * grid if ALT else 0)
+            if not ALT and item < n_items and item_nqt(item) <= qt:
+                item += grid
+                while item < n_items and item_nqt(item) <= qt:
+                    item += grid
+            while item < n_items:
+                assert mma_tiles.get((item, qt)) == 1, (item, qt)  # the MMA thread serves this tile
+                for row in range(128):
+                    r = row - roff if ALT else (item % n_groups) * 256 + qt * 128 + row
+                    if 0 <= r < n_q:
+                        key = (item // n_groups, r)
+                        written[key] = written.get(key, 0) + 1
+                if ALT:
+                    item += 2 * grid
+                else:
+                    item += grid
+                    while item < n_items and item_nqt(item) <= qt:
+                        item += grid
+    return written
+
+
+@pytest.mark.parametrize("n_q", [5, 16, 64, 100, 128, 129, 169, 256, 300, 576, 1024])
+def test_every_query_row_is_written_once(n_q):
+    for BH, grid in ((1, 1), (3, 2), (7, 148), (40, 148), (300, 148)):
+        w = pipe_rows_written(n_q, BH, grid)
+        assert set(w) == {(bh, r) for bh in range(BH) for r in range(n_q)}
+        assert set(w.values()) == {1}
