@@ -134,8 +134,11 @@ vq_status vq_cache_append(const vq_cache_desc* desc, const vq_layer_cache* cache
  *   out: device, same indexing with out_strides, dtype `out_dtype` (VQ_F32
  *        gives the accuracy the tests check; VQ_BF16 rounds the float32 result);
  *   softmax_scale: the logit multiplier, usually 1/sqrt(head_dim).
- * Arithmetic: logits and softmax in float32 with the quantization scales
- * folded into the queries; see the kernel source for the operand precision. */
+ * Arithmetic: float32 accumulation of logits, softmax and output over the
+ * cache's dequantized values (on the tensor cores as exact-sum fp16 hi/lo
+ * operand pairs); the result is within 2e-3 x output RMS of float64 attention
+ * over the same dequantized cache. See the kernel sources for the operand
+ * precision of each kernel. */
 vq_status vq_attention_block(const vq_cache_desc* desc, const vq_layer_cache* cache,
                              int32_t block, const void* q, const int64_t q_strides[3],
                              float softmax_scale, void* out, vq_dtype out_dtype,
