@@ -100,6 +100,18 @@ def attn_work(w, bits, s):
     return flops, byts
 
 
+def workload_config(w, bits):
+    """The `config` of both arms' JSON lines: the workload and what the timed
+    region reads (inputs larger than L2, so no flush between steps)."""
+    esize = 4 if w.kv_dtype == "f32" else 2
+    inputs = w.layers * w.batch * w.heads * w.tokens * w.head_dim * (2 * esize + 2)
+    return {"workload": w.name, "bits": bits, "layers": w.layers, "heads": w.heads, "head_dim": w.head_dim,
+            "batch": w.batch, "blocks": w.num_blocks, "tokens": w.tokens, "kv_dtype": w.kv_dtype,
+            "per_rank": "one full decode per step",
+            "l2": f"inputs {inputs / 1e9:.1f} GB > L2 (126 MB), no flush",
+            "token_unit": "B*N*L query tokens x layers per step (append + attention)"}
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -215,6 +227,14 @@ def oracle_unit(w, bits, layer_kv, q, b, h, sigma):
     return time.perf_counter() - t0
 
 
+def host_cores():
+    """CPU cores this process may run on (the host's core count)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -283,11 +303,12 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_unit * args.ref_units * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "bits": bits, "layers": w.layers, "heads": w.heads, "head_dim": w.head_dim,
-                   "batch": w.batch, "blocks": w.num_blocks, "tokens": w.tokens},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+        "config": workload_config(w, bits),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                         "blas_threads": blas_threads(), "quantize_threads": 1,
                          "sample": f"each step: {args.ref_units} (batch, head) units of layer 0 through the oracle (append of all "
-                                   "blocks of K and V + every block's float64 attention), scaled by B*H*L units"},
+                                   "blocks of K and V + every block's float64 attention), scaled by B*H*L units; the "
+                                   "quantize steps run single-threaded numpy, the attention matmuls on the BLAS threads"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -295,20 +316,23 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args):
-    from bit_kv_cache_25_b200 import vq
+def roofline_entry(kernel, bound, achieved, peak, unit, algorithmic, traffic, tnote, peak_note, extra=None):
+    r = {"kernel": kernel, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+         "frac": achieved / peak, "traffic": traffic, "algorithmic": algorithmic,
+         "traffic_unit": "DRAM bytes read + written per step (all launches of the kernel family in one decode)",
+         "traffic_source": tnote, "peak_source": peak_note}
+    if extra:
+        r.update(extra)
+    return r
 
-    world, rank, local = dist_setup(args.gpus)
-    dev = torch.device("cuda", torch.cuda.current_device())
-    w = WORKLOADS[args.workload]
-    if args.layers:
-        import dataclasses
-        w = dataclasses.replace(w, layers=args.layers)   # smaller case for profiler captures
-    bits = args.bits or w.bits[0]
+
+def measure(args, vq, w, bits, world, seed, dev):
+    """One workload: inputs resident in HBM, the whole decode captured as a CUDA
+    graph and timed over args.steps replays (barrier + synchronize on both
+    sides, max over ranks), then each kernel family of each block replayed
+    alone for the per-kernel numbers. Returns the JSON fields of this workload."""
     L, S, B, H, D, N = w.layers, w.num_blocks, w.batch, w.heads, w.head_dim, w.tokens
     sigma = default_softmax_scale(w)
-    seed = 1000003 * rank
-
     desc = vq.CacheDesc(B, H, D, bits, w.block_tokens)
     ks, vs, qs, caches = [], [], [], []
     for layer in range(L):
@@ -320,7 +344,6 @@ def run_ours(args):
     nmax = max(w.block_tokens)
     out = torch.empty((B, H, nmax, D), dtype=torch.float32, device=dev)
     outs = [out[:, :, :n] for n in w.block_tokens]
-    stream = torch.cuda.current_stream()
 
     def enqueue(blocks, layers, do_quant=True, do_attn=True):
         for s in blocks:
@@ -397,67 +420,101 @@ def run_ours(args):
                              "attn_gbs": round(ab * L / (ta / 1e3) / 1e9, 1),
                              "attn_tflops": round(af * L / (ta / 1e3) / 1e12, 2)})
     barrier(world)
-    elapsed_ms = start.elapsed_time(stop)
-    elapsed_ms = max_over_ranks(elapsed_ms, world)
-    t_quant *= args.steps
-    t_attn *= args.steps
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world)
     assert vq.vq_poll_device_error() == 0
-    clocks = clk.summary()
-    n_launch = 2 * L * S
     ms_step = elapsed_ms / args.steps
     tokens_step = B * N * L
-    value = weak_scaling_value(tokens_step, world, ms_step)
     peaks, peak_src = load_peaks()
-    hbm = peaks["hbm_gbs"]
-    tc = peaks["bf16_tflops_sustained"]
-    q_ms = t_quant / args.steps
-    a_ms = t_attn / args.steps
+    hbm, tc_burst, tc_sus = peaks["hbm_gbs"], peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+    peak_note = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+    q_ms, a_ms = t_quant, t_attn
     q_gbs = q_bytes / (q_ms / 1e3) / 1e9
     a_gbs = a_bytes / (a_ms / 1e3) / 1e9
     a_tflops = a_flops / (a_ms / 1e3) / 1e12
-    a_bound = "hbm" if a_bytes / (hbm * 1e9) >= a_flops / (tc * 1e12) else "tensor"
-    a_frac = (a_gbs / hbm) if a_bound == "hbm" else (a_tflops / tc)
-    if a_ms >= q_ms:
-        traffic, tnote = measured_traffic(w.name, "attention", L)
-        roof = {"kernel": "attention", "bound": a_bound, "achieved": a_gbs if a_bound == "hbm" else a_tflops,
-                "peak": hbm if a_bound == "hbm" else tc, "unit": "GB/s" if a_bound == "hbm" else "TFLOP/s",
-                "frac": a_frac, "traffic": traffic, "algorithmic_bytes": a_bytes}
+    # the attention's bound: the larger of its HBM time and its tensor time at the burst peak
+    a_bound = "hbm" if a_bytes / (hbm * 1e9) >= a_flops / (tc_burst * 1e12) else "tensor"
+    if a_bound == "hbm":
+        a_frac = {"frac": a_gbs / hbm}
     else:
-        traffic, tnote = measured_traffic(w.name, "quant_pack", L)
-        roof = {"kernel": "quant_pack", "bound": "hbm", "achieved": q_gbs, "peak": hbm, "unit": "GB/s",
-                "frac": q_gbs / hbm, "traffic": traffic, "algorithmic_bytes": q_bytes}
-    roof["traffic_unit"] = "DRAM bytes read + written per step (all launches of the kernel family in one decode)"
-    roof["traffic_source"] = tnote
-    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name, "bits": bits, "layers": L, "heads": H, "head_dim": D, "batch": B,
-                   "blocks": S, "tokens": N, "kv_dtype": w.kv_dtype, "per_rank": "one full decode per step",
-                   "l2": f"inputs {sum(t.numel() * t.element_size() for t in ks + vs + qs) / 1e9:.1f} GB > L2, no flush",
-                   "token_unit": "B*N*L query tokens x layers per step (append + attention)"},
-        "quant_pack": {"ms_per_step": q_ms, "gbs": q_gbs, "frac_hbm": q_gbs / hbm,
-                       "bytes_per_step": q_bytes},
+        a_frac = {"frac": a_tflops / tc_burst, "frac_vs_sustained": a_tflops / tc_sus}
+    rooflines = {}
+    traffic, tnote = measured_traffic(w.name, "attention", L)
+    if a_bound == "hbm":
+        rooflines["attention"] = roofline_entry("attention", "hbm", a_gbs, hbm, "GB/s", a_bytes, traffic, tnote,
+                                                peak_note)
+    else:
+        rooflines["attention"] = roofline_entry(
+            "attention", "tensor", a_tflops, tc_burst, "TFLOP/s", a_flops, traffic, tnote,
+            peak_note + "; bf16 burst peak", {"peak_sustained": tc_sus, "frac_vs_sustained": a_tflops / tc_sus})
+    traffic, tnote = measured_traffic(w.name, "quant_pack", L)
+    rooflines["quant_pack"] = roofline_entry("quant_pack", "hbm", q_gbs, hbm, "GB/s", q_bytes, traffic, tnote,
+                                             peak_note)
+    dominant = "attention" if a_ms >= q_ms else "quant_pack"
+    res = {
+        "workload": w.name, "bits": bits, "ms_per_step": ms_step,
+        "value": weak_scaling_value(tokens_step, world, ms_step), "unit": "tokens/s",
+        "config": workload_config(w, bits),
+        "quant_pack": {"ms_per_step": q_ms, "gbs": q_gbs, "frac_hbm": q_gbs / hbm, "bytes_per_step": q_bytes},
         "attention": {"ms_per_step": a_ms, "tokens_per_s": tokens_step / (a_ms / 1e3), "gbs": a_gbs,
-                      "tflops": a_tflops, "bound": a_bound, "frac_roofline": a_frac,
+                      "tflops": a_tflops, "bound": a_bound, "frac_roofline": a_frac["frac"],
+                      **({"frac_vs_sustained": a_frac["frac_vs_sustained"]} if "frac_vs_sustained" in a_frac else {}),
                       "flops_per_step": a_flops, "bytes_per_step": a_bytes},
-        "roofline": roof,
-        "clocks": clocks,
-        "gpu_launches": n_launch * args.steps,
-        "timing": "step = one CUDA-graph replay of the whole decode; per-kernel times from graphs of each kernel "
-                  "family per block, replayed alone",
+        "roofline": rooflines[dominant],
+        "roofline_other": rooflines["quant_pack" if dominant == "attention" else "attention"],
+        "clocks": clk.summary(),
+        "gpu_launches": 2 * L * S * args.steps,
         "by_block": by_block,
     }
-    if not args.no_e2e:
-        line["e2e"] = run_e2e(args, vq, w, bits, desc, caches, outs, dev, world)
+    if args.e2e and w.name == args.workload:
+        res["e2e"] = run_e2e(args, vq, w, bits, desc, caches, outs, dev, world)
+    del graphs, ks, vs, qs, caches, out, outs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args):
+    from bit_kv_cache_25_b200 import vq
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    import dataclasses
+    names = [args.workload] + [x for x in args.also.split(",") if x and x != "none" and x != args.workload]
+    results = []
+    for name in names:
+        w = WORKLOADS[name]
+        if args.layers:
+            w = dataclasses.replace(w, layers=args.layers)   # smaller case for profiler captures
+        bits = (args.bits or w.bits[0]) if name == args.workload else w.bits[0]
+        results.append(measure(args, vq, w, bits, world, 1000003 * rank, dev))
+    head = results[0]
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": head["config"],
+        "quant_pack": head["quant_pack"], "attention": head["attention"], "roofline": head["roofline"],
+        "roofline_other": head["roofline_other"], "clocks": head["clocks"],
+        "gpu_launches": sum(r["gpu_launches"] for r in results),
+        "timing": "step = one CUDA-graph replay of the whole decode; per-kernel times from graphs of each kernel "
+                  "family per block, replayed alone",
+        "by_block": head["by_block"],
+    }
+    if "e2e" in head:
+        line["e2e"] = head["e2e"]
+    for r in results[1:]:
+        line[r["workload"]] = {k: r[k] for k in ("bits", "ms_per_step", "value", "unit", "config", "quant_pack",
+                                                 "attention", "roofline", "roofline_other", "clocks",
+                                                 "gpu_launches", "by_block")}
     if rank == 0 and not args.no_cpu:
+        w = WORKLOADS[args.workload]
+        bits = args.bits or w.bits[0]
         tps, units, secs = cpu_sample(w, bits, budget_s=args.cpu_budget)
-        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"{units} (batch, head) units of layer 0 through the oracle (append of all "
-                                          f"blocks + float64 attention of every block), {secs:.1f} s, scaled by "
-                                          f"B*H*L units per step"}
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                                "blas_threads": blas_threads(), "quantize_threads": 1,
+                                "sample": f"{units} (batch, head) units of layer 0 of {w.name} through the oracle "
+                                          f"(append of all blocks + float64 attention of every block), {secs:.1f} s, "
+                                          f"scaled by B*H*L units per step; the quantize steps run single-threaded "
+                                          f"numpy, the attention matmuls on the BLAS threads"}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
@@ -519,7 +576,9 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="var_d30", choices=sorted(WORKLOADS))
     ap.add_argument("--bits", type=int, default=0)
-    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--also", default="infinity_2b",
+                    help="comma-separated workloads measured after the headline one ('none' to skip)")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

@@ -12,7 +12,7 @@
 //
 // This file holds the two CUDA-core kernels and the dispatch between them and
 // the tensor-core kernel (attention_pipe.cuh), by measured speed on the VAR
-// and Infinity shapes: at most 4 queries -> attention_small_kernel; up to 32
+// and Infinity shapes: at most 4 queries -> attention_small_kernel; up to 64
 // queries whose keys fit in shared memory -> attention_cc_kernel; the rest ->
 // attention_pipe_kernel (a 128-row MMA tile is mostly padding below that).
 //
@@ -152,7 +152,9 @@ cudaError_t launch_attention_small(const AttnParams& p, cudaStream_t stream) {
 
 
 // ---- attention_cc_kernel
-constexpr int kCcMaxSmem = 76 * 1024;  // three CTAs per SM at most this
+// Largest shared-memory plan; two CTAs per SM at this size (a third would need
+// 3 x (76 + 1) KB, above the 228 KB of an SM), three at 74 KB or less.
+constexpr int kCcMaxSmem = 76 * 1024;
 constexpr int kCcMaxQueries = 64;
 
 // Shared-memory plan of one CTA (offsets in floats).

@@ -23,18 +23,19 @@
 //     named barrier of the group. Min/max is exact, so the order of reduction
 //     does not matter.
 //   * scale/inv: one IEEE division and one IEEE reciprocal per group (every
-//     lane computes its own channels' values).
+//     lane computes its own channels' values); for a scale below 2^-100 both
+//     d and scale are first multiplied by 2^64 (exact), so 1/scale never
+//     overflows and the codes stay the nearest grid levels.
 //   * pass 2: the warp re-reads its rows (now in L2), one word-row per lane and
 //     vector, all cpw row loads issued first: d = x - min and t = d * inv, each
-//     correctly rounded (no FMA contraction), then round half to even by adding
-//     1.5*2^23. The rounded value's low mantissa bits are the code
-//     (t <= 2^bits - 1 + tiny, so no clamp is needed). The codes are summed
+//     correctly rounded, t clamped to 2^bits - 1 (a subnormal scale can put
+//     the max past the top level), then round half to even by adding 1.5*2^23.
+//     The rounded value's low mantissa bits are the code. The codes are summed
 //     into the word with shifts and a final constant correction, then stored
 //     with 128-bit coalesced stores.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include <cfloat>
 #include <cstdint>
 
 #include "vq_device.cuh"
@@ -117,6 +118,7 @@ template <class Vec, int BITS>
 __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __grid_constant__ QuantParams p) {
   constexpr int CPW = 32 / BITS;
   constexpr int CH = Vec::kCh;
+  constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
   extern __shared__ __align__(16) float qred[];  // [2][groups][P][2][D]
   const int D = p.D;
   const int V = p.vecs_per_row;
@@ -193,12 +195,19 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
         }
       }
     }
-    float scl[CH], zer[CH], inv[CH];
+    // pre = 2^64 for a scale below 2^-100 (1/scale would overflow from 2^-128
+    // down): d and scale are both multiplied by it, exactly, so the encode
+    // behaves as float32 with an unbounded exponent. d = fma(x, pre, -min*pre)
+    // = RN(x - min) * pre bit for bit (one rounding of an exactly scaled
+    // difference; a difference below 2^-126 is exact).
+    float scl[CH], zer[CH], inv[CH], pre[CH], nmp[CH];
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-      scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), static_cast<float>((1 << BITS) - 1));
+      scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), kLevels);
       zer[c] = __fadd_rn(fmn[c], 0.0f);
-      inv[c] = (scl[c] > 0.0f) ? fminf(__frcp_rn(scl[c]), FLT_MAX) : 0.0f;
+      pre[c] = (scl[c] > 0.0f && scl[c] < 0x1p-100f) ? 0x1p64f : 1.0f;
+      inv[c] = (scl[c] > 0.0f) ? __frcp_rn(__fmul_rn(scl[c], pre[c])) : 0.0f;
+      nmp[c] = __fmul_rn(-fmn[c], pre[c]);
     }
     if (live && part == 0 && rsub == 0) {
       float* sd = T.scale + static_cast<size_t>(bh) * D + CH * j;
@@ -226,8 +235,8 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
           corr += kRoundMagicBits << (BITS * i);
 #pragma unroll
           for (int c = 0; c < CH; ++c) {
-            const float d = __fsub_rn(Vec::elem(v[i], c), fmn[c]);
-            const float t = __fmul_rn(d, inv[c]);
+            const float d = __fmaf_rn(Vec::elem(v[i], c), pre[c], nmp[c]);
+            const float t = fminf(__fmul_rn(d, inv[c]), kLevels);
             const float rq = __fadd_rn(t, kRoundMagic);
             acc[c] += __float_as_uint(rq) << (BITS * i);
           }

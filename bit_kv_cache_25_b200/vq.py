@@ -109,6 +109,60 @@ def _strides(t: torch.Tensor, ndim_expected: int = 4):
     return (ctypes.c_int64 * 3)(t.stride(0), t.stride(1), t.stride(2))
 
 
+def _block_tokens(desc: "CacheDesc", block: int) -> int:
+    if not 0 <= int(block) < desc.num_blocks:
+        raise ValueError(f"block {block} out of range [0, {desc.num_blocks})")
+    return desc.block_tokens[int(block)]
+
+
+def _check_slab(name: str, t: torch.Tensor, desc: "CacheDesc", n: int):
+    """t must be a [B][H][n][D] view of the block (any strides, channels contiguous)."""
+    want = (desc.batch, desc.heads, n, desc.head_dim)
+    if tuple(t.shape) != want:
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want} ([B][H][n_s][D] of this block)")
+
+
+def _check_flat(name: str, t: torch.Tensor, numel: int, dtypes):
+    """t is written or read as a flat array of at least numel elements from data_ptr()."""
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs at least {numel}")
+
+
+def _check_devices(*named):
+    """Every tensor on the same CUDA device (a host pointer would become an
+    out-of-bounds device access)."""
+    dev = None
+    for name, t in named:
+        if not t.is_cuda:
+            raise ValueError(f"{name} is on {t.device}, not a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other tensors on {dev}")
+
+
+_WORDS = (torch.int32, torch.uint32) if hasattr(torch, "uint32") else (torch.int32,)
+_F32 = (torch.float32,)
+
+
+def _check_cache(desc: "CacheDesc", cache: "LayerCache"):
+    words, meta, _ = vq_cache_layout(desc)
+    for name in ("packed_k", "packed_v"):
+        _check_flat(f"cache.{name}", getattr(cache, name), words, _WORDS)
+    for name in ("scale_k", "zero_k", "scale_v", "zero_v"):
+        _check_flat(f"cache.{name}", getattr(cache, name), meta, _F32)
+    ptrs = (cache.packed_k.data_ptr(), cache.packed_v.data_ptr(), cache.scale_k.data_ptr(),
+            cache.zero_k.data_ptr(), cache.scale_v.data_ptr(), cache.zero_v.data_ptr())
+    if ptrs != (cache.c.packed_k, cache.c.packed_v, cache.c.scale_k, cache.c.zero_k, cache.c.scale_v, cache.c.zero_v):
+        raise ValueError("cache tensors were replaced after the LayerCache was built")
+    return [(f"cache.{n}", getattr(cache, n)) for n in
+            ("packed_k", "packed_v", "scale_k", "zero_k", "scale_v", "zero_v")]
+
+
 def _dtype(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return VQ_BF16
@@ -156,6 +210,13 @@ class LayerCache:
 def vq_quantize_pack_block(desc: CacheDesc, block: int, x: torch.Tensor, packed: torch.Tensor,
                            scale: torch.Tensor, zero: torch.Tensor, stream=None):
     """Quantize + bit-pack one block of one tensor x [B][H][n_s][D] (bf16/fp32)."""
+    n = _block_tokens(desc, block)
+    _check_slab("x", x, desc, n)
+    bhd = desc.batch * desc.heads * desc.head_dim
+    _check_flat("packed", packed, bhd * desc.word_rows(block), _WORDS)
+    _check_flat("scale", scale, bhd, _F32)
+    _check_flat("zero", zero, bhd, _F32)
+    _check_devices(("x", x), ("packed", packed), ("scale", scale), ("zero", zero))
     _check(_lib.vq_quantize_pack_block(ctypes.byref(desc.c), block, x.data_ptr(), _dtype(x), _strides(x),
                                        packed.data_ptr(), scale.data_ptr(), zero.data_ptr(), _stream(stream)))
 
@@ -164,6 +225,10 @@ def vq_cache_append(desc: CacheDesc, cache: LayerCache, block: int, k: torch.Ten
     """Quantize block `block` of K and V ([B][H][n_s][D] views) into the layer cache."""
     if k.dtype != v.dtype:
         raise ValueError("k and v must have the same dtype")
+    n = _block_tokens(desc, block)
+    _check_slab("k", k, desc, n)
+    _check_slab("v", v, desc, n)
+    _check_devices(("k", k), ("v", v), *_check_cache(desc, cache))
     _check(_lib.vq_cache_append(ctypes.byref(desc.c), ctypes.byref(cache.c), block, k.data_ptr(), v.data_ptr(),
                                 _dtype(k), _strides(k), _strides(v), _stream(stream)))
 
@@ -174,6 +239,10 @@ def vq_attention_block(desc: CacheDesc, cache: LayerCache, block: int, q: torch.
     cache of blocks 0..block; writes out [B][H][n_s][D] (fp32 or bf16)."""
     if q.dtype != torch.bfloat16:
         raise ValueError("q must be bfloat16")
+    n = _block_tokens(desc, block)
+    _check_slab("q", q, desc, n)
+    _check_slab("out", out, desc, n)
+    _check_devices(("q", q), ("out", out), *_check_cache(desc, cache))
     _check(_lib.vq_attention_block(ctypes.byref(desc.c), ctypes.byref(cache.c), block, q.data_ptr(), _strides(q),
                                    ctypes.c_float(softmax_scale), out.data_ptr(), _dtype(out), _strides(out),
                                    _stream(stream)))
@@ -184,6 +253,13 @@ def vq_dequantize(desc: CacheDesc, block: int, packed: torch.Tensor, scale: torc
     """Check-only: dequantize one packed block into out [B][H][n_s][D] float32 (contiguous)."""
     if out.dtype != torch.float32 or not out.is_contiguous():
         raise ValueError("out must be contiguous float32")
+    n = _block_tokens(desc, block)
+    _check_slab("out", out, desc, n)
+    bhd = desc.batch * desc.heads * desc.head_dim
+    _check_flat("packed", packed, bhd * desc.word_rows(block), _WORDS)
+    _check_flat("scale", scale, bhd, _F32)
+    _check_flat("zero", zero, bhd, _F32)
+    _check_devices(("packed", packed), ("scale", scale), ("zero", zero), ("out", out))
     _check(_lib.vq_dequantize(ctypes.byref(desc.c), block, packed.data_ptr(), scale.data_ptr(), zero.data_ptr(),
                               out.data_ptr(), _stream(stream)))
 

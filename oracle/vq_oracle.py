@@ -23,7 +23,8 @@ emulated exactly, and `attention_f64`, which is float64. Function by function:
 
   group_min_max     exact min/max over the block's tokens, per (b, h, channel)
   scale_zero        scale = (max - min) / (2^b - 1); zero = min (+0 for a zero min)
-  encode            code = clamp(rint((x - min) * (1/scale)), 0, 2^b - 1); 0 if scale == 0
+  encode            code = clamp(rint((x - min) * (1/scale)), 0, 2^b - 1); 0 if scale == 0;
+                    float32 steps with an unbounded exponent (see `prescale`)
   pack / unpack     codes along tokens, floor(32/b) per 32-bit word, least significant first
   dequantize        x_hat = fma(code, scale, zero), one rounding
   attention_f64     softmax(sigma * q . k_hat) . v_hat over blocks 0..s, float64
@@ -39,7 +40,6 @@ import numpy as np
 
 F32 = np.float32
 F64 = np.float64
-FLT_MAX = F32(np.finfo(np.float32).max)
 
 
 # ---------------------------------------------------------------- layout
@@ -93,25 +93,50 @@ def scale_zero(mn: np.ndarray, mx: np.ndarray, bits: int):
     return scale, zero
 
 
+TINY_SCALE = F32(2.0 ** -100)
+PRESCALE = F32(2.0 ** 64)
+
+
+def prescale(scale: np.ndarray) -> np.ndarray:
+    """Power of two applied to both d = x - min and scale before the reciprocal.
+
+    2^64 where 0 < scale < 2^-100, else 1. Without it, 1/scale overflows float32
+    for scales below 2^-128 (groups whose range lies in the subnormal range) and
+    the codes stop being the nearest grid levels. Multiplying d and scale by the
+    same power of two is exact here (the products stay normal and below 2^-28),
+    so inv and t come out as float32 arithmetic with an unbounded exponent would
+    give them: the asymmetric min/max grid of the abstract (paragraph 3) holds
+    for every finite group, and every normal-range group is unaffected.
+    """
+    return np.where((scale > 0) & (scale < TINY_SCALE), PRESCALE, F32(1.0)).astype(F32)
+
+
 def reciprocal(scale: np.ndarray) -> np.ndarray:
-    """inv = 1/scale (IEEE float32), saturated at FLT_MAX; 0 where scale == 0 (unused there)."""
+    """inv = 1/(scale * prescale(scale)), IEEE float32; 0 where scale == 0 (unused there).
+
+    With |x| < 2^126 and at least 3 levels, scale < 2^126 and the scaled scale
+    is at least 2^-85, so inv is a normal float32 that never overflows.
+    """
+    s2 = (scale * prescale(scale)).astype(F32)
     with np.errstate(divide="ignore", over="ignore"):
-        inv = (F32(1.0) / scale).astype(F32)
-    inv = np.where(scale > 0, np.minimum(inv, FLT_MAX), F32(0)).astype(F32)
-    return inv
+        inv = (F32(1.0) / s2).astype(F32)
+    return np.where(scale > 0, inv, F32(0)).astype(F32)
 
 
 def encode(x: np.ndarray, mn: np.ndarray, scale: np.ndarray, bits: int) -> np.ndarray:
     """Integer codes of one block: clamp(rint((x - min) * inv), 0, 2^b - 1).
 
-    Three IEEE float32 steps, in this order: d = x - min, t = d * inv, then
-    round half to even. A group whose scale is 0 (constant group, or a single
-    token) encodes to 0 everywhere.
+    IEEE float32 steps, in this order: d = x - min, d = d * pre (pre =
+    prescale(scale), exact), t = d * inv, then round half to even. A group
+    whose scale is 0 (constant group, or a single token) encodes to 0
+    everywhere.
     """
     x = np.asarray(x, dtype=F32)
     mn4 = mn[:, :, None, :]
     inv4 = reciprocal(scale)[:, :, None, :]
+    pre4 = prescale(scale)[:, :, None, :]
     d = (x - mn4).astype(F32)
+    d = (d * pre4).astype(F32)
     t = (d * inv4).astype(F32)
     r = np.rint(t)
     code = np.clip(r, 0, (1 << bits) - 1).astype(np.uint8)

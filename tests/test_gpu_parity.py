@@ -316,3 +316,28 @@ def test_bf16_output(vq):
     vq.vq_attention_block(desc, cache, s, q[:, :, p0:p0 + n], 0.125, o16)
     torch.cuda.synchronize()
     assert torch.equal(o32.to(torch.bfloat16), o16)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_bf16_output_every_kernel(vq, D):
+    """bf16 output = the float32 output rounded to nearest even, for every
+    attention kernel's epilogue: a block of 3 queries (warp per query), 40
+    (CUDA-core kernel), 100 (tensor cores, one query tile per item) and 200
+    (tensor cores, two query tiles per item)."""
+    sched = [3, 40, 100, 200]
+    B, H = 1, 2
+    k, v, q = _ragged_kv(sched, D, H=H, B=B, seed=13)
+    for bits in (3, 4):
+        desc = vq.CacheDesc(B, H, D, bits, sched)
+        cache = vq.LayerCache(desc)
+        p0 = 0
+        for s, n in enumerate(sched):
+            vq.vq_cache_append(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+            o32 = torch.empty((B, H, n, D), dtype=torch.float32, device="cuda")
+            o16 = torch.empty((B, H, n, D), dtype=torch.bfloat16, device="cuda")
+            vq.vq_attention_block(desc, cache, s, q[:, :, p0:p0 + n], 0.125, o32)
+            vq.vq_attention_block(desc, cache, s, q[:, :, p0:p0 + n], 0.125, o16)
+            torch.cuda.synchronize()
+            assert torch.equal(o32.to(torch.bfloat16), o16), (bits, s, n)
+            p0 += n
+    assert vq.vq_poll_device_error() == 0

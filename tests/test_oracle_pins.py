@@ -130,6 +130,77 @@ def test_quantizer_grid_properties():
     check_grid_properties(vo.quantize_pack_block, vo.dequantize, np.random.default_rng(1))
 
 
+def _tiny_range_blocks(rng):
+    """Groups whose whole range is tiny: subnormal values (scale below 2^-128,
+    where 1/scale overflows float32), normal values with a scale just under and
+    over 2^-100, and the arithmetic progression 1e-40 * [0, 19]."""
+    cols = [1e-40 * np.arange(20, dtype=np.float64),
+            1e-40 * np.arange(20, dtype=np.float64)[::-1] - 3e-40,
+            rng.uniform(-1, 1, 20) * 2.0 ** -135,
+            rng.uniform(0, 1, 20) * 2.0 ** -146,
+            2.0 ** -110 * (1 + rng.uniform(0, 2.0 ** -6, 20)),
+            rng.uniform(-1, 1, 20) * 2.0 ** -96,
+            rng.uniform(-1, 1, 20) * 2.0 ** -99,
+            rng.standard_normal(20)]
+    x = np.stack(cols, axis=-1).astype(np.float32)          # [20][8]
+    return x.reshape(1, 1, 20, len(cols))
+
+
+def check_tiny_range_groups(quantize_pack_block, dequantize, rng):
+    """Exact-rational check of the nearest grid level on tiny-range groups.
+
+    With t_exact = (x - min) / scale computed in exact rationals from the stored
+    scale and clamped to [0, 2^b - 1], every code must be within 1/2 + 2^-16 of
+    t_exact (the nearest level up to the float32 roundings of d and t), min -> 0,
+    max -> 2^b - 1 where the scale is a normal float, and the dequantized value
+    within scale/2 (1 + 2^-16) + one ulp of the input + (2^b - 1) 2^-150 (the
+    rounding of a subnormal scale, accumulated over the levels).
+    """
+    for bits in (2, 3, 4, 8):
+        for n in (20, 11, 3):
+            x = _tiny_range_blocks(rng)[:, :, :n]
+            words, scale, zero = quantize_pack_block(x, bits)
+            codes = vo.unpack(words, bits, n).astype(np.int64)
+            for c in range(x.shape[-1]):
+                col = [float(v) for v in x[0, 0, :, c]]
+                lo, hi = min(col), max(col)
+                s = float(scale[0, 0, c])
+                if s == 0.0:
+                    # flat group, or a range so small that (max - min)/(2^b - 1)
+                    # rounds to zero (below half the smallest subnormal): codes 0
+                    assert (Fraction(hi) - Fraction(lo)) / ((1 << bits) - 1) <= Fraction(1, 2**150)
+                    assert all(codes[0, 0, :, c] == 0)
+                    continue
+                assert codes[0, 0, col.index(lo), c] == 0
+                if s >= 2.0 ** -126:
+                    # a normal scale is within 2^-24 of (max - min)/(2^b - 1), so the
+                    # max is nearest the top level; a subnormal scale can be off by
+                    # more than half a level over 2^b - 1 steps, and then the
+                    # nearest-level check below is the property that holds
+                    assert codes[0, 0, col.index(hi), c] == (1 << bits) - 1, (bits, n, c)
+                for t in range(n):
+                    # exact grid position, clamped to the 2^b levels (a subnormal
+                    # scale can put the max past the top level)
+                    t_exact = min(max((Fraction(col[t]) - Fraction(lo)) / Fraction(s), Fraction(0)),
+                                  Fraction((1 << bits) - 1))
+                    assert abs(codes[0, 0, t, c] - t_exact) <= Fraction(1, 2) + Fraction(1, 2**16), \
+                        (bits, n, c, t, float(t_exact), codes[0, 0, t, c])
+            xh = dequantize(words, scale, zero, bits, n)
+            err = np.abs(xh.astype(np.float64) - x.astype(np.float64))
+            mn = x.min(axis=2, keepdims=True)
+            # plus (2^b - 1) * 2^-150: a subnormal scale is rounded to an absolute
+            # 2^-150, so the top level can fall that far short of the max
+            bound = scale[:, :, None, :].astype(np.float64) / 2 * (1 + 2.0 ** -16) + \
+                np.spacing(np.abs(x) + np.abs(mn)).astype(np.float64) + ((1 << bits) - 1) * 2.0 ** -150
+            flat = (scale == 0)[:, :, None, :]
+            bound = np.where(flat, (x.max(axis=2, keepdims=True) - mn).astype(np.float64), bound)
+            assert np.all(err <= bound), (bits, n, float(np.max(err / bound)))
+
+
+def test_quantizer_tiny_range_groups():
+    check_tiny_range_groups(vo.quantize_pack_block, vo.dequantize, np.random.default_rng(10))
+
+
 def test_quantizer_bf16_inputs_and_min_max_exact():
     rng = np.random.default_rng(2)
     x = _rand_block(rng, 2, 3, 29, 64, kind="bf16")
@@ -346,22 +417,25 @@ def test_tiny_workload_end_to_end_consistency():
 
 # ------------------------------------------------------------------ planted mistakes
 def test_planted_mistakes_are_caught(monkeypatch):
-    """Plausible oracle mistakes (wrong level count, floor instead of round, missing
-    sigma, transposed value operand, double-rounded fma, payload 3 bits for INT3)
-    each fail at least one pin above."""
+    """Plausible oracle mistakes (wrong level count, floor instead of round, a
+    saturated 1/scale without the power-of-two prescale, missing sigma,
+    transposed value operand, double-rounded fma, payload 3 bits for INT3) each
+    fail at least one pin above."""
     rng = np.random.default_rng(9)
 
     def wrong_levels(mn, mx, bits):
         levels = np.float32(1 << bits)
         return ((mx - mn) / levels).astype(np.float32), (mn + np.float32(0)).astype(np.float32)
 
-    def qpb_with(scale_zero=None, rint=None):
+    def qpb_with(scale_zero=None, rint=None, recip=None):
         def f(x, bits):
             x = np.asarray(x, dtype=np.float32)
             mn, mx = vo.group_min_max(x)
             sc, z = (scale_zero or vo.scale_zero)(mn, mx, bits)
-            inv = vo.reciprocal(sc)[:, :, None, :]
-            t = ((x - mn[:, :, None, :]).astype(np.float32) * inv).astype(np.float32)
+            inv = (recip or vo.reciprocal)(sc)[:, :, None, :]
+            pre = (vo.prescale(sc) if recip is None else np.ones_like(sc))[:, :, None, :]
+            d = ((x - mn[:, :, None, :]).astype(np.float32) * pre).astype(np.float32)
+            t = (d * inv).astype(np.float32)
             r = (rint or np.rint)(t)
             codes = np.where(sc[:, :, None, :] > 0, np.clip(r, 0, (1 << bits) - 1), 0).astype(np.uint8)
             return vo.pack(codes, bits), sc, z
@@ -371,6 +445,17 @@ def test_planted_mistakes_are_caught(monkeypatch):
         check_grid_properties(qpb_with(scale_zero=wrong_levels), vo.dequantize, rng)
     with pytest.raises(AssertionError):
         check_grid_properties(qpb_with(rint=np.floor), vo.dequantize, rng)
+
+    def saturating_reciprocal(sc):
+        # 1/scale capped at FLT_MAX, with no power-of-two prescale of d and scale
+        with np.errstate(divide="ignore", over="ignore"):
+            inv = (np.float32(1) / sc).astype(np.float32)
+        return np.where(sc > 0, np.minimum(inv, np.finfo(np.float32).max), 0).astype(np.float32)
+
+    with pytest.raises(AssertionError):
+        check_tiny_range_groups(qpb_with(recip=saturating_reciprocal), vo.dequantize, rng)
+    # the pins still pass through the same helper with the oracle's own steps
+    check_tiny_range_groups(qpb_with(), vo.dequantize, rng)
     with pytest.raises(AssertionError):
         check_attention(lambda q, k, v, s: vo.attention_f64(q, k, v, 1.0))
     with pytest.raises(AssertionError):
