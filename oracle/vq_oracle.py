@@ -44,8 +44,9 @@ F64 = np.float64
 
 # ---------------------------------------------------------------- layout
 def codes_per_word(bits: int) -> int:
-    """Codes held by one 32-bit word: 8 (INT4), 10 (INT3; bits 30-31 unused), 16 (INT2), 4 (INT8)."""
-    if bits not in (2, 3, 4, 8):
+    """Codes held by one 32-bit word: 8 (INT4), 10 (INT3; bits 30-31 unused), 16 (INT2),
+    5 (INT6; bits 30-31 unused), 4 (INT8)."""
+    if bits not in (2, 3, 4, 6, 8):
         raise ValueError(f"unsupported bit width {bits}")
     return 32 // bits
 
@@ -273,7 +274,10 @@ def attention_f64(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, softmax_s
 
 # ---------------------------------------------------------------- accounting
 def payload_bits(bits: int) -> float:
-    """Stored bits per code: b, except INT3 at 10 codes per 32-bit word (3.2)."""
+    """Stored bits per code in the results tables' accounting: b, except INT3 at
+    10 codes per 32-bit word (3.2). (INT6 rows appear only for the video models
+    of Table 4, whose token schedules the pages do not give, so no printed
+    number fixes its accounting; 5 codes per word would be 6.4.)"""
     return 32.0 / codes_per_word(bits) if bits == 3 else float(bits)
 
 

@@ -85,8 +85,8 @@ def _rand_block(rng, B, H, n, D, kind="normal"):
 
 def check_grid_properties(quantize_pack_block, dequantize, rng):
     """Codes are in range, hit the extreme levels, and pick the nearest grid level."""
-    for bits in (4, 3, 2, 8):
-        for n in (1, 2, 3, 7, 10, 11, 16, 33):
+    for bits in (4, 3, 2, 6, 8):
+        for n in (1, 2, 3, 5, 7, 10, 11, 16, 33):
             x = _rand_block(rng, 2, 2, n, 16)
             words, scale, zero = quantize_pack_block(x, bits)
             codes = vo.unpack(words, bits, n).astype(np.int64)
@@ -156,7 +156,7 @@ def check_tiny_range_groups(quantize_pack_block, dequantize, rng):
     within scale/2 (1 + 2^-16) + one ulp of the input + (2^b - 1) 2^-150 (the
     rounding of a subnormal scale, accumulated over the levels).
     """
-    for bits in (2, 3, 4, 8):
+    for bits in (2, 3, 4, 6, 8):
         for n in (20, 11, 3):
             x = _tiny_range_blocks(rng)[:, :, :n]
             words, scale, zero = quantize_pack_block(x, bits)
@@ -220,7 +220,7 @@ def test_quantizer_matches_scalar_brute_force():
     is an independent check that the vectorised oracle really works in float32.
     """
     rng = np.random.default_rng(3)
-    for bits in (4, 3):
+    for bits in (4, 3, 6, 8):
         x = _rand_block(rng, 1, 2, 13, 8)
         words, scale, zero = vo.quantize_pack_block(x, bits)
         codes = vo.unpack(words, bits, 13)
@@ -244,7 +244,7 @@ def test_special_cases_constant_equispaced_single_token():
     assert np.all(s == 0) and np.all(w == 0)
     np.testing.assert_array_equal(vo.dequantize(w, s, z, 4, 9), x)
     # exactly 2^b equispaced levels reconstruct exactly
-    for bits in (2, 3, 4):
+    for bits in (2, 3, 4, 6):
         levels = (1 << bits)
         base = np.float32(-1.5)
         step = np.float32(0.25)
@@ -267,7 +267,7 @@ def test_special_cases_constant_equispaced_single_token():
 
 def test_pack_layout_bit_level_and_round_trip():
     rng = np.random.default_rng(5)
-    for bits in (2, 3, 4, 8):
+    for bits in (2, 3, 4, 6, 8):
         cpw = 32 // bits
         for n in (1, cpw - 1, cpw, cpw + 1, 3 * cpw + 2):
             codes = rng.integers(0, 1 << bits, size=(2, 1, n, 5)).astype(np.uint8)

@@ -37,14 +37,15 @@ class Workload:
     outlier_style: str              # "fixed30" (x30, per-block offset) or "massive" (x U(20,50) per cell + bias)
     rope_k: bool                    # pairwise rotation of K channels (RoPE scattering)
     bits: Tuple[int, ...]           # precisions exercised on this workload
+    chunks: Tuple[int, ...] = ()    # explicit block sizes (next-frame video); empty: r_s**2 per scale
 
     @property
     def block_tokens(self) -> Tuple[int, ...]:
-        return tuple(r * r for r in self.sides)
+        return tuple(self.chunks) if self.chunks else tuple(r * r for r in self.sides)
 
     @property
     def num_blocks(self) -> int:
-        return len(self.sides)
+        return len(self.block_tokens)
 
     @property
     def tokens(self) -> int:
@@ -62,12 +63,27 @@ class Workload:
 VAR_SIDES = (1, 2, 3, 4, 5, 6, 8, 10, 13, 16)
 INFINITY_SIDES = (1, 2, 4, 6, 8, 12, 16, 20, 24, 32, 40, 48, 64)
 
+# Next-frame video ("VAR-Q results data (Tables 2-4)", Table 4: Self-Forcing
+# 1.3B, 5-second clips, batch 12; LongLive 1.3B, 30-second clips, batch 20).
+# The pages give no schedule. Assumed here: a 1.3B video model of 30 layers,
+# 12 heads x 128 (hidden 1536), latent frames of 30 x 52 = 1560 tokens,
+# generated in chunks of 3 frames (4680 tokens) that attend block-causally to
+# the cached chunks. Self-Forcing: 21 latent frames, 7 chunks, 32760 tokens
+# (the BF16 KV of Table 4, 67.49 GiB, is 30 * 2 * N * 1536 * 2 B * 12 with
+# N = 32760 to within 0.01 GiB). LongLive: a cache window of 12 frames, 4
+# chunks, 18720 tokens (its BF16 KV, 64.28 GiB at batch 20, gives N = 18720).
+VIDEO_CHUNK = 3 * 1560
+
 WORKLOADS: Dict[str, Workload] = {
     "tiny": Workload("tiny", 1, 1, 64, 1, (1, 2, 3, 4), "f32", 2, "fixed30", False, (4, 3)),
     "var_d16": Workload("var_d16", 16, 16, 64, 8, VAR_SIDES, "bf16", 6, "massive", False, (4, 3)),
     "var_d20": Workload("var_d20", 20, 20, 64, 128, VAR_SIDES, "bf16", 6, "massive", True, (4, 3)),
     "var_d30": Workload("var_d30", 30, 30, 64, 128, VAR_SIDES, "bf16", 6, "massive", True, (3,)),
     "infinity_2b": Workload("infinity_2b", 32, 16, 128, 8, INFINITY_SIDES, "bf16", 8, "massive", True, (4, 3)),
+    "video_self_forcing": Workload("video_self_forcing", 30, 12, 128, 12, (), "bf16", 8, "massive", True, (4, 3),
+                                   chunks=(VIDEO_CHUNK,) * 7),
+    "video_longlive": Workload("video_longlive", 30, 12, 128, 20, (), "bf16", 8, "massive", True, (4, 3),
+                               chunks=(VIDEO_CHUNK,) * 4),
 }
 
 
