@@ -396,36 +396,41 @@ cudaError_t launch_attention_cc(const AttnParams& p, cudaStream_t stream) {
 
 namespace vq {
 
-cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
-  // few queries over few keys: the CUDA-core kernel (a 128-row MMA tile would
-  // be mostly padding); otherwise the tensor cores. More than 128 queries: two
-  // query tiles per work item sharing every dequantized K/V tile; otherwise one
-  // query tile per item, the two softmax warpgroups taking the items in turn
-  if (p.n_q <= kSmallMaxQueries) {
-    if (p.bits == 4 && p.D == 64) return launch_attention_small<4, 64>(p, stream);
-    if (p.bits == 4 && p.D == 128) return launch_attention_small<4, 128>(p, stream);
-    if (p.bits == 3 && p.D == 64) return launch_attention_small<3, 64>(p, stream);
-    if (p.bits == 3 && p.D == 128) return launch_attention_small<3, 128>(p, stream);
-    return cudaErrorInvalidValue;
-  }
-  if (cc_fits(p)) {
-    const bool wide = p.n_q > 16;
-    if (p.bits == 4 && p.D == 64) return wide ? launch_attention_cc<4, 64, 256>(p, stream) : launch_attention_cc<4, 64, 128>(p, stream);
-    if (p.bits == 4 && p.D == 128) return wide ? launch_attention_cc<4, 128, 256>(p, stream) : launch_attention_cc<4, 128, 128>(p, stream);
-    if (p.bits == 3 && p.D == 64) return wide ? launch_attention_cc<3, 64, 256>(p, stream) : launch_attention_cc<3, 64, 128>(p, stream);
-    if (p.bits == 3 && p.D == 128) return wide ? launch_attention_cc<3, 128, 256>(p, stream) : launch_attention_cc<3, 128, 128>(p, stream);
-    return cudaErrorInvalidValue;
-  }
-  const bool pair = p.n_q > 128;
-  if (p.bits == 4 && p.D == 64)
-    return pair ? launch_attention_pipe<4, 64, 2, false>(p, stream) : launch_attention_pipe<4, 64, 2, true>(p, stream);
-  if (p.bits == 4 && p.D == 128)
-    return pair ? launch_attention_pipe<4, 128, 2, false>(p, stream) : launch_attention_pipe<4, 128, 2, true>(p, stream);
-  if (p.bits == 3 && p.D == 64)
-    return pair ? launch_attention_pipe<3, 64, 2, false>(p, stream) : launch_attention_pipe<3, 64, 2, true>(p, stream);
-  if (p.bits == 3 && p.D == 128)
-    return pair ? launch_attention_pipe<3, 128, 2, false>(p, stream) : launch_attention_pipe<3, 128, 2, true>(p, stream);
+namespace {
+
+// Kernel choice per block, by measured speed on the VAR and Infinity shapes:
+// few queries -> one warp per query; few queries over few keys -> the
+// CUDA-core kernel (a 128-row MMA tile would be mostly padding); otherwise the
+// tensor cores. More than 128 queries: two query tiles per work item sharing
+// every dequantized K/V tile; otherwise one query tile per item, the two
+// softmax warpgroups taking the items in turn.
+template <int BITS, int D>
+cudaError_t launch_attention_typed(const AttnParams& p, cudaStream_t stream) {
+  if (p.n_q <= kSmallMaxQueries) return launch_attention_small<BITS, D>(p, stream);
+  if (cc_fits(p))
+    return p.n_q > 16 ? launch_attention_cc<BITS, D, 256>(p, stream) : launch_attention_cc<BITS, D, 128>(p, stream);
+  return p.n_q > 128 ? launch_attention_pipe<BITS, D, 2, false>(p, stream)
+                     : launch_attention_pipe<BITS, D, 2, true>(p, stream);
+}
+
+template <int BITS>
+cudaError_t launch_attention_bits(const AttnParams& p, cudaStream_t stream) {
+  if (p.D == 64) return launch_attention_typed<BITS, 64>(p, stream);
+  if (p.D == 128) return launch_attention_typed<BITS, 128>(p, stream);
   return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream) {
+  switch (p.bits) {
+    case 2: return launch_attention_bits<2>(p, stream);
+    case 3: return launch_attention_bits<3>(p, stream);
+    case 4: return launch_attention_bits<4>(p, stream);
+    case 6: return launch_attention_bits<6>(p, stream);
+    case 8: return launch_attention_bits<8>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace vq

@@ -71,7 +71,8 @@ struct PipeCfg {
   static constexpr int TM_QT = 512 / NQT;                  // tensor-memory columns per query tile
   static constexpr int NS = (NQT == 1) ? 4 : ((D == 64) ? 3 : 2);  // S slots per query tile
   static constexpr int NKV = (D == 64) ? (NQT == 1 ? 4 : 3) : (NQT == 1 ? 3 : 2);  // K/V tile slots
-  static constexpr int NSTG = (D == 64) ? 3 : 2;           // packed-word stages (a third does not fit at 128)
+  // packed-word stages: a third fits only at head_dim 64 with at least 8 codes per word
+  static constexpr int NSTG = (D == 64 && BITS <= 4) ? 3 : 2;
   // K and V of a tile are unpacked as two phases, each announced on its own,
   // when the K/V ring is short (K of a later tile then overlaps the PV that
   // still holds the slot's V); otherwise as one

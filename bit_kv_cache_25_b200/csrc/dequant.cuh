@@ -48,6 +48,7 @@ cudaError_t launch_dequant(const DequantParams& p, cudaStream_t stream) {
     case 2: dequant_kernel<2><<<grid, threads, 0, stream>>>(p); break;
     case 3: dequant_kernel<3><<<grid, threads, 0, stream>>>(p); break;
     case 4: dequant_kernel<4><<<grid, threads, 0, stream>>>(p); break;
+    case 6: dequant_kernel<6><<<grid, threads, 0, stream>>>(p); break;
     case 8: dequant_kernel<8><<<grid, threads, 0, stream>>>(p); break;
     default: return cudaErrorInvalidValue;
   }

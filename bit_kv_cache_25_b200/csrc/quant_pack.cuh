@@ -290,6 +290,7 @@ cudaError_t launch_quant_pack(const QuantParams& p, cudaStream_t stream) {
     VQ_QP_CASE(2)
     VQ_QP_CASE(3)
     VQ_QP_CASE(4)
+    VQ_QP_CASE(6)
     VQ_QP_CASE(8)
     default:
       return cudaErrorInvalidValue;

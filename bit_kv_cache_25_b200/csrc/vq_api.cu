@@ -49,8 +49,8 @@ vq_status check_desc(const vq_cache_desc* d) {
   if (d->batch < 1 || d->heads < 1) return fail(VQ_ERR_INVALID_ARGUMENT, "batch and heads must be >= 1");
   if (d->head_dim != 64 && d->head_dim != 128)
     return fail(VQ_ERR_UNSUPPORTED, "head_dim %d unsupported (64 or 128)", d->head_dim);
-  if (d->bits != 2 && d->bits != 3 && d->bits != 4 && d->bits != 8)
-    return fail(VQ_ERR_UNSUPPORTED, "bits %d unsupported (2, 3, 4 or 8)", d->bits);
+  if (d->bits != 2 && d->bits != 3 && d->bits != 4 && d->bits != 6 && d->bits != 8)
+    return fail(VQ_ERR_UNSUPPORTED, "bits %d unsupported (2, 3, 4, 6 or 8)", d->bits);
   if (d->num_blocks < 1) return fail(VQ_ERR_INVALID_ARGUMENT, "num_blocks must be >= 1");
   if (!d->block_tokens) return fail(VQ_ERR_INVALID_ARGUMENT, "block_tokens is NULL");
   int64_t total = 0;
@@ -202,7 +202,6 @@ vq_status vq_attention_block(const vq_cache_desc* desc, const vq_layer_cache* ca
   vq_status st = check_desc(desc);
   if (st != VQ_OK) return st;
   if ((st = check_block(desc, block)) != VQ_OK) return st;
-  if (desc->bits != 3 && desc->bits != 4) return fail(VQ_ERR_UNSUPPORTED, "attention supports bits 3 and 4");
   if (block >= vq::kMaxBlocks) return fail(VQ_ERR_UNSUPPORTED, "attention supports at most %d blocks", vq::kMaxBlocks);
   if (!cache || !q || !out) return fail(VQ_ERR_INVALID_ARGUMENT, "NULL cache, q or out");
   if (!cache->packed_k || !cache->packed_v || !cache->scale_k || !cache->zero_k || !cache->scale_v || !cache->zero_v)

@@ -23,7 +23,7 @@
  *   packing = codes along tokens: word (w, c) of block s holds tokens
  *             w*cpw .. w*cpw+cpw-1 of channel c, token w*cpw+i in bits
  *             [bits*i, bits*i+bits), cpw = floor(32/bits) (INT4: 8, INT3: 10,
- *             INT2: 16, INT8: 4); unused slots and bits are 0.
+ *             INT2: 16, INT6: 5, INT8: 4); unused slots and bits are 0.
  * Attention of block s (the page gives no attention kernel; this is the plainest
  * reading): every query of block s attends to every cached token of blocks
  * 0..s, its own block included. The cached K/V are the dequantized values
@@ -51,8 +51,8 @@
  *     must be a multiple of 16 bytes. Channels are contiguous (stride 1).
  *   - Strides are in elements, ordered {batch, head, token}.
  *   - Inputs must be finite, with |x| < 2^126 so that max - min stays finite.
- *   - Supported: head_dim 64 or 128; bits 2, 3, 4, 8 for quantize/dequantize;
- *     bits 3 and 4 for attention; K/V in bf16 or float32; queries in bf16.
+ *   - Supported: head_dim 64 or 128; bits 2, 3, 4, 6 or 8; K/V in bf16 or
+ *     float32; queries in bf16; attention over at most 64 blocks.
  */
 #ifndef VQ_H_
 #define VQ_H_
@@ -79,7 +79,7 @@ typedef struct {
   int32_t batch;               /* B >= 1 */
   int32_t heads;               /* H >= 1 */
   int32_t head_dim;            /* D: 64 or 128 */
-  int32_t bits;                /* 2, 3, 4 or 8 */
+  int32_t bits;                /* 2, 3, 4, 6 or 8 */
   int32_t num_blocks;          /* S >= 1: number of blocks (scales) in the schedule */
   const int32_t* block_tokens; /* host array [S]; n_s >= 1 tokens in block s */
 } vq_cache_desc;

@@ -40,10 +40,10 @@ def _desc(**kw):
     return vq.CacheDesc(**a)
 
 
-def test_layout_matches_definition():
-    d = _desc()
+@pytest.mark.parametrize("bits,cpw", [(2, 16), (3, 10), (4, 8), (6, 5), (8, 4)])
+def test_layout_matches_definition(bits, cpw):
+    d = _desc(bits=bits)
     words, meta, offs = vq.vq_cache_layout(d)
-    cpw = 10
     W = [(n + cpw - 1) // cpw for n in d.block_tokens]
     assert offs == [2 * 3 * 64 * sum(W[:s]) for s in range(5)]
     assert words == offs[-1] and meta == 4 * 2 * 3 * 64
@@ -52,6 +52,7 @@ def test_layout_matches_definition():
 @pytest.mark.parametrize("kw,status", [
     (dict(head_dim=96), vq.VQ_ERR_UNSUPPORTED),
     (dict(bits=5), vq.VQ_ERR_UNSUPPORTED),
+    (dict(bits=7), vq.VQ_ERR_UNSUPPORTED),
     (dict(batch=0), vq.VQ_ERR_INVALID_ARGUMENT),
     (dict(block_tokens=[3, 0]), vq.VQ_ERR_INVALID_ARGUMENT),
 ])
@@ -77,11 +78,11 @@ def test_host_validation_before_launch():
     assert _call_quant(d, 1, BAD, [3 * 30 * 64, 30 * 64, 60]) == vq.VQ_ERR_MISALIGNED         # row stride
     assert _call_quant(d, 1, BAD, [3 * 30 * 64, 30 * 64, 64], dtype=7) == vq.VQ_ERR_UNSUPPORTED
     assert b"16 bytes" in lib.vq_last_error() or b"dtype" in lib.vq_last_error()
-    # attention: only bits 3 and 4; NULL cache
-    d2 = _desc(bits=8)
+    # attention: at most 64 blocks; NULL cache (every case fails before a launch)
+    d2 = _desc(bits=8, block_tokens=[1] * 70)
     st = (ctypes.c_int64 * 3)(3 * 30 * 64, 30 * 64, 64)
     cache = vq.vq_layer_cache(BAD, BAD, BAD, BAD, BAD, BAD)
-    assert lib.vq_attention_block(ctypes.byref(d2.c), ctypes.byref(cache), 0, BAD, st, ctypes.c_float(0.125), BAD,
+    assert lib.vq_attention_block(ctypes.byref(d2.c), ctypes.byref(cache), 64, BAD, st, ctypes.c_float(0.125), BAD,
                                   vq.VQ_F32, st, None) == vq.VQ_ERR_UNSUPPORTED
     assert lib.vq_attention_block(ctypes.byref(d.c), None, 0, BAD, st, ctypes.c_float(0.125), BAD,
                                   vq.VQ_F32, st, None) == vq.VQ_ERR_INVALID_ARGUMENT

@@ -33,7 +33,7 @@ def pipe_cfg(BITS, D, NQT):
     TM_QT = 512 // NQT
     c["NS"] = NS = 4 if NQT == 1 else (3 if D == 64 else 2)
     c["NKV"] = NKV = (4 if NQT == 1 else 3) if D == 64 else (3 if NQT == 1 else 2)
-    c["NSTG"] = NSTG = 3 if D == 64 else 2
+    c["NSTG"] = NSTG = 3 if (D == 64 and BITS <= 4) else 2
     c["SPLIT"] = NKV <= 2
     STAGE_Q = D == 64
     QPF = 2 if (STAGE_Q and NQT == 1) else 1
@@ -71,7 +71,7 @@ def pipe_cfg(BITS, D, NQT):
     return c
 
 
-LAUNCHED = [(b, d, 2) for b in (3, 4) for d in (64, 128)]  # every dispatched instantiation
+LAUNCHED = [(b, d, 2) for b in (2, 3, 4, 6, 8) for d in (64, 128)]  # every dispatched instantiation
 
 
 @pytest.mark.parametrize("BITS,D,NQT", LAUNCHED)
@@ -155,7 +155,7 @@ VAR_BLOCKS = [1, 4, 9, 16, 25, 36, 64, 100, 169, 256]
 INFINITY_BLOCKS = [1, 4, 16, 36, 64, 144, 256, 400, 576, 1024, 1600, 2304, 4096]
 
 
-@pytest.mark.parametrize("BITS,D", [(3, 64), (4, 64), (3, 128), (4, 128)])
+@pytest.mark.parametrize("BITS,D", [(b, d) for b in (2, 3, 4, 6, 8) for d in (64, 128)])
 def test_tile_walk_and_unpack_cover_every_key_once(BITS, D):
     check_tiles(BITS, D, VAR_BLOCKS)
     check_tiles(BITS, D, [1, 2, 3, 4])
@@ -369,8 +369,8 @@ def simulate(NQT, NS, NKV, T, n_items, grid, n_qt, cta, seed, ALT, SPLIT, hazard
     return errors
 
 
-def protocol_cases(D, ALT):
-    c = pipe_cfg(3, D, 2)
+def protocol_cases(D, ALT, BITS=3):
+    c = pipe_cfg(BITS, D, 2)
     for T in (1, 2, 3, 11):
         for n_qt in ((1, 2, 3) if ALT else (1, 2, 3, 5)):
             for grid, cta in ((1, 0), (3, 1), (7, 6)):
@@ -381,10 +381,13 @@ def protocol_cases(D, ALT):
                                    n_qt=n_qt, cta=cta, ALT=ALT, SPLIT=c["SPLIT"], NSTG=c["NSTG"])
 
 
-@pytest.mark.parametrize("D,ALT", [(64, True), (64, False), (128, True), (128, False)])
-def test_barrier_protocol_is_clean(D, ALT):
+@pytest.mark.parametrize("D,ALT,BITS", [(64, True, 3), (64, False, 3), (128, True, 3), (128, False, 3),
+                                         (64, True, 8), (64, False, 8)])
+def test_barrier_protocol_is_clean(D, ALT, BITS):
+    """Every ring configuration the kernel is built with: (3 K/V slots, 3 stages)
+    and (3, 2) at head_dim 64 (8+ and fewer codes per word), (2, 2) at 128."""
     n = 0
-    for case in protocol_cases(D, ALT):
+    for case in protocol_cases(D, ALT, BITS):
         for seed in range(2):
             errs = simulate(seed=seed, **case)
             assert not errs, (case, seed, errs[:2])
@@ -456,7 +459,7 @@ def test_cc_kernel_layout_and_dispatch(D):
     for sched in scheds:
         for s in range(len(sched)):
             if dispatch(sched[s], sum(sched[: s + 1]), D) == "cc":
-                for bits in (3, 4):
+                for bits in (2, 3, 4, 6, 8):
                     check_cc_block(sched, s, D, bits)
     # the VAR schedule at head_dim 64: blocks 0-1 warp per query, 2-5 CUDA-core, 6-9 tensor cores
     if D == 64:

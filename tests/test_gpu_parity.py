@@ -141,6 +141,50 @@ def test_full_size_configs_parity(vq, name):
         torch.cuda.empty_cache()
 
 
+# ---------------------------------------------------------------- other bit widths, video shapes
+@pytest.mark.parametrize("name", ["var_d16", "infinity_2b"])
+def test_other_bit_widths_parity(vq, name):
+    """INT2, INT6 and INT8 caches: bit-exact cache and attention parity on the
+    VAR-d16 shape (every row of one layer) and the Infinity-2B shape (sampled)."""
+    w = WORKLOADS[name]
+    layer = 2
+    k, v = make_kv(w, layer, device="cuda")
+    q = make_q(w, layer, device="cuda")
+    full = name == "var_d16"
+    bsel = list(range(w.batch)) if full else [0, w.batch - 1]
+    last = w.num_blocks - 2
+
+    def rows(s, n):
+        if full:
+            return slice(0, n)
+        if s >= last:
+            return slice(0, min(n, 512))
+        return slice(0, min(n, 64)) if s % 4 == 0 else None
+
+    for bits in (2, 6, 8):
+        desc, cache = _append_all(vq, w, bits, k, v)
+        _check_cache_bit_exact(vq, w, bits, desc, cache, k, v, bsel)
+        _check_attention(vq, w, bits, desc, cache, q, k, v, bsel, rows)
+        del cache
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["video_self_forcing", "video_longlive"])
+def test_video_chunk_parity(vq, name):
+    """Next-frame video shapes (uniform 4680-token chunks, head_dim 128) at the
+    video rows' INT6 and INT4: one layer, two batch entries, the first three
+    chunks, 128 sampled query rows per chunk."""
+    import dataclasses
+    w0 = WORKLOADS[name]
+    w = dataclasses.replace(w0, layers=1, batch=2, chunks=w0.chunks[:3])
+    k, v = make_kv(w, 0, device="cuda")
+    q = make_q(w, 0, device="cuda")
+    for bits in w.bits:
+        desc, cache = _append_all(vq, w, bits, k, v)
+        _check_cache_bit_exact(vq, w, bits, desc, cache, k, v, [0, 1])
+        _check_attention(vq, w, bits, desc, cache, q, k, v, [0, 1], lambda s, n: slice(n // 2, n // 2 + 128))
+
+
 # ---------------------------------------------------------------- edge cases
 def _ragged_kv(sched, D, H=3, B=1, dtype=torch.bfloat16, seed=5):
     g = torch.Generator(device="cuda").manual_seed(seed)
@@ -154,12 +198,12 @@ def _ragged_kv(sched, D, H=3, B=1, dtype=torch.bfloat16, seed=5):
 
 @pytest.mark.parametrize("D", [64, 128])
 def test_ragged_blocks_all_bit_widths(vq, D):
-    """Odd block sizes (1, INT3 word-row tails, slabs split across warp groups) for bits 2/3/4/8;
-    dequantize is bit-exact too."""
+    """Odd block sizes (1, INT3 word-row tails, slabs split across warp groups) for bits 2/3/4/6/8;
+    dequantize is bit-exact too, and attention is within the bar at every width."""
     sched = [1, 2, 7, 11, 81, 300, 1100, 4095]
     k, v, q = _ragged_kv(sched, D)
     B, H = 1, 3
-    for bits in (2, 3, 4, 8):
+    for bits in (2, 3, 4, 6, 8):
         desc = vq.CacheDesc(B, H, D, bits, sched)
         cache = vq.LayerCache(desc)
         p0 = 0
@@ -189,8 +233,7 @@ def test_ragged_blocks_all_bit_widths(vq, D):
             np.testing.assert_array_equal(deq.cpu().numpy().view(np.uint32), x_ref.view(np.uint32))
             p0 += n
         assert vq.vq_poll_device_error() == 0
-        if bits in (3, 4):
-            _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D)
+        _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D)
 
 
 @pytest.mark.parametrize("D", [64, 128])

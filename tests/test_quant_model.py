@@ -64,7 +64,7 @@ def check(n, bits, V, units, grid):
 
 @pytest.mark.parametrize("n", [1, 2, 4, 9, 16, 17, 25, 36, 64, 100, 256])
 def test_quant_work_split_covers_every_vector_once(n):
-    for bits, V, units, grid in itertools.product((2, 3, 4, 8), (8, 16, 32), (3, 256, 1000), (1, 148)):
+    for bits, V, units, grid in itertools.product((2, 3, 4, 6, 8), (8, 16, 32), (3, 256, 1000), (1, 148)):
         if units * n <= 16000:
             check(n, bits, V, units, grid)
 

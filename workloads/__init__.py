@@ -80,9 +80,9 @@ WORKLOADS: Dict[str, Workload] = {
     "var_d20": Workload("var_d20", 20, 20, 64, 128, VAR_SIDES, "bf16", 6, "massive", True, (4, 3)),
     "var_d30": Workload("var_d30", 30, 30, 64, 128, VAR_SIDES, "bf16", 6, "massive", True, (3,)),
     "infinity_2b": Workload("infinity_2b", 32, 16, 128, 8, INFINITY_SIDES, "bf16", 8, "massive", True, (4, 3)),
-    "video_self_forcing": Workload("video_self_forcing", 30, 12, 128, 12, (), "bf16", 8, "massive", True, (4, 3),
+    "video_self_forcing": Workload("video_self_forcing", 30, 12, 128, 12, (), "bf16", 8, "massive", True, (6, 4),
                                    chunks=(VIDEO_CHUNK,) * 7),
-    "video_longlive": Workload("video_longlive", 30, 12, 128, 20, (), "bf16", 8, "massive", True, (4, 3),
+    "video_longlive": Workload("video_longlive", 30, 12, 128, 20, (), "bf16", 8, "massive", True, (6, 4),
                                chunks=(VIDEO_CHUNK,) * 4),
 }
 
