@@ -275,6 +275,282 @@ cudaError_t launch_typed(const QuantParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// ---- register-resident variant: every input byte is loaded once.
+// A task is one word row of one 16-byte channel vector (cpw rows x 16 bytes).
+// A team of TT threads owns a unit; thread i holds tasks i, i + TT*C, ... (at
+// most R) in registers, all loads issued before the first use. Teams of up to
+// 32 threads live inside one warp (32 / TT units per warp); larger teams sync
+// on a named barrier; a unit larger than one CTA is split over a cluster of C
+// CTAs whose min/max meet in distributed shared memory. The group statistics
+// then come from the registers, so the encode needs no second read.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float4 ld_dsmem_f4(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(remote)
+               : "memory");
+  return v;
+}
+
+template <class Vec, int BITS>
+__global__ void __launch_bounds__(kQuantRegThreads, 1) quant_reg_kernel(const __grid_constant__ QuantParams p) {
+  constexpr int CPW = 32 / BITS;
+  constexpr int CH = Vec::kCh;
+  constexpr int R = quant_reg_tasks(BITS);
+  constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
+  extern __shared__ __align__(16) float qsm[];  // red [2][16 warps][2][D], cred [2][2][D]
+  const int D = p.D;
+  const int V = p.vecs_per_row;
+  const int TT = p.TT;
+  const int C = p.C;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int team = tid / TT;
+  const int i = tid - team * TT;
+  const int teams = kQuantRegThreads / TT;
+  const int j = i % V;
+  const int rank = (C > 1) ? static_cast<int>(cluster_rank()) : 0;
+  const int cl = blockIdx.x / C, ncl = gridDim.x / C;
+  const int tasks = p.W * V;
+  const int tstride = TT * C;
+  const int tfirst = rank * TT + i;
+  const int BH = p.B * p.H;
+  const int span = min(TT, 32);        // lanes of a warp that share one unit
+  float* red = qsm;                    // [2][16][2][D]
+  float* cred = qsm + 2 * 16 * 2 * D;  // [2][2][D]
+  int par = 0;
+  // every thread of the CTA runs the same rounds (shuffles, barriers); a team
+  // whose unit is past the end loads a valid address and stores nothing
+  for (int r0 = cl * teams; r0 < p.units; r0 += ncl * teams, par ^= 1) {
+    const int unit = r0 + team;
+    const bool live = unit < p.units;
+    const QuantTensor& T = p.t[(live ? unit : r0) / BH];
+    const int bh = (live ? unit : r0) % BH;
+    const unsigned char* slab =
+        static_cast<const unsigned char*>(T.x) + ((bh / p.H) * T.sb + (bh % p.H) * T.sh) * p.esize + j * 16;
+    const int64_t rstride = T.st * p.esize;
+    // the first task's loads always go out (a thread without a task reads row
+    // 0 of a valid slab and ignores it), the others only where the task exists
+    uint4 v[R][CPW];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int t = tfirst + k * tstride;
+      const bool has = live && t < tasks;
+      const int w = has ? t / V : 0;
+      if (k == 0 || has) {
+#pragma unroll
+        for (int c2 = 0; c2 < CPW; ++c2) v[k][c2] = ldg128(slab + min(w * CPW + c2, p.n - 1) * rstride);
+      }
+    }
+    uint32_t mn[4], mx[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      mn[k] = Vec::kMnInit;
+      mx[k] = Vec::kMxInit;
+    }
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      if (live && tfirst + k * tstride < tasks) {
+#pragma unroll
+        for (int c2 = 0; c2 < CPW; ++c2) Vec::minmax_acc(mn, mx, v[k][c2]);  // rows past n repeat row n-1
+      }
+    }
+    float fmn[CH], fmx[CH];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      fmn[c] = Vec::ch(mn, c);
+      fmx[c] = Vec::ch(mx, c);
+    }
+    for (int off = V; off < span; off <<= 1) {
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        fmn[c] = fminf(fmn[c], __shfl_xor_sync(0xffffffffu, fmn[c], off));
+        fmx[c] = fmaxf(fmx[c], __shfl_xor_sync(0xffffffffu, fmx[c], off));
+      }
+    }
+    if (TT > 32) {
+      // warp partials of this team -> shared memory, then every thread reduces
+      // its channels over the team's warps (and, in a cluster, over the CTAs)
+      const int nw = TT / 32;
+      const int wt = (i >> 5);
+      float* rb = red + ((par * 16) + team * nw) * 2 * D;
+      if (lane < V) {
+#pragma unroll
+        for (int q = 0; q < CH / 4; ++q) {
+          reinterpret_cast<float4*>(rb + wt * 2 * D + CH * j)[q] =
+              make_float4(fmn[4 * q], fmn[4 * q + 1], fmn[4 * q + 2], fmn[4 * q + 3]);
+          reinterpret_cast<float4*>(rb + wt * 2 * D + D + CH * j)[q] =
+              make_float4(fmx[4 * q], fmx[4 * q + 1], fmx[4 * q + 2], fmx[4 * q + 3]);
+        }
+      }
+      if (C > 1) {
+        __syncthreads();
+        // thread c < D: channel c over the CTA's 16 warps -> cred[par]
+        if (tid < D) {
+          float a = INFINITY, b = -INFINITY;
+          for (int q = 0; q < nw; ++q) {
+            a = fminf(a, rb[q * 2 * D + tid]);
+            b = fmaxf(b, rb[q * 2 * D + D + tid]);
+          }
+          cred[(par * 2) * D + tid] = a;
+          cred[(par * 2 + 1) * D + tid] = b;
+        }
+        cluster_sync();
+        for (int q = 0; q < C; ++q) {
+#pragma unroll
+          for (int c4 = 0; c4 < CH / 4; ++c4) {
+            const float4 a = ld_dsmem_f4(cred + (par * 2) * D + CH * j + 4 * c4, q);
+            const float4 b = ld_dsmem_f4(cred + (par * 2 + 1) * D + CH * j + 4 * c4, q);
+            fmn[4 * c4] = fminf(fmn[4 * c4], a.x);
+            fmn[4 * c4 + 1] = fminf(fmn[4 * c4 + 1], a.y);
+            fmn[4 * c4 + 2] = fminf(fmn[4 * c4 + 2], a.z);
+            fmn[4 * c4 + 3] = fminf(fmn[4 * c4 + 3], a.w);
+            fmx[4 * c4] = fmaxf(fmx[4 * c4], b.x);
+            fmx[4 * c4 + 1] = fmaxf(fmx[4 * c4 + 1], b.y);
+            fmx[4 * c4 + 2] = fmaxf(fmx[4 * c4 + 2], b.z);
+            fmx[4 * c4 + 3] = fmaxf(fmx[4 * c4 + 3], b.w);
+          }
+        }
+      } else {
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(TT) : "memory");
+        for (int q = 0; q < nw; ++q) {
+#pragma unroll
+          for (int c4 = 0; c4 < CH / 4; ++c4) {
+            const float4 a = reinterpret_cast<const float4*>(rb + q * 2 * D + CH * j)[c4];
+            const float4 b = reinterpret_cast<const float4*>(rb + q * 2 * D + D + CH * j)[c4];
+            fmn[4 * c4] = fminf(fmn[4 * c4], a.x);
+            fmn[4 * c4 + 1] = fminf(fmn[4 * c4 + 1], a.y);
+            fmn[4 * c4 + 2] = fminf(fmn[4 * c4 + 2], a.z);
+            fmn[4 * c4 + 3] = fminf(fmn[4 * c4 + 3], a.w);
+            fmx[4 * c4] = fmaxf(fmx[4 * c4], b.x);
+            fmx[4 * c4 + 1] = fmaxf(fmx[4 * c4 + 1], b.y);
+            fmx[4 * c4 + 2] = fmaxf(fmx[4 * c4 + 2], b.z);
+            fmx[4 * c4 + 3] = fmaxf(fmx[4 * c4 + 3], b.w);
+          }
+        }
+      }
+    }
+    // scale, zero and the encode constants of this thread's channels (see the
+    // streaming kernel above for the 2^64 prescale of tiny scales)
+    float inv[CH], pre[CH], nmp[CH];
+    {
+      float scl[CH], zer[CH];
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), kLevels);
+        zer[c] = __fadd_rn(fmn[c], 0.0f);
+        pre[c] = (scl[c] > 0.0f && scl[c] < 0x1p-100f) ? 0x1p64f : 1.0f;
+        inv[c] = (scl[c] > 0.0f) ? __frcp_rn(__fmul_rn(scl[c], pre[c])) : 0.0f;
+        nmp[c] = __fmul_rn(-fmn[c], pre[c]);
+      }
+      if (live && tfirst < V) {
+        float* sd = T.scale + static_cast<size_t>(bh) * D + CH * j;
+        float* zd = T.zero + static_cast<size_t>(bh) * D + CH * j;
+#pragma unroll
+        for (int q = 0; q < CH / 4; ++q) {
+          reinterpret_cast<float4*>(sd)[q] = make_float4(scl[4 * q], scl[4 * q + 1], scl[4 * q + 2], scl[4 * q + 3]);
+          reinterpret_cast<float4*>(zd)[q] = make_float4(zer[4 * q], zer[4 * q + 1], zer[4 * q + 2], zer[4 * q + 3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int t = tfirst + k * tstride;
+      if (live && t < tasks) {
+        const int w = t / V;
+        const int nvalid = min(CPW, p.n - w * CPW);
+        uint32_t acc[CH];
+#pragma unroll
+        for (int c = 0; c < CH; ++c) acc[c] = 0u;
+        uint32_t corr = 0u;
+#pragma unroll
+        for (int c2 = 0; c2 < CPW; ++c2) {
+          if (c2 < nvalid) {
+            corr += kRoundMagicBits << (BITS * c2);
+#pragma unroll
+            for (int c = 0; c < CH; ++c) {
+              const float d = __fmaf_rn(Vec::elem(v[k][c2], c), pre[c], nmp[c]);
+              const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
+              const float rq = __fadd_rn(tq, kRoundMagic);
+              acc[c] += __float_as_uint(rq) << (BITS * c2);
+            }
+          }
+        }
+        uint32_t* dst = T.packed + (static_cast<size_t>(bh) * p.W + w) * D + CH * j;
+#pragma unroll
+        for (int q = 0; q < CH / 4; ++q)
+          reinterpret_cast<uint4*>(dst)[q] =
+              make_uint4(acc[4 * q] - corr, acc[4 * q + 1] - corr, acc[4 * q + 2] - corr, acc[4 * q + 3] - corr);
+      }
+    }
+  }
+  // no CTA of a cluster may leave while another can still read its shared memory
+  if (C > 1) cluster_sync();
+}
+
+size_t quant_reg_smem_bytes(int D) { return static_cast<size_t>(2 * 16 * 2 * D + 2 * 2 * D) * sizeof(float); }
+
+template <class Vec, int BITS>
+cudaError_t launch_reg(const QuantParams& p, cudaStream_t stream) {
+  auto kern = quant_reg_kernel<Vec, BITS>;
+  static int sm_count[kMaxDevices] = {};
+  static bool configured[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(quant_reg_smem_bytes(128)));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const size_t smem = quant_reg_smem_bytes(p.D);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(kQuantRegThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  if (p.C > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(p.C, 1, 1);
+    int max_clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+    if (e != cudaSuccess || max_clusters < 1) {
+      cudaGetLastError();  // clear a sticky-free query error; the streaming kernel takes the unit
+      return launch_typed<Vec, BITS>(p, stream);
+    }
+    const int clusters = p.units < max_clusters ? p.units : max_clusters;
+    cfg.gridDim = dim3(clusters * p.C, 1, 1);
+  } else {
+    const int teams = kQuantRegThreads / p.TT;
+    const int ctas = (p.units + teams - 1) / teams;
+    cfg.gridDim = dim3(ctas < sm_count[dev] ? ctas : sm_count[dev], 1, 1);
+  }
+  e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t quant_smem_bytes(int D) { return static_cast<size_t>(2) * kQuantWarps * 2 * D * sizeof(float); }
@@ -283,8 +559,9 @@ int quant_warps() { return kQuantWarps; }
 
 cudaError_t launch_quant_pack(const QuantParams& p, cudaStream_t stream) {
   const bool bf16 = (p.esize == 2);
-#define VQ_QP_CASE(B)                                                                   \
-  case B:                                                                               \
+#define VQ_QP_CASE(B)                                                                          \
+  case B:                                                                                      \
+    if (p.reg) return bf16 ? launch_reg<Bf16Vec, B>(p, stream) : launch_reg<F32Vec, B>(p, stream); \
     return bf16 ? launch_typed<Bf16Vec, B>(p, stream) : launch_typed<F32Vec, B>(p, stream);
   switch (p.bits) {
     VQ_QP_CASE(2)
