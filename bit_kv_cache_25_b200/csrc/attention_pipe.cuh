@@ -69,8 +69,11 @@ struct PipeCfg {
   static constexpr int MAXSEG = (D == 64) ? 8 : 4;         // block segments per tile
   static constexpr int MAXROWS = (KT + CPW - 1) / CPW + 2 * MAXSEG;  // staged word rows per tensor
   static constexpr int TM_QT = 512 / NQT;                  // tensor-memory columns per query tile
-  static constexpr int NS = (NQT == 1) ? 4 : ((D == 64) ? 3 : 2);  // S slots per query tile
-  static constexpr int NKV = (D == 64) ? (NQT == 1 ? 4 : 3) : (NQT == 1 ? 3 : 2);  // K/V tile slots
+  // head_dim 64: the queries live in tensor memory (the QK^T MMAs then read
+  // only K from shared memory); at 128 their D/2 columns do not fit
+  static constexpr bool Q_TMEM = (D == 64);
+  static constexpr int NS = (NQT == 1) ? 4 : 2;            // S slots per query tile
+  static constexpr int NKV = (D == 64) ? 4 : (NQT == 1 ? 3 : 2);  // K/V tile slots
   // packed-word stages: a third fits only at head_dim 64 with at least 8 codes per word
   static constexpr int NSTG = (D == 64 && BITS <= 4) ? 3 : 2;
   // K and V of a tile are unpacked as two phases, each announced on its own,
@@ -86,7 +89,7 @@ struct PipeCfg {
   static constexpr int MMA_WARP = PROD_WARP + 1;
   static constexpr int THREADS = (MMA_WARP + 1) * 32;
   // ---- shared memory (byte offsets from a 1024-aligned base)
-  static constexpr int Q_SZ = 128 * D * 2;                 // fp16 q [128][D] per query tile, K-major SW128
+  static constexpr int Q_SZ = Q_TMEM ? 0 : 128 * D * 2;    // fp16 q [128][D] per query tile, K-major SW128
   static constexpr int Q0 = 0;
   static constexpr int TILE_SZ = KT * D * 2;               // fp16 [KT][D], K-major SW128
   static constexpr int KV0 = Q0 + NQT * Q_SZ;              // NKV x {K hi, K lo, V hi, V lo}
@@ -115,10 +118,13 @@ struct PipeCfg {
   static_assert(HDR0 % 16 == 0 && BARS % 8 == 0, "header alignment");
   static_assert(SMEM_ALLOC <= 232448, "shared memory per CTA");
   static_assert(NRED > NKV, "exponent slots");
-  // ---- tensor memory: query tile qt owns columns [qt * TM_QT, +TM_QT): NS S slots of KT columns, then O
+  // ---- tensor memory: query tile qt owns columns [qt * TM_QT, +TM_QT): NS S
+  // slots of KT columns, then O (D columns), then (Q_TMEM) q as fp16 pairs:
+  // column COL_Q + c/2 holds channels c, c+1 of the lane's query row
   static constexpr int COL_O = NS * KT;
+  static constexpr int COL_Q = COL_O + D;
   static constexpr int TMEM_COLS = 512;
-  static_assert(NS * KT + D <= TM_QT, "tensor memory");
+  static_assert(NS * KT + D + (Q_TMEM ? D / 2 : 0) <= TM_QT, "tensor memory");
 };
 
 // 16-byte asynchronous copy global -> shared (L2 only); src_bytes = 0 fills zeros.
@@ -331,16 +337,27 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       // misses on code that no other warp shares.
       auto issue_qk = [&](int qt, int slot, int kvs, int nk16) {
         const uint32_t idesc = tc::idesc_f16_f32(128, nk16);
-        const uint64_t qd = qdesc + static_cast<uint64_t>((qt * C::Q_SZ) >> 4);
         const uint64_t kd = kdesc0 + static_cast<uint64_t>((kvs * C::KV_SZ) >> 4);
         const uint32_t d = tmem + qt * C::TM_QT + slot * KT;
         constexpr int kSlabA = 128 * 128, kSlabB = KT * 128;
+        if constexpr (C::Q_TMEM) {
+          // A = q from tensor memory: 8 columns (16 fp16 channels) per k-step
+          const uint32_t qa = tmem + qt * C::TM_QT + C::COL_Q;
 #pragma unroll 1
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = qd + static_cast<uint64_t>(((kk >> 2) * kSlabA + (kk & 3) * 32) >> 4);
-          const uint64_t b = kd + static_cast<uint64_t>(((kk >> 2) * kSlabB + (kk & 3) * 32) >> 4);
-          tc::mma_f16_ss(d, a, b, idesc, kk > 0 ? 1u : 0u);                         // q . K^hi
-          tc::mma_f16_ss(d, a, b + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc, 1u);  // q . K^lo
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t b = kd + static_cast<uint64_t>(((kk >> 2) * kSlabB + (kk & 3) * 32) >> 4);
+            tc::mma_f16_ts(d, qa + 8 * kk, b, idesc, kk > 0 ? 1u : 0u);                         // q . K^hi
+            tc::mma_f16_ts(d, qa + 8 * kk, b + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc, 1u);  // q . K^lo
+          }
+        } else {
+          const uint64_t qd = qdesc + static_cast<uint64_t>((qt * C::Q_SZ) >> 4);
+#pragma unroll 1
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = qd + static_cast<uint64_t>(((kk >> 2) * kSlabA + (kk & 3) * 32) >> 4);
+            const uint64_t b = kd + static_cast<uint64_t>(((kk >> 2) * kSlabB + (kk & 3) * 32) >> 4);
+            tc::mma_f16_ss(d, a, b, idesc, kk > 0 ? 1u : 0u);                         // q . K^hi
+            tc::mma_f16_ss(d, a, b + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc, 1u);  // q . K^lo
+          }
         }
         tc::commit(s_full(qt, slot));
       };
@@ -696,17 +713,37 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       const uint32_t a2 = __vmaxu2(__vmaxu2(am[0], am[1]), __vmaxu2(am[2], am[3]));
       float mul, inv;
       pipe_pow2(__uint_as_float(max(a2 & 0xffffu, a2 >> 16) << 16), mul, inv);
-#pragma unroll 4
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 v = q_chunk(item, buf, c);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t h[4];
+      if constexpr (C::Q_TMEM) {
+        // fp16 pairs of the row into this lane's D/2 tensor-memory columns
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          h[k] = tc::cvt_half2(__uint_as_float(w[k] << 16) * inv, __uint_as_float(w[k] & 0xffff0000u) * inv);
-        tc::sts128(qs + tc::sw128_offset(row, 8 * c, 128), h[0], h[1], h[2], h[3]);
+        for (int c16 = 0; c16 < D / 32; ++c16) {
+          uint32_t h[16];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const uint4 v = q_chunk(item, buf, 4 * c16 + cc);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              h[4 * cc + k] =
+                  tc::cvt_half2(__uint_as_float(w[k] << 16) * inv, __uint_as_float(w[k] & 0xffff0000u) * inv);
+          }
+          tc::tmem_st16(tq + C::COL_Q + 16 * c16, h);
+        }
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+      } else {
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 v = q_chunk(item, buf, c);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          uint32_t h[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            h[k] = tc::cvt_half2(__uint_as_float(w[k] << 16) * inv, __uint_as_float(w[k] & 0xffff0000u) * inv);
+          tc::sts128(qs + tc::sw128_offset(row, 8 * c, 128), h[0], h[1], h[2], h[3]);
+        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(q_full(qt));
       return mul;

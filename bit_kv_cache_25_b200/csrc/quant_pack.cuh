@@ -291,24 +291,48 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ float4 ld_dsmem_f4(const float* local, uint32_t rank) {
+
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(remote)
-               : "memory");
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
   return v;
 }
 
 template <class Vec, int BITS>
+struct QReg {
+  static constexpr int CPW = 32 / BITS;
+  static constexpr int CH = Vec::kCh;
+  static constexpr int R = quant_reg_tasks(BITS);
+  // the next unit's rows are loaded while this unit is encoded when two sets
+  // of input registers fit (at most 40 registers each)
+  static constexpr int PF = (R * CPW * 4 <= 40) ? 2 : 1;
+  using Rows = uint4[R][CPW];
+};
+
+// Team-wide encode constants of one channel: inv = 1/(scale * pre),
+// pre = 2^64 for a scale below 2^-100 (else 1), nmp = -min * pre.
+__device__ __forceinline__ void qreg_params(float mn, float mx, float levels, float& scl, float& zer, float& inv,
+                                            float& pre, float& nmp) {
+  scl = __fdiv_rn(__fsub_rn(mx, mn), levels);
+  zer = __fadd_rn(mn, 0.0f);
+  pre = (scl > 0.0f && scl < 0x1p-100f) ? 0x1p64f : 1.0f;
+  inv = (scl > 0.0f) ? __frcp_rn(__fmul_rn(scl, pre)) : 0.0f;
+  nmp = __fmul_rn(-mn, pre);
+}
+
+template <class Vec, int BITS>
 __global__ void __launch_bounds__(kQuantRegThreads, 1) quant_reg_kernel(const __grid_constant__ QuantParams p) {
-  constexpr int CPW = 32 / BITS;
-  constexpr int CH = Vec::kCh;
-  constexpr int R = quant_reg_tasks(BITS);
+  using Q = QReg<Vec, BITS>;
+  constexpr int CPW = Q::CPW;
+  constexpr int CH = Q::CH;
+  constexpr int R = Q::R;
   constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
-  extern __shared__ __align__(16) float qsm[];  // red [2][16 warps][2][D], cred [2][2][D]
+  // shared memory: red [16 warps][2][D] partials, cred [2][2][D] per-CTA
+  // partials read by the cluster, prm [8 teams][3][D] encode constants, and
+  // per unit parity and team a "some group needs the prescale" flag
+  extern __shared__ __align__(16) float qsm[];
   const int D = p.D;
   const int V = p.vecs_per_row;
   const int TT = p.TT;
@@ -325,23 +349,31 @@ __global__ void __launch_bounds__(kQuantRegThreads, 1) quant_reg_kernel(const __
   const int tstride = TT * C;
   const int tfirst = rank * TT + i;
   const int BH = p.B * p.H;
-  const int span = min(TT, 32);        // lanes of a warp that share one unit
-  float* red = qsm;                    // [2][16][2][D]
-  float* cred = qsm + 2 * 16 * 2 * D;  // [2][2][D]
-  int par = 0;
-  // every thread of the CTA runs the same rounds (shuffles, barriers); a team
-  // whose unit is past the end loads a valid address and stores nothing
-  for (int r0 = cl * teams; r0 < p.units; r0 += ncl * teams, par ^= 1) {
+  const int span = min(TT, 32);
+  const int G = span / V;              // lanes of one team warp that share vector j
+  const int kk = i / V;                // this lane's index among them (TT <= 32)
+  float* red = qsm;                                  // [16][2][D]
+  float* cred = red + 16 * 2 * D;                    // [2][2][D]
+  float* prm = cred + 2 * 2 * D;                     // [8][3][D]
+  int* tiny = reinterpret_cast<int*>(prm + 8 * 3 * D);  // [2][8]
+  const int rstep = ncl * teams;
+
+  auto unit_of = [&](int r0, int& bh, const QuantTensor*& T) -> bool {
     const int unit = r0 + team;
     const bool live = unit < p.units;
-    const QuantTensor& T = p.t[(live ? unit : r0) / BH];
-    const int bh = (live ? unit : r0) % BH;
+    T = &p.t[(live ? unit : r0) / BH];
+    bh = (live ? unit : r0) % BH;
+    return live;
+  };
+  // issue every load of this thread's tasks of round r0 (a thread without a
+  // task reads row 0 of a valid slab for its first task and ignores it)
+  auto load = [&](int r0, uint4 (&v)[R][CPW]) {
+    int bh;
+    const QuantTensor* T;
+    const bool live = unit_of(r0, bh, T);
     const unsigned char* slab =
-        static_cast<const unsigned char*>(T.x) + ((bh / p.H) * T.sb + (bh % p.H) * T.sh) * p.esize + j * 16;
-    const int64_t rstride = T.st * p.esize;
-    // the first task's loads always go out (a thread without a task reads row
-    // 0 of a valid slab and ignores it), the others only where the task exists
-    uint4 v[R][CPW];
+        static_cast<const unsigned char*>(T->x) + ((bh / p.H) * T->sb + (bh % p.H) * T->sh) * p.esize + j * 16;
+    const int64_t rstride = T->st * p.esize;
 #pragma unroll
     for (int k = 0; k < R; ++k) {
       const int t = tfirst + k * tstride;
@@ -352,6 +384,11 @@ __global__ void __launch_bounds__(kQuantRegThreads, 1) quant_reg_kernel(const __
         for (int c2 = 0; c2 < CPW; ++c2) v[k][c2] = ldg128(slab + min(w * CPW + c2, p.n - 1) * rstride);
       }
     }
+  };
+  auto process = [&](int r0, const uint4 (&v)[R][CPW], int par) {
+    int bh;
+    const QuantTensor* T;
+    const bool live = unit_of(r0, bh, T);
     uint32_t mn[4], mx[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -378,12 +415,36 @@ __global__ void __launch_bounds__(kQuantRegThreads, 1) quant_reg_kernel(const __
         fmx[c] = fmaxf(fmx[c], __shfl_xor_sync(0xffffffffu, fmx[c], off));
       }
     }
-    if (TT > 32) {
-      // warp partials of this team -> shared memory, then every thread reduces
-      // its channels over the team's warps (and, in a cluster, over the CTAs)
+    // encode constants of this thread's CH channels
+    float inv[CH], nmp[CH], pre[CH];
+    bool any_tiny;
+    if (TT <= 32) {
+      // the G lanes of vector j split its channels: channel c is owned by lane
+      // kk == c % G, which also writes its scale and zero
+      bool t_own = false;
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        float scl, zer, iv, pr, nm;
+        if (c % G == kk) {
+          qreg_params(fmn[c], fmx[c], kLevels, scl, zer, iv, pr, nm);
+          t_own |= (pr != 1.0f);
+          if (live) {
+            T->scale[static_cast<size_t>(bh) * D + CH * j + c] = scl;
+            T->zero[static_cast<size_t>(bh) * D + CH * j + c] = zer;
+          }
+        } else {
+          iv = pr = nm = 0.0f;
+        }
+        const int src = (lane - kk * V) + (c % G) * V;  // owner lane of channel c in this warp
+        inv[c] = __shfl_sync(0xffffffffu, iv, src);
+        pre[c] = __shfl_sync(0xffffffffu, pr, src);
+        nmp[c] = __shfl_sync(0xffffffffu, nm, src);
+      }
+      any_tiny = __any_sync(0xffffffffu, t_own);
+    } else {
       const int nw = TT / 32;
-      const int wt = (i >> 5);
-      float* rb = red + ((par * 16) + team * nw) * 2 * D;
+      const int wt = i >> 5;
+      float* rb = red + (team * nw) * 2 * D;
       if (lane < V) {
 #pragma unroll
         for (int q = 0; q < CH / 4; ++q) {
@@ -393,9 +454,9 @@ __global__ void __launch_bounds__(kQuantRegThreads, 1) quant_reg_kernel(const __
               make_float4(fmx[4 * q], fmx[4 * q + 1], fmx[4 * q + 2], fmx[4 * q + 3]);
         }
       }
+      float* pm = prm + team * 3 * D;
       if (C > 1) {
         __syncthreads();
-        // thread c < D: channel c over the CTA's 16 warps -> cred[par]
         if (tid < D) {
           float a = INFINITY, b = -INFINITY;
           for (int q = 0; q < nw; ++q) {
@@ -406,61 +467,58 @@ __global__ void __launch_bounds__(kQuantRegThreads, 1) quant_reg_kernel(const __
           cred[(par * 2 + 1) * D + tid] = b;
         }
         cluster_sync();
-        for (int q = 0; q < C; ++q) {
-#pragma unroll
-          for (int c4 = 0; c4 < CH / 4; ++c4) {
-            const float4 a = ld_dsmem_f4(cred + (par * 2) * D + CH * j + 4 * c4, q);
-            const float4 b = ld_dsmem_f4(cred + (par * 2 + 1) * D + CH * j + 4 * c4, q);
-            fmn[4 * c4] = fminf(fmn[4 * c4], a.x);
-            fmn[4 * c4 + 1] = fminf(fmn[4 * c4 + 1], a.y);
-            fmn[4 * c4 + 2] = fminf(fmn[4 * c4 + 2], a.z);
-            fmn[4 * c4 + 3] = fminf(fmn[4 * c4 + 3], a.w);
-            fmx[4 * c4] = fmaxf(fmx[4 * c4], b.x);
-            fmx[4 * c4 + 1] = fmaxf(fmx[4 * c4 + 1], b.y);
-            fmx[4 * c4 + 2] = fmaxf(fmx[4 * c4 + 2], b.z);
-            fmx[4 * c4 + 3] = fmaxf(fmx[4 * c4 + 3], b.w);
+        // the flag of the other parity was last read before this unit's first
+        // barrier and is next set after the next unit's: clear it here
+        if (tid == 0) tiny[(par ^ 1) * 8] = 0;
+        if (tid < D) {
+          float a = INFINITY, b = -INFINITY;
+          for (int q = 0; q < C; ++q) {
+            a = fminf(a, ld_dsmem_f32(cred + (par * 2) * D + tid, q));
+            b = fmaxf(b, ld_dsmem_f32(cred + (par * 2 + 1) * D + tid, q));
+          }
+          float scl, zer, iv, pr, nm;
+          qreg_params(a, b, kLevels, scl, zer, iv, pr, nm);
+          pm[tid] = iv;
+          pm[D + tid] = pr;
+          pm[2 * D + tid] = nm;
+          if (pr != 1.0f) tiny[par * 8 + team] = 1;
+          if (live && rank == 0) {
+            T->scale[static_cast<size_t>(bh) * D + tid] = scl;
+            T->zero[static_cast<size_t>(bh) * D + tid] = zer;
           }
         }
+        __syncthreads();
       } else {
         asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(TT) : "memory");
-        for (int q = 0; q < nw; ++q) {
-#pragma unroll
-          for (int c4 = 0; c4 < CH / 4; ++c4) {
-            const float4 a = reinterpret_cast<const float4*>(rb + q * 2 * D + CH * j)[c4];
-            const float4 b = reinterpret_cast<const float4*>(rb + q * 2 * D + D + CH * j)[c4];
-            fmn[4 * c4] = fminf(fmn[4 * c4], a.x);
-            fmn[4 * c4 + 1] = fminf(fmn[4 * c4 + 1], a.y);
-            fmn[4 * c4 + 2] = fminf(fmn[4 * c4 + 2], a.z);
-            fmn[4 * c4 + 3] = fminf(fmn[4 * c4 + 3], a.w);
-            fmx[4 * c4] = fmaxf(fmx[4 * c4], b.x);
-            fmx[4 * c4 + 1] = fmaxf(fmx[4 * c4 + 1], b.y);
-            fmx[4 * c4 + 2] = fmaxf(fmx[4 * c4 + 2], b.z);
-            fmx[4 * c4 + 3] = fmaxf(fmx[4 * c4 + 3], b.w);
+        if (i == 0) tiny[(par ^ 1) * 8 + team] = 0;  // see the cluster branch
+        for (int c = i; c < D; c += TT) {
+          float a = INFINITY, b = -INFINITY;
+          for (int q = 0; q < nw; ++q) {
+            a = fminf(a, rb[q * 2 * D + c]);
+            b = fmaxf(b, rb[q * 2 * D + D + c]);
+          }
+          float scl, zer, iv, pr, nm;
+          qreg_params(a, b, kLevels, scl, zer, iv, pr, nm);
+          pm[c] = iv;
+          pm[D + c] = pr;
+          pm[2 * D + c] = nm;
+          if (pr != 1.0f) tiny[par * 8 + team] = 1;
+          if (live) {
+            T->scale[static_cast<size_t>(bh) * D + c] = scl;
+            T->zero[static_cast<size_t>(bh) * D + c] = zer;
           }
         }
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(TT) : "memory");
       }
-    }
-    // scale, zero and the encode constants of this thread's channels (see the
-    // streaming kernel above for the 2^64 prescale of tiny scales)
-    float inv[CH], pre[CH], nmp[CH];
-    {
-      float scl[CH], zer[CH];
+      any_tiny = tiny[par * 8 + team] != 0;
 #pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), kLevels);
-        zer[c] = __fadd_rn(fmn[c], 0.0f);
-        pre[c] = (scl[c] > 0.0f && scl[c] < 0x1p-100f) ? 0x1p64f : 1.0f;
-        inv[c] = (scl[c] > 0.0f) ? __frcp_rn(__fmul_rn(scl[c], pre[c])) : 0.0f;
-        nmp[c] = __fmul_rn(-fmn[c], pre[c]);
-      }
-      if (live && tfirst < V) {
-        float* sd = T.scale + static_cast<size_t>(bh) * D + CH * j;
-        float* zd = T.zero + static_cast<size_t>(bh) * D + CH * j;
-#pragma unroll
-        for (int q = 0; q < CH / 4; ++q) {
-          reinterpret_cast<float4*>(sd)[q] = make_float4(scl[4 * q], scl[4 * q + 1], scl[4 * q + 2], scl[4 * q + 3]);
-          reinterpret_cast<float4*>(zd)[q] = make_float4(zer[4 * q], zer[4 * q + 1], zer[4 * q + 2], zer[4 * q + 3]);
-        }
+      for (int q = 0; q < CH / 4; ++q) {
+        const float4 a = reinterpret_cast<const float4*>(pm + CH * j)[q];
+        const float4 b = reinterpret_cast<const float4*>(pm + D + CH * j)[q];
+        const float4 c4 = reinterpret_cast<const float4*>(pm + 2 * D + CH * j)[q];
+        inv[4 * q] = a.x, inv[4 * q + 1] = a.y, inv[4 * q + 2] = a.z, inv[4 * q + 3] = a.w;
+        pre[4 * q] = b.x, pre[4 * q + 1] = b.y, pre[4 * q + 2] = b.z, pre[4 * q + 3] = b.w;
+        nmp[4 * q] = c4.x, nmp[4 * q + 1] = c4.y, nmp[4 * q + 2] = c4.z, nmp[4 * q + 3] = c4.w;
       }
     }
 #pragma unroll
@@ -473,24 +531,72 @@ __global__ void __launch_bounds__(kQuantRegThreads, 1) quant_reg_kernel(const __
 #pragma unroll
         for (int c = 0; c < CH; ++c) acc[c] = 0u;
         uint32_t corr = 0u;
+        if (!any_tiny) {
+          // d = x - min: fma(x, 1, -min) is the same single rounding
 #pragma unroll
-        for (int c2 = 0; c2 < CPW; ++c2) {
-          if (c2 < nvalid) {
-            corr += kRoundMagicBits << (BITS * c2);
+          for (int c2 = 0; c2 < CPW; ++c2) {
+            if (c2 < nvalid) {
+              corr += kRoundMagicBits << (BITS * c2);
 #pragma unroll
-            for (int c = 0; c < CH; ++c) {
-              const float d = __fmaf_rn(Vec::elem(v[k][c2], c), pre[c], nmp[c]);
-              const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
-              const float rq = __fadd_rn(tq, kRoundMagic);
-              acc[c] += __float_as_uint(rq) << (BITS * c2);
+              for (int c = 0; c < CH; ++c) {
+                const float d = __fadd_rn(Vec::elem(v[k][c2], c), nmp[c]);
+                const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
+                acc[c] += __float_as_uint(__fadd_rn(tq, kRoundMagic)) << (BITS * c2);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c2 = 0; c2 < CPW; ++c2) {
+            if (c2 < nvalid) {
+              corr += kRoundMagicBits << (BITS * c2);
+#pragma unroll
+              for (int c = 0; c < CH; ++c) {
+                const float d = __fmaf_rn(Vec::elem(v[k][c2], c), pre[c], nmp[c]);
+                const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
+                acc[c] += __float_as_uint(__fadd_rn(tq, kRoundMagic)) << (BITS * c2);
+              }
             }
           }
         }
-        uint32_t* dst = T.packed + (static_cast<size_t>(bh) * p.W + w) * D + CH * j;
+        uint32_t* dst = T->packed + (static_cast<size_t>(bh) * p.W + w) * D + CH * j;
 #pragma unroll
         for (int q = 0; q < CH / 4; ++q)
           reinterpret_cast<uint4*>(dst)[q] =
               make_uint4(acc[4 * q] - corr, acc[4 * q + 1] - corr, acc[4 * q + 2] - corr, acc[4 * q + 3] - corr);
+      }
+    }
+  };
+
+  if (tid < 16) tiny[tid] = 0;
+  __syncthreads();
+  // every thread of the CTA runs the same rounds (shuffles, barriers); the next
+  // round's loads are issued before this round is processed
+  int r0 = cl * teams;
+  if (r0 < p.units) {
+    if constexpr (Q::PF == 2) {
+      uint4 va[R][CPW], vb[R][CPW];
+      int par = 0;
+      load(r0, va);
+      while (true) {
+        const int r1 = r0 + rstep;
+        if (r1 < p.units) load(r1, vb);
+        process(r0, va, par);
+        par ^= 1;
+        if (r1 >= p.units) break;
+        const int r2 = r1 + rstep;
+        if (r2 < p.units) load(r2, va);
+        process(r1, vb, par);
+        par ^= 1;
+        if (r2 >= p.units) break;
+        r0 = r2;
+      }
+    } else {
+      uint4 va[R][CPW];
+      int par = 0;
+      for (; r0 < p.units; r0 += rstep, par ^= 1) {
+        load(r0, va);
+        process(r0, va, par);
       }
     }
   }
@@ -498,7 +604,9 @@ __global__ void __launch_bounds__(kQuantRegThreads, 1) quant_reg_kernel(const __
   if (C > 1) cluster_sync();
 }
 
-size_t quant_reg_smem_bytes(int D) { return static_cast<size_t>(2 * 16 * 2 * D + 2 * 2 * D) * sizeof(float); }
+size_t quant_reg_smem_bytes(int D) {
+  return static_cast<size_t>(16 * 2 * D + 2 * 2 * D + 8 * 3 * D) * sizeof(float) + 16 * sizeof(int);
+}
 
 template <class Vec, int BITS>
 cudaError_t launch_reg(const QuantParams& p, cudaStream_t stream) {

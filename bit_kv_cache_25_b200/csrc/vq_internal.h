@@ -38,8 +38,12 @@ struct QuantParams {
 };
 
 // Tasks (word-row x 16-byte vector) one thread of the register-resident
-// quantize kernel holds: at most 64 registers of input (R * cpw * 4).
-__host__ __device__ constexpr int quant_reg_tasks(int bits) { return (32 / bits) >= 16 ? 1 : 16 / (32 / bits); }
+// quantize kernel holds: at most 40 registers of input (R * cpw * 4), so that
+// a second set (the next unit's rows, loaded while this one is encoded) fits;
+// INT2 (16 rows per task, 64 registers) keeps one set.
+__host__ __device__ constexpr int quant_reg_tasks(int bits) {
+  return (32 / bits) >= 16 ? 1 : (10 / (32 / bits) > 1 ? 10 / (32 / bits) : 1);
+}
 constexpr int kQuantRegThreads = 512;
 constexpr int kQuantRegMaxCluster = 16;  // above 8 needs the non-portable cluster size
 

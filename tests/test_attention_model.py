@@ -31,14 +31,15 @@ def pipe_cfg(BITS, D, NQT):
     c["MAXSEG"] = MAXSEG = 8 if D == 64 else 4
     c["MAXROWS"] = MAXROWS = -(-KT // CPW) + 2 * MAXSEG
     TM_QT = 512 // NQT
-    c["NS"] = NS = 4 if NQT == 1 else (3 if D == 64 else 2)
-    c["NKV"] = NKV = (4 if NQT == 1 else 3) if D == 64 else (3 if NQT == 1 else 2)
+    c["Q_TMEM"] = Q_TMEM = D == 64
+    c["NS"] = NS = 4 if NQT == 1 else 2
+    c["NKV"] = NKV = 4 if D == 64 else (3 if NQT == 1 else 2)
     c["NSTG"] = NSTG = 3 if (D == 64 and BITS <= 4) else 2
     c["SPLIT"] = NKV <= 2
     STAGE_Q = D == 64
     QPF = 2 if (STAGE_Q and NQT == 1) else 1
     UW = 8 if NQT == 1 else 4
-    Q_SZ = 128 * D * 2
+    Q_SZ = 0 if Q_TMEM else 128 * D * 2
     c["TILE_SZ"] = TILE_SZ = KT * D * 2
     KV0 = NQT * Q_SZ
     KV_SZ = 4 * TILE_SZ
@@ -64,7 +65,7 @@ def pipe_cfg(BITS, D, NQT):
         "header alignment": HDR0 % 16 == 0 and BARS % 8 == 0,
         "shared memory": c["SMEM_ALLOC"] <= SMEM_OPTIN,
         "exponent slots": NRED > NKV,
-        "tensor memory": NS * KT + D <= TM_QT,
+        "tensor memory": NS * KT + D + (D // 2 if Q_TMEM else 0) <= TM_QT,
         "threads": NQT * 128 + UW * 32 + 64 == 448,
     }
     c["UW"] = UW

@@ -82,7 +82,7 @@ REG_THREADS, REG_MAX_CLUSTER = 512, 16
 
 def reg_tasks(bits):
     cpw = 32 // bits
-    return 1 if cpw >= 16 else 16 // cpw
+    return 1 if cpw >= 16 else max(1, 10 // cpw)
 
 
 def reg_plan(W, V, bits):
@@ -188,7 +188,7 @@ def test_reg_quant_plans_of_the_workloads():
     assert reg_plan(-(-16 // 10), 8, 3) == (16, 1)
     assert reg_plan(1, 8, 3) == (8, 1)
     # Infinity-2B (D 128: 16 vectors per row), last block of 4096 tokens: a
-    # cluster of 16 CTAs at INT3, 8 at INT4; video chunks of 4680 tokens at INT6: 16
+    # cluster of 16 CTAs at INT3 and INT4; video chunks of 4680 tokens at INT6: 16
     assert reg_plan(-(-4096 // 10), 16, 3) == (512, 16)
-    assert reg_plan(-(-4096 // 8), 16, 4) == (512, 8)
+    assert reg_plan(-(-4096 // 8), 16, 4) == (512, 16)
     assert reg_plan(-(-4680 // 5), 16, 6) == (512, 16)
