@@ -324,30 +324,33 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       }
     }
   } else if (warp == C::MMA_WARP) {
-    // =========================================================== MMA thread
-    if (lane == 0) {
+    // =========================================================== MMA warp
+    // The whole warp runs this loop (warp-uniform waits and descriptors); one
+    // elected lane issues each tcgen05 instruction. With a single thread
+    // running it, consecutive MMAs issued 85-110 cycles apart in the kernel.
+    {
+      const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
       constexpr uint32_t kLbo = KT * 128;  // 64-channel groups of a [KT][D] V tile read MN-major
       const uint32_t idesc_pv = tc::idesc_f16_f32(128, D, /*b_mn_major=*/true);
       const uint64_t qdesc = tc::sw128_desc(sbase + C::Q0);
       const uint64_t kdesc0 = tc::sw128_desc(sbase + C::KV0);
       const uint64_t vdesc0 = tc::sw128_desc_mn(sbase + C::KV0 + 2 * C::TILE_SZ, kLbo);
-      // The issue loops stay rolled, to keep this warp's code small: with the
-      // sequences unrolled, consecutive MMAs issued 100-190 cycles apart in the
-      // kernel (about 50 when replayed alone), the pattern of instruction-cache
-      // misses on code that no other warp shares.
+      // The issue loops stay rolled, to keep this warp's code small (unrolled,
+      // the single-thread version issued 100-190 cycles apart: instruction-cache
+      // misses on code that no other warp shares).
       auto issue_qk = [&](int qt, int slot, int kvs, int nk16) {
         const uint32_t idesc = tc::idesc_f16_f32(128, nk16);
         const uint64_t kd = kdesc0 + static_cast<uint64_t>((kvs * C::KV_SZ) >> 4);
-        const uint32_t d = tmem + qt * C::TM_QT + slot * KT;
+        const uint32_t d = tm + qt * C::TM_QT + slot * KT;
         constexpr int kSlabA = 128 * 128, kSlabB = KT * 128;
         if constexpr (C::Q_TMEM) {
           // A = q from tensor memory: 8 columns (16 fp16 channels) per k-step
-          const uint32_t qa = tmem + qt * C::TM_QT + C::COL_Q;
+          const uint32_t qa = tm + qt * C::TM_QT + C::COL_Q;
 #pragma unroll 1
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t b = kd + static_cast<uint64_t>(((kk >> 2) * kSlabB + (kk & 3) * 32) >> 4);
-            tc::mma_f16_ts(d, qa + 8 * kk, b, idesc, kk > 0 ? 1u : 0u);                         // q . K^hi
-            tc::mma_f16_ts(d, qa + 8 * kk, b + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc, 1u);  // q . K^lo
+            tc::mma_f16_ts_warp(d, qa + 8 * kk, b, idesc, kk > 0 ? 1u : 0u);                         // q . K^hi
+            tc::mma_f16_ts_warp(d, qa + 8 * kk, b + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc, 1u);  // q . K^lo
           }
         } else {
           const uint64_t qd = qdesc + static_cast<uint64_t>((qt * C::Q_SZ) >> 4);
@@ -355,27 +358,27 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t a = qd + static_cast<uint64_t>(((kk >> 2) * kSlabA + (kk & 3) * 32) >> 4);
             const uint64_t b = kd + static_cast<uint64_t>(((kk >> 2) * kSlabB + (kk & 3) * 32) >> 4);
-            tc::mma_f16_ss(d, a, b, idesc, kk > 0 ? 1u : 0u);                         // q . K^hi
-            tc::mma_f16_ss(d, a, b + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc, 1u);  // q . K^lo
+            tc::mma_f16_ss_warp(d, a, b, idesc, kk > 0 ? 1u : 0u);                         // q . K^hi
+            tc::mma_f16_ss_warp(d, a, b + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc, 1u);  // q . K^lo
           }
         }
-        tc::commit(s_full(qt, slot));
+        tc::commit_warp(s_full(qt, slot));
       };
       auto issue_pv = [&](int qt, int slot, int kvs, int nk16, bool first) {
         const uint64_t vd = vdesc0 + static_cast<uint64_t>((kvs * C::KV_SZ) >> 4);
-        const uint32_t pa = tmem + qt * C::TM_QT + slot * KT;
-        const uint32_t o = tmem + qt * C::TM_QT + C::COL_O;
+        const uint32_t pa = tm + qt * C::TM_QT + slot * KT;
+        const uint32_t o = tm + qt * C::TM_QT + C::COL_O;
         const int nkk = nk16 / 16;
         // per 16-key step: (P hi, V hi), (P lo, V hi), (P hi, V lo); P lo sits 8 columns after P hi
 #pragma unroll 1
         for (int kk = 0; kk < nkk; ++kk) {
           const uint64_t v = vd + static_cast<uint64_t>((kk * 2048) >> 4);
           const uint32_t a = pa + 16 * kk;
-          tc::mma_f16_ts(o, a, v, idesc_pv, (first && kk == 0) ? 0u : 1u);
-          tc::mma_f16_ts(o, a + 8, v, idesc_pv, 1u);
-          tc::mma_f16_ts(o, a, v + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc_pv, 1u);
+          tc::mma_f16_ts_warp(o, a, v, idesc_pv, (first && kk == 0) ? 0u : 1u);
+          tc::mma_f16_ts_warp(o, a + 8, v, idesc_pv, 1u);
+          tc::mma_f16_ts_warp(o, a, v + static_cast<uint64_t>(C::TILE_SZ >> 4), idesc_pv, 1u);
         }
-        tc::commit(pv_done(qt, slot));
+        tc::commit_warp(pv_done(qt, slot));
       };
 
       bool ok = true;
@@ -393,11 +396,11 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           const int nk = tabled ? nktab[j] : w.next(p);
           const int nk16 = (nk + 15) & ~15;
           const int kvs = g % NKV;
-          if (!(ok = mbar_wait_bounded(&k_full[kvs], (g / NKV) & 1))) break;
+          if (!(ok = mbar_wait_warp(&k_full[kvs], (g / NKV) & 1))) break;
           if (j == 0) {
 #pragma unroll
             for (int qt = 0; qt < NQT; ++qt)
-              if (qt >= qlo && qt < qhi && ok) ok = mbar_wait_bounded(q_full(qt), iq[qt]++ & 1);
+              if (qt >= qlo && qt < qhi && ok) ok = mbar_wait_warp(q_full(qt), iq[qt]++ & 1);
             if (!ok) break;
           }
 #pragma unroll
@@ -405,7 +408,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             if (qt >= qlo && qt < qhi && ok) {
               const int n = nq[qt];
               const int slot = n % NS;
-              if (n >= NS) ok = mbar_wait_bounded(pv_done(qt, slot), ((n / NS) - 1) & 1);
+              if (n >= NS) ok = mbar_wait_warp(pv_done(qt, slot), ((n / NS) - 1) & 1);
               if (ok) {
                 tc::fence_after_sync();
                 issue_qk(qt, slot, kvs, nk16);
@@ -413,14 +416,14 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             }
           }
           if (!ok) break;
-          if constexpr (C::SPLIT_KV) tc::commit(&k_empty[kvs]);
+          if constexpr (C::SPLIT_KV) tc::commit_warp(&k_empty[kvs]);
           if (prev) {
-            if (C::SPLIT_KV && !(ok = mbar_wait_bounded(&v_full[prev_kvs], (prev_g / NKV) & 1))) break;
+            if (C::SPLIT_KV && !(ok = mbar_wait_warp(&v_full[prev_kvs], (prev_g / NKV) & 1))) break;
 #pragma unroll
             for (int qt = 0; qt < NQT; ++qt) {
               if (qt >= prev_qlo && qt < prev_qhi && ok) {
                 const int n = prev_n[qt];
-                ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1);
+                ok = mbar_wait_warp(p_full(qt, n % NS), (n / NS) & 1);
                 if (ok) {
                   tc::fence_after_sync();
                   issue_pv(qt, n % NS, prev_kvs, prev_nk16, prev_first);
@@ -428,7 +431,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
               }
             }
             if (!ok) break;
-            tc::commit(&v_empty[prev_kvs]);
+            tc::commit_warp(&v_empty[prev_kvs]);
           }
           prev = true;
           prev_first = (j == 0);
@@ -442,20 +445,20 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             if (qt >= qlo && qt < qhi) prev_n[qt] = nq[qt]++;
         }
       }
-      if (C::SPLIT_KV && ok && prev) ok = mbar_wait_bounded(&v_full[prev_kvs], (prev_g / NKV) & 1);
+      if (C::SPLIT_KV && ok && prev) ok = mbar_wait_warp(&v_full[prev_kvs], (prev_g / NKV) & 1);
       if (ok && prev) {
 #pragma unroll
         for (int qt = 0; qt < NQT; ++qt) {
           if (qt >= prev_qlo && qt < prev_qhi && ok) {
             const int n = prev_n[qt];
-            ok = mbar_wait_bounded(p_full(qt, n % NS), (n / NS) & 1);
+            ok = mbar_wait_warp(p_full(qt, n % NS), (n / NS) & 1);
             if (ok) {
               tc::fence_after_sync();
               issue_pv(qt, n % NS, prev_kvs, prev_nk16, prev_first);
             }
           }
         }
-        if (ok) tc::commit(&v_empty[prev_kvs]);
+        if (ok) tc::commit_warp(&v_empty[prev_kvs]);
       }
     }
   } else if (tid >= C::UNPACK_T0) {
@@ -715,19 +718,19 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       pipe_pow2(__uint_as_float(max(a2 & 0xffffu, a2 >> 16) << 16), mul, inv);
       if constexpr (C::Q_TMEM) {
         // fp16 pairs of the row into this lane's D/2 tensor-memory columns
+#pragma unroll 1
+        for (int c8 = 0; c8 < D / 16; ++c8) {
+          uint32_t h[8];
 #pragma unroll
-        for (int c16 = 0; c16 < D / 32; ++c16) {
-          uint32_t h[16];
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const uint4 v = q_chunk(item, buf, 4 * c16 + cc);
+          for (int cc = 0; cc < 2; ++cc) {
+            const uint4 v = q_chunk(item, buf, 2 * c8 + cc);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               h[4 * cc + k] =
                   tc::cvt_half2(__uint_as_float(w[k] << 16) * inv, __uint_as_float(w[k] & 0xffff0000u) * inv);
           }
-          tc::tmem_st16(tq + C::COL_Q + 16 * c16, h);
+          tc::tmem_st8(tq + C::COL_Q + 8 * c8, h);
         }
         tc::tmem_wait_st();
         tc::fence_before_sync();

@@ -95,10 +95,6 @@ vq_status check_strides(const int64_t st[3], int esize, const char* name) {
 // blocks put several units in flight per warp. Returns false if one slab is
 // too large.
 bool plan_quant(vq::QuantParams& p) {
-  // Streaming kernel (also the fallback): warps per unit (P, enough units x
-  // warps to fill the GPU) and, with one warp per unit, the lanes per unit (TL):
-  // the fewest rows per team load that still cover the unit's rows in one
-  // batch of loads, so that small blocks put several units in flight per warp.
   constexpr int64_t kTargetWarps = 2048;
   constexpr int kBatch = 16;  // loads in flight per lane in pass 1 (kQuantUnroll)
   int P = 1;
@@ -109,31 +105,6 @@ bool plan_quant(vq::QuantParams& p) {
   while (rw * kBatch < p.n && rw * p.vecs_per_row < 32) rw *= 2;
   p.TL = (P == 1) ? rw * p.vecs_per_row : 32;
   if (p.TL > 32) p.TL = 32;
-  // Register-resident kernel: a team of TT threads (the smallest power of two,
-  // at least one 16-byte vector row, whose registers hold the unit's tasks),
-  // or a cluster of C CTAs when one CTA cannot hold the unit.
-  const int R = vq::quant_reg_tasks(p.bits);
-  const int64_t tasks = int64_t(p.W) * p.vecs_per_row;
-  const int64_t cap = int64_t(vq::kQuantRegThreads) * R;
-  p.reg = 0;
-  p.TT = 0;
-  p.C = 1;
-  if (tasks <= cap * vq::kQuantRegMaxCluster) {
-    p.reg = 1;
-    if (tasks <= cap) {
-      int TT = p.vecs_per_row;
-      while (TT < 32 && TT < tasks) TT *= 2;
-      if (TT >= 32) {
-        TT = 32;
-        while (int64_t(TT) * R < tasks) TT *= 2;
-      }
-      p.TT = TT;
-    } else {
-      p.TT = vq::kQuantRegThreads;
-      p.C = 2;
-      while (int64_t(p.C) * cap < tasks) p.C *= 2;
-    }
-  }
   return true;
 }
 

@@ -30,22 +30,8 @@ struct QuantParams {
   int P;                // warps per unit (1, 2, 4, 8 or 16)
   int WP;               // word-rows per warp of a unit (ceil(W / P))
   int TL;               // lanes per unit when P == 1 (vecs_per_row * rows per load; 32 / TL units per warp)
-  // register-resident kernel (reg == 1): a team of TT threads (8 ... 512) per
-  // unit, or C CTAs of a cluster (TT == 512) for units larger than one CTA holds
-  int reg;
-  int TT;
-  int C;
 };
 
-// Tasks (word-row x 16-byte vector) one thread of the register-resident
-// quantize kernel holds: at most 40 registers of input (R * cpw * 4), so that
-// a second set (the next unit's rows, loaded while this one is encoded) fits;
-// INT2 (16 rows per task, 64 registers) keeps one set.
-__host__ __device__ constexpr int quant_reg_tasks(int bits) {
-  return (32 / bits) >= 16 ? 1 : (10 / (32 / bits) > 1 ? 10 / (32 / bits) : 1);
-}
-constexpr int kQuantRegThreads = 512;
-constexpr int kQuantRegMaxCluster = 16;  // above 8 needs the non-portable cluster size
 
 size_t quant_smem_bytes(int D);
 int quant_warps();
