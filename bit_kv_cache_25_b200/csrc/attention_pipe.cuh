@@ -20,7 +20,7 @@
 // tensor memory over S. The dropped Plo . V^lo term is below 2^-20 of O. The
 // scales live in the operands, so O collects every block directly.
 //
-// Roles of one CTA (one CTA per SM, 448 threads, NQT = 1 or 2 query tiles of
+// Roles of one CTA (one CTA per SM, 512 threads, NQT = 1 or 2 query tiles of
 // 128 rows of one (batch, head) per work item):
 //   one softmax warpgroup per query tile (one query row per thread,
 //     tensor-memory lanes 0-127 of that tile's columns): query load and
@@ -28,17 +28,19 @@
 //     in tensor memory only when a row maximum grows by more than kPipeTau),
 //     normalisation and output. With two query tiles the two warpgroups take
 //     turns on the tensor cores and hide each other's tensor-memory latency;
-//   unpack warps (8 with one query tile, 4 with two): staged packed words ->
+//   unpack warps (8 with one query tile, 6 with two): staged packed words ->
 //     dequantized fp16 hi/lo K and V tiles (ring of NKV slots) shared by the
 //     item's query tiles, and the per-(batch, head) powers of two. With a
 //     two-slot ring (head_dim 128) K and V of a slot are released and refilled
 //     separately: the next K overlaps the PV that still reads this slot's V;
 //   producer warp, one thread: bulk copies of each tile's packed K/V word
 //     rows and of its blocks' scale/zero vectors into a stage ring;
-//   MMA warp, one thread: every tcgen05.mma, with shared-memory descriptors
-//     built once and advanced by constant offsets: QK^T of tile g for each
-//     query tile, then PV of tile g-1 for each (the hi/lo parts of one k-step
-//     back to back).
+//   MMA warp: every tcgen05.mma and commit, issued by one elected lane while
+//     the whole warp runs the (warp-uniform) loop, with shared-memory
+//     descriptors built once and advanced by constant offsets: QK^T of tile g
+//     for each query tile, then PV of tile g-1 for each (the hi/lo parts of one
+//     k-step back to back). At head_dim 64 the QK^T MMAs read q from tensor
+//     memory (written there by the softmax warpgroup), K from shared memory.
 // The CTA is persistent: it walks work items (batch*head, group of NQT query
 // tiles) with a stride of gridDim.x. Every ring runs on across items, so the
 // next item's copies, unpacking and first QK^T overlap this item's last tiles,
@@ -82,7 +84,7 @@ struct PipeCfg {
   static constexpr bool SPLIT_KV = (NKV <= 2);
   static constexpr bool STAGE_Q = (D == 64);               // queries of later items prefetched by cp.async
   static constexpr int QPF = (STAGE_Q && NQT == 1) ? 2 : 1;  // items ahead the query staging runs
-  static constexpr int UNPACK_WARPS = (NQT == 1) ? 8 : 4;
+  static constexpr int UNPACK_WARPS = (NQT == 1) ? 8 : 6;
   static constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
   static constexpr int UNPACK_T0 = NQT * 128;
   static constexpr int PROD_WARP = (NQT * 128 + UNPACK_THREADS) / 32;
@@ -112,7 +114,7 @@ struct PipeCfg {
   static constexpr int NKTAB = TMEM_SLOT + 16;             // kPipeMaxTable x uint8: keys of each tile of an item
   static constexpr int SMEM = NKTAB + kPipeMaxTable;
   static constexpr int SMEM_ALLOC = SMEM + 1024;           // room to align the base
-  static_assert(THREADS == 448, "one CTA per SM at 128 registers per thread");
+  static_assert(THREADS <= 512, "one CTA per SM at 128 registers per thread");
   static_assert(KV0 % 1024 == 0 && TILE_SZ % 1024 == 0 && Q_SZ % 1024 == 0, "operand alignment");
   static_assert(STG0 % 16 == 0 && STG_SZ % 16 == 0 && STG_V % 16 == 0 && STG_META % 16 == 0, "stage alignment");
   static_assert(HDR0 % 16 == 0 && BARS % 8 == 0, "header alignment");
@@ -566,7 +568,8 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             const float* meta =
                 reinterpret_cast<const float*>(stage + C::STG_META) + (i * 4 + 2 * tsel) * D + 8 * jj;
             const float mul = tsel ? vinv : kinv;
-            float sc[8], ze[8];  // scale and zero of the 8 channels, times 2^-e (exact)
+            uint64_t sc2[4], ze2[4];  // scale and zero of the 8 channels, times 2^-e (exact), in pairs
+            const uint64_t kMagic2 = tc::f2pack(8388608.0f, 8388608.0f);
             {
               const uint4 s0 = *reinterpret_cast<const uint4*>(meta + 4 * sw);
               const uint4 s1 = *reinterpret_cast<const uint4*>(meta + 4 * (sw ^ 1));
@@ -577,9 +580,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
               const uint32_t sv8[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
               const uint32_t zv8[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                sc[u] = __uint_as_float(sv8[u]) * mul;
-                ze[u] = __uint_as_float(zv8[u]) * mul;
+              for (int u = 0; u < 4; ++u) {
+                sc2[u] = tc::f2pack(__uint_as_float(sv8[2 * u]) * mul, __uint_as_float(sv8[2 * u + 1]) * mul);
+                ze2[u] = tc::f2pack(__uint_as_float(zv8[2 * u]) * mul, __uint_as_float(zv8[2 * u + 1]) * mul);
               }
             }
             // block token of slot 0 of this word row, and its tile key
@@ -593,20 +596,19 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             for (int s = s_lo; s < s_hi; ++s) {
               const int sh = BITS * s;
               const uint32_t row = static_cast<uint32_t>(kbase + s);
-              float h[8], l[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                // code c as the float 2^23 + c, minus 2^23: exact; then fma(c, scale, zero) * 2^-e
-                const float c = __uint_as_float(((wd[u] >> sh) & C::MASK) | 0x4B000000u) - 8388608.0f;
-                const float x = fmaf(c, sc[u], ze[u]);
-                h[u] = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
-                l[u] = x - h[u];
-              }
               uint32_t hi[4], lo[4];
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
-                hi[u] = tc::cvt_half2(h[2 * u], h[2 * u + 1]);
-                lo[u] = tc::cvt_half2(l[2 * u], l[2 * u + 1]);
+                // codes c as the floats 2^23 + c, minus 2^23 (exact), then
+                // fma(c, scale, zero) * 2^-e, two channels per packed op
+                const uint64_t cb = tc::f2pack(__uint_as_float(((wd[2 * u] >> sh) & C::MASK) | 0x4B000000u),
+                                               __uint_as_float(((wd[2 * u + 1] >> sh) & C::MASK) | 0x4B000000u));
+                const uint64_t x = tc::fma2(tc::sub2(cb, kMagic2), sc2[u], ze2[u]);
+                const float h0 = __uint_as_float(__float_as_uint(tc::f2lo(x)) & 0xffffe000u);
+                const float h1 = __uint_as_float(__float_as_uint(tc::f2hi(x)) & 0xffffe000u);
+                const uint64_t l = tc::sub2(x, tc::f2pack(h0, h1));
+                hi[u] = tc::cvt_half2(h0, h1);
+                lo[u] = tc::cvt_half2(tc::f2lo(l), tc::f2hi(l));
               }
               const uint32_t off = row * 128 + ((oct ^ (row & 7)) << 4);
               tc::sts128(dst + off, hi[0], hi[1], hi[2], hi[3]);
@@ -895,7 +897,8 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           }
           const float up2 = up * kLog2e;
           const float c2 = -m_ref * kLog2e;
-          float rs = 0.0f;
+          const uint64_t up2v = tc::f2pack(up2, up2), c2v = tc::f2pack(c2, c2);
+          uint64_t rs2 = tc::f2pack(0.0f, 0.0f);
           // pass 2: p = 2^(S up log2e - m log2e); hi = p cut to 10 mantissa bits,
           // lo = p - hi; both as fp16 pairs in place over S, 64 keys at a time
 #pragma unroll 1
@@ -905,19 +908,21 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
 #pragma unroll
               for (int c8 = 0; c8 < 64; c8 += 8) {
                 if (c0 + c8 < nk16) {
-                  float ph[8], pl[8];
-#pragma unroll
-                  for (int u = 0; u < 8; ++u) {
-                    const float pv = tc::ex2(fmaf(__uint_as_float(sr[c8 + u]), up2, c2));
-                    ph[u] = __uint_as_float(__float_as_uint(pv) & 0xffffe000u);
-                    pl[u] = pv - ph[u];
-                    rs += pv;
-                  }
                   uint32_t hi[4], lo[4];
 #pragma unroll
                   for (int u = 0; u < 4; ++u) {
-                    hi[u] = tc::cvt_half2(ph[2 * u], ph[2 * u + 1]);
-                    lo[u] = tc::cvt_half2(pl[2 * u], pl[2 * u + 1]);
+                    // two keys per packed op: t = S up log2e - m log2e, p = 2^t,
+                    // hi = p cut to 10 mantissa bits, lo = p - hi
+                    const uint64_t t = tc::fma2(tc::f2pack(__uint_as_float(sr[c8 + 2 * u]),
+                                                           __uint_as_float(sr[c8 + 2 * u + 1])), up2v, c2v);
+                    const float p0 = tc::ex2(tc::f2lo(t)), p1 = tc::ex2(tc::f2hi(t));
+                    const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
+                    const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
+                    const uint64_t pp = tc::f2pack(p0, p1);
+                    const uint64_t l = tc::sub2(pp, tc::f2pack(h0, h1));
+                    rs2 = tc::add2(rs2, pp);
+                    hi[u] = tc::cvt_half2(h0, h1);
+                    lo[u] = tc::cvt_half2(tc::f2lo(l), tc::f2hi(l));
                   }
                   // keys c0+c8..+7: P hi at columns (key / 16) * 16 + (key % 16) / 2, lo 8 further
                   const int key = c0 + c8;
@@ -929,7 +934,7 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             }
           }
           tc::tmem_wait_st();
-          l += rs;
+          l += tc::f2lo(rs2) + tc::f2hi(rs2);
         }
         // the previous item's output, once its last PV is done (before this
         // item's first PV overwrites O)
