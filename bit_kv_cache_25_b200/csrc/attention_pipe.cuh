@@ -906,15 +906,15 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
             if (c0 < nk16) {
               if (KT > 64) load_s64(t_s, c0, nk16, sr, nk);  // (KT == 64: still in sr from pass 1)
 #pragma unroll
-              for (int c8 = 0; c8 < 64; c8 += 8) {
-                if (c0 + c8 < nk16) {
-                  uint32_t hi[4], lo[4];
+              for (int c16 = 0; c16 < 64; c16 += 16) {
+                if (c0 + c16 < nk16) {
+                  uint32_t hi[8], lo[8];
 #pragma unroll
-                  for (int u = 0; u < 4; ++u) {
+                  for (int u = 0; u < 8; ++u) {
                     // two keys per packed op: t = S up log2e - m log2e, p = 2^t,
                     // hi = p cut to 10 mantissa bits, lo = p - hi
-                    const uint64_t t = tc::fma2(tc::f2pack(__uint_as_float(sr[c8 + 2 * u]),
-                                                           __uint_as_float(sr[c8 + 2 * u + 1])), up2v, c2v);
+                    const uint64_t t = tc::fma2(tc::f2pack(__uint_as_float(sr[c16 + 2 * u]),
+                                                           __uint_as_float(sr[c16 + 2 * u + 1])), up2v, c2v);
                     const float p0 = tc::ex2(tc::f2lo(t)), p1 = tc::ex2(tc::f2hi(t));
                     const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
                     const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
@@ -924,11 +924,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
                     hi[u] = tc::cvt_half2(h0, h1);
                     lo[u] = tc::cvt_half2(tc::f2lo(l), tc::f2hi(l));
                   }
-                  // keys c0+c8..+7: P hi at columns (key / 16) * 16 + (key % 16) / 2, lo 8 further
-                  const int key = c0 + c8;
-                  const uint32_t col = (key & ~15) + (key & 15) / 2;
-                  tc::tmem_st4(t_s + col, hi);
-                  tc::tmem_st4(t_s + col + 8, lo);
+                  // keys c0+c16 .. +15: P hi at the 8 columns from c0+c16, lo at the 8 after
+                  tc::tmem_st8(t_s + c0 + c16, hi);
+                  tc::tmem_st8(t_s + c0 + c16 + 8, lo);
                 }
               }
             }
