@@ -12,7 +12,7 @@
 //
 // This file holds the two CUDA-core kernels and the dispatch between them and
 // the tensor-core kernel (attention_pipe.cuh), by measured speed on the VAR
-// and Infinity shapes: at most 4 queries -> attention_small_kernel; up to 64
+// and Infinity shapes: at most 4 queries -> attention_small_kernel; up to 32
 // queries whose keys fit in shared memory -> attention_cc_kernel; the rest ->
 // attention_pipe_kernel (a 128-row MMA tile is mostly padding below that).
 //
@@ -155,7 +155,7 @@ cudaError_t launch_attention_small(const AttnParams& p, cudaStream_t stream) {
 // Largest shared-memory plan; two CTAs per SM at this size (a third would need
 // 3 x (76 + 1) KB, above the 228 KB of an SM), three at 74 KB or less.
 constexpr int kCcMaxSmem = 76 * 1024;
-constexpr int kCcMaxQueries = 64;
+constexpr int kCcMaxQueries = 32;  // from 36 queries on the tensor-core kernel is faster (VAR-d30 block 5)
 
 // Shared-memory plan of one CTA (offsets in floats).
 struct CcLayout {

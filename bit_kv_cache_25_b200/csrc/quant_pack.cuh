@@ -251,6 +251,202 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
   }
 }
 
+// ---- ring variant: the slab of each unit is bulk-copied into a shared-memory
+// slot, so min/max and the encode both read it from shared memory and HBM sees
+// every input byte once. Warp 0 (one lane) is the producer; consumer warp w
+// owns NSLOT slots and takes every RW-th unit of its CTA, one unit per warp,
+// no CTA-wide barrier: full/empty mbarriers per slot, waits bounded.
+template <class Vec, int BITS>
+__global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel(const __grid_constant__ QuantParams p) {
+  constexpr int CPW = 32 / BITS;
+  constexpr int CH = Vec::kCh;
+  constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
+  extern __shared__ __align__(128) unsigned char rsm[];
+  const int RW = p.RW, NS = p.NSLOT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(rsm);        // [RW][NS]
+  uint64_t* empty = full + kRingMaxWarps * 4;               // [RW][NS]
+  unsigned char* slots = rsm + 2 * kRingMaxWarps * 4 * 8;   // [RW][NS][slot_bytes]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = p.B * p.H;
+  const int D = p.D, V = p.vecs_per_row;
+  const int64_t rowb = static_cast<int64_t>(D) * p.esize;   // bytes of one token row
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < RW * NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      for (int k = 0;; ++k) {
+        const int u = blockIdx.x + k * gridDim.x;
+        if (u >= p.units) break;
+        const int w = k % RW, s = (k / RW) % NS, use = k / (RW * NS);
+        const int b = w * NS + s;
+        if (use > 0 && !mbar_wait_bounded(&empty[b], (use - 1) & 1)) break;
+        const QuantTensor& T = p.t[u / BH];
+        const int bh = u % BH;
+        const unsigned char* src =
+            static_cast<const unsigned char*>(T.x) + ((bh / p.H) * T.sb + (bh % p.H) * T.sh) * p.esize;
+        unsigned char* dst = slots + static_cast<size_t>(b) * p.slot_bytes;
+        const uint32_t bytes = static_cast<uint32_t>(p.n * rowb);
+        mbar_arrive_expect_tx(&full[b], bytes);
+        if (T.st * p.esize == rowb) {
+          bulk_copy_g2s(dst, src, bytes, &full[b]);  // contiguous rows: one copy
+        } else {
+          for (int r = 0; r < p.n; ++r)
+            bulk_copy_g2s(dst + r * rowb, src + r * T.st * p.esize, static_cast<uint32_t>(rowb), &full[b]);
+        }
+      }
+    }
+    return;
+  }
+  // ------------------------------------------------------------------ consumers
+  const int cw = warp - 1;
+  if (cw >= RW) return;
+  const int j = lane % V;          // 16-byte channel vector of this lane
+  const int rsub = lane / V;       // row (or word row) offset of this lane
+  const int RL = 32 / V;           // rows (word rows) one warp step covers
+  for (int k = cw;; k += RW) {
+    const int u = blockIdx.x + k * gridDim.x;
+    if (u >= p.units) break;
+    const int s = (k / RW) % NS, use = k / (RW * NS);
+    const int b = cw * NS + s;
+    if (!mbar_wait_bounded(&full[b], use & 1)) break;
+    const unsigned char* slab = slots + static_cast<size_t>(b) * p.slot_bytes + j * 16;
+    const QuantTensor& T = p.t[u / BH];
+    const int bh = u % BH;
+    // pass 1: min/max of this lane's rows, 8 loads in flight
+    uint32_t mn[4], mx[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      mn[q] = Vec::kMnInit;
+      mx[q] = Vec::kMxInit;
+    }
+    for (int r = rsub; r < p.n; r += 8 * RL) {
+      uint4 v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = lds128(slab + min(r + q * RL, p.n - 1) * rowb);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) Vec::minmax_acc(mn, mx, v[q]);  // repeats of row n-1 change nothing
+    }
+    float fmn[CH], fmx[CH];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      fmn[c] = Vec::ch(mn, c);
+      fmx[c] = Vec::ch(mx, c);
+    }
+    for (int off = V; off < 32; off <<= 1) {
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        fmn[c] = fminf(fmn[c], __shfl_xor_sync(0xffffffffu, fmn[c], off));
+        fmx[c] = fmaxf(fmx[c], __shfl_xor_sync(0xffffffffu, fmx[c], off));
+      }
+    }
+    // scale, zero and encode constants (2^64 prescale of tiny scales, see the
+    // streaming kernel)
+    float inv[CH], pre[CH], nmp[CH];
+    bool tiny = false;
+    {
+      float scl[CH], zer[CH];
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), kLevels);
+        zer[c] = __fadd_rn(fmn[c], 0.0f);
+        pre[c] = (scl[c] > 0.0f && scl[c] < 0x1p-100f) ? 0x1p64f : 1.0f;
+        inv[c] = (scl[c] > 0.0f) ? __frcp_rn(__fmul_rn(scl[c], pre[c])) : 0.0f;
+        nmp[c] = __fmul_rn(-fmn[c], pre[c]);
+        tiny |= (pre[c] != 1.0f);
+      }
+      if (rsub == 0) {
+        float* sd = T.scale + static_cast<size_t>(bh) * D + CH * j;
+        float* zd = T.zero + static_cast<size_t>(bh) * D + CH * j;
+#pragma unroll
+        for (int q = 0; q < CH / 4; ++q) {
+          reinterpret_cast<float4*>(sd)[q] = make_float4(scl[4 * q], scl[4 * q + 1], scl[4 * q + 2], scl[4 * q + 3]);
+          reinterpret_cast<float4*>(zd)[q] = make_float4(zer[4 * q], zer[4 * q + 1], zer[4 * q + 2], zer[4 * q + 3]);
+        }
+      }
+    }
+    tiny = __any_sync(0xffffffffu, tiny);
+    // pass 2: word rows of this lane's vector
+    for (int w = rsub; w < p.W; w += RL) {
+      const int t0 = w * CPW;
+      const int nvalid = min(CPW, p.n - t0);
+      uint4 v[CPW];
+#pragma unroll
+      for (int i = 0; i < CPW; ++i) v[i] = lds128(slab + (t0 + min(i, nvalid - 1)) * rowb);
+      uint32_t acc[CH];
+#pragma unroll
+      for (int c = 0; c < CH; ++c) acc[c] = 0u;
+      uint32_t corr = 0u;
+      if (!tiny) {
+#pragma unroll
+        for (int i = 0; i < CPW; ++i) {
+          if (i < nvalid) {
+            corr += kRoundMagicBits << (BITS * i);
+#pragma unroll
+            for (int c = 0; c < CH; ++c) {
+              const float d = __fadd_rn(Vec::elem(v[i], c), nmp[c]);  // = x - min
+              const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
+              acc[c] += __float_as_uint(__fadd_rn(tq, kRoundMagic)) << (BITS * i);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < CPW; ++i) {
+          if (i < nvalid) {
+            corr += kRoundMagicBits << (BITS * i);
+#pragma unroll
+            for (int c = 0; c < CH; ++c) {
+              const float d = __fmaf_rn(Vec::elem(v[i], c), pre[c], nmp[c]);
+              const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
+              acc[c] += __float_as_uint(__fadd_rn(tq, kRoundMagic)) << (BITS * i);
+            }
+          }
+        }
+      }
+      uint32_t* dst = T.packed + (static_cast<size_t>(bh) * p.W + w) * D + CH * j;
+#pragma unroll
+      for (int q = 0; q < CH / 4; ++q)
+        reinterpret_cast<uint4*>(dst)[q] =
+            make_uint4(acc[4 * q] - corr, acc[4 * q + 1] - corr, acc[4 * q + 2] - corr, acc[4 * q + 3] - corr);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[b]);
+  }
+}
+
+size_t quant_ring_smem_bytes(const QuantParams& p) {
+  return static_cast<size_t>(2 * kRingMaxWarps * 4 * 8) + static_cast<size_t>(p.RW) * p.NSLOT * p.slot_bytes;
+}
+
+template <class Vec, int BITS>
+cudaError_t launch_ring(const QuantParams& p, cudaStream_t stream) {
+  auto kern = quant_ring_kernel<Vec, BITS>;
+  static int sm_count[kMaxDevices] = {};
+  static bool configured[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * kRingMaxWarps * 4 * 8 + kRingSmemBudget);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int grid = p.units < sm_count[dev] ? p.units : sm_count[dev];
+  kern<<<grid, 32 * (1 + p.RW), quant_ring_smem_bytes(p), stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <class Vec, int BITS>
 cudaError_t launch_typed(const QuantParams& p, cudaStream_t stream) {
   auto kern = quant_pack_kernel<Vec, BITS>;
@@ -283,8 +479,9 @@ int quant_warps() { return kQuantWarps; }
 
 cudaError_t launch_quant_pack(const QuantParams& p, cudaStream_t stream) {
   const bool bf16 = (p.esize == 2);
-#define VQ_QP_CASE(B)                                                                   \
-  case B:                                                                               \
+#define VQ_QP_CASE(B)                                                                         \
+  case B:                                                                                     \
+    if (p.ring) return bf16 ? launch_ring<Bf16Vec, B>(p, stream) : launch_ring<F32Vec, B>(p, stream); \
     return bf16 ? launch_typed<Bf16Vec, B>(p, stream) : launch_typed<F32Vec, B>(p, stream);
   switch (p.bits) {
     VQ_QP_CASE(2)

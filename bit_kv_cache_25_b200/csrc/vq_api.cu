@@ -105,6 +105,26 @@ bool plan_quant(vq::QuantParams& p) {
   while (rw * kBatch < p.n && rw * p.vecs_per_row < 32) rw *= 2;
   p.TL = (P == 1) ? rw * p.vecs_per_row : 32;
   if (p.TL > 32) p.TL = 32;
+  // Ring kernel for slabs from 8 KB up to half the slot budget: every unit is
+  // bulk-copied into a shared-memory slot and read from there twice. Two slots
+  // per consumer warp while that leaves at least four warps, else one.
+  p.ring = 0;
+  const int64_t slab = int64_t(p.n) * p.D * p.esize;
+  if (slab >= 8192 && slab <= vq::kRingSmemBudget / 2) {
+    int ns = 2;
+    int64_t rwarps = vq::kRingSmemBudget / (2 * slab);
+    if (rwarps < 4) {
+      ns = 1;
+      rwarps = vq::kRingSmemBudget / slab;
+    }
+    if (rwarps > vq::kRingMaxWarps) rwarps = vq::kRingMaxWarps;
+    if (rwarps >= 2) {
+      p.ring = 1;
+      p.RW = static_cast<int>(rwarps);
+      p.NSLOT = ns;
+      p.slot_bytes = static_cast<int>(slab);
+    }
+  }
   return true;
 }
 

@@ -30,7 +30,16 @@ struct QuantParams {
   int P;                // warps per unit (1, 2, 4, 8 or 16)
   int WP;               // word-rows per warp of a unit (ceil(W / P))
   int TL;               // lanes per unit when P == 1 (vecs_per_row * rows per load; 32 / TL units per warp)
+  // ring kernel (ring == 1): each unit's slab is bulk-copied into a shared-memory
+  // slot of slot_bytes; RW consumer warps with NSLOT slots each
+  int ring;
+  int RW;
+  int NSLOT;
+  int slot_bytes;
 };
+
+constexpr int kRingMaxWarps = 12;            // consumer warps per CTA
+constexpr int kRingSmemBudget = 200 * 1024;  // bytes of slots per CTA
 
 
 size_t quant_smem_bytes(int D);

@@ -306,7 +306,8 @@ def test_strided_inputs_and_outputs(vq):
 
 def test_degenerate_groups(vq):
     """Constant channels (scale 0), a zero min stored as +0, a single-token block,
-    and a group whose range is in the float32 subnormal range."""
+    and groups whose range is in the float32 subnormal range (scale below
+    2^-128: the 2^64 prescale path), on both quantize kernels."""
     B, H, D = 1, 1, 64
     sched = [1, 20]
     x = torch.randn((B, H, 21, D), device="cuda", dtype=torch.float32)
@@ -329,6 +330,27 @@ def test_degenerate_groups(vq):
             np.testing.assert_array_equal(zero.cpu().numpy().view(np.uint32), z_ref.reshape(-1).view(np.uint32))
             if n == 1:
                 assert torch.all(scale == 0) and torch.all(packed == 0)
+    # a bf16 block large enough for the shared-memory ring kernel, with a
+    # constant channel and channels whose range is subnormal (bf16 keeps the
+    # float32 exponent range)
+    n = 81
+    xb = torch.randn((B, H, n, D), device="cuda", dtype=torch.float32) * 3
+    xb[..., 5] = -2.0
+    xb[..., 9] = 1e-39 * torch.arange(n, device="cuda", dtype=torch.float32)
+    xb[..., 10] = 2.0 ** -128 * torch.randn(n, device="cuda")
+    xb = xb.to(torch.bfloat16)
+    for bits in (2, 3, 4, 6, 8):
+        desc = vq.CacheDesc(B, H, D, bits, [n])
+        W = desc.word_rows(0)
+        packed = torch.zeros(B * H * W * D, dtype=torch.int32, device="cuda")
+        scale = torch.zeros(B * H * D, device="cuda")
+        zero = torch.zeros(B * H * D, device="cuda")
+        vq.vq_quantize_pack_block(desc, 0, xb, packed, scale, zero)
+        torch.cuda.synchronize()
+        words, s_ref, z_ref = vo.quantize_pack_block(_host(xb), bits)
+        np.testing.assert_array_equal(packed.cpu().numpy().view(np.uint32).reshape(words.shape), words)
+        np.testing.assert_array_equal(scale.cpu().numpy().view(np.uint32), s_ref.reshape(-1).view(np.uint32))
+        np.testing.assert_array_equal(zero.cpu().numpy().view(np.uint32), z_ref.reshape(-1).view(np.uint32))
     assert vq.vq_poll_device_error() == 0
 
 

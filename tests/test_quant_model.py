@@ -74,3 +74,57 @@ def test_quant_plan_small_blocks_share_warps():
     # 16 tokens take 4 units per warp, 25 tokens 2, larger blocks a whole warp
     tl = {n: plan(7680, -(-n // 10), n, 8)[2] for n in (1, 4, 9, 16, 25, 36, 64, 256)}
     assert tl == {1: 8, 4: 8, 9: 8, 16: 8, 25: 16, 36: 32, 64: 32, 256: 32}
+
+
+# ------------------------------------------------------------------ ring kernel
+RING_MAX_WARPS, RING_BUDGET = 12, 200 * 1024
+
+
+def ring_plan(n, D, esize):
+    slab = n * D * esize
+    if not (8192 <= slab <= RING_BUDGET // 2):
+        return None
+    ns, rw = 2, RING_BUDGET // (2 * slab)
+    if rw < 4:
+        ns, rw = 1, RING_BUDGET // slab
+    rw = min(rw, RING_MAX_WARPS)
+    return (rw, ns, slab) if rw >= 2 else None
+
+
+@pytest.mark.parametrize("D,esize", [(64, 2), (128, 2), (64, 4), (128, 4)])
+def test_ring_quant_plan_and_protocol(D, esize):
+    """Ring kernel: the slots fit the shared-memory budget (and the barrier
+    arrays), every unit goes to exactly one consumer warp, and each slot is
+    filled and drained in the same order by its producer and its warp, so the
+    parity of every full/empty wait is the use count of that slot."""
+    ran = 0
+    for n in (16, 36, 64, 100, 144, 169, 256, 300, 400, 576, 800):
+        pl = ring_plan(n, D, esize)
+        if pl is None:
+            continue
+        rw, ns, slab = pl
+        assert 2 <= rw <= RING_MAX_WARPS and ns in (1, 2) and slab % 16 == 0
+        assert rw * ns * slab <= RING_BUDGET and rw * ns <= RING_MAX_WARPS * 4
+        for units, grid in ((7680, 148), (256, 148), (5, 3)):
+            grid = min(grid, units)
+            seen = {}
+            for cta in range(grid):
+                fills = []                     # producer order: (slot, use)
+                k = 0
+                while cta + k * grid < units:
+                    w, s, use = k % rw, (k // rw) % ns, k // (rw * ns)
+                    fills.append((w * ns + s, use, cta + k * grid))
+                    k += 1
+                for w in range(rw):          # consumer w: its own units in order
+                    kk = w
+                    drains = []
+                    while cta + kk * grid < units:
+                        u = cta + kk * grid
+                        assert u not in seen
+                        seen[u] = w
+                        drains.append((w * ns + (kk // rw) % ns, kk // (rw * ns), u))
+                        kk += rw
+                    assert drains == [f for f in fills if f[0] // ns == w]
+            assert len(seen) == units
+            ran += 1
+    assert ran > 0
