@@ -345,6 +345,13 @@ def measure(args, vq, w, bits, world, seed, dev):
     out = torch.empty((B, H, nmax, D), dtype=torch.float32, device=dev)
     outs = [out[:, :, :n] for n in w.block_tokens]
 
+    def enqueue_fused(blocks, layers):
+        for s in blocks:
+            p0, n = w.prefix(s), w.block_tokens[s]
+            for layer in layers:
+                vq.vq_append_attention_block(desc, caches[layer], s, ks[layer][:, :, p0:p0 + n],
+                                             vs[layer][:, :, p0:p0 + n], qs[layer][:, :, p0:p0 + n], sigma, outs[s])
+
     def enqueue(blocks, layers, do_quant=True, do_attn=True):
         for s in blocks:
             p0, n = w.prefix(s), w.block_tokens[s]
@@ -360,6 +367,7 @@ def measure(args, vq, w, bits, world, seed, dev):
     # time the kernels themselves.
     all_blocks, all_layers = range(S), range(L)
     enqueue(all_blocks, all_layers)           # eager warm-up: configures kernel attributes
+    enqueue_fused(all_blocks, all_layers)
     torch.cuda.synchronize()
     cap = torch.cuda.Stream()
     cap.wait_stream(torch.cuda.current_stream())
@@ -369,6 +377,10 @@ def measure(args, vq, w, bits, world, seed, dev):
         with torch.cuda.graph(g, stream=cap):
             enqueue(all_blocks, all_layers)
         graphs["step"] = g
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            enqueue_fused(all_blocks, all_layers)
+        graphs["fused"] = g
         for s in all_blocks:
             for kind in ("quant", "attn"):
                 g = torch.cuda.CUDAGraph()
@@ -405,6 +417,8 @@ def measure(args, vq, w, bits, world, seed, dev):
             graphs["step"].replay()
         stop.record(stream)
         torch.cuda.synchronize()
+        # the same decode through the fused append+attention entry point
+        fused_ms = timed(graphs["fused"], args.steps)
         # per-kernel, per-block times (same replays, each family alone)
         by_block = []
         t_quant = t_attn = 0.0
@@ -461,6 +475,10 @@ def measure(args, vq, w, bits, world, seed, dev):
                       "flops_per_step": a_flops, "bytes_per_step": a_bytes},
         "roofline": rooflines[dominant],
         "roofline_other": rooflines["quant_pack" if dominant == "attention" else "attention"],
+        "fused": {"ms_per_step": fused_ms, "value": weak_scaling_value(tokens_step, world, fused_ms),
+                  "unit": "tokens/s", "launches_per_step": L * sum(1 if n <= 256 else 2 for n in w.block_tokens),
+                  "note": "the same decode through vq_append_attention_block (append and attention in one launch "
+                          "for blocks of at most 256 queries), replayed alone after the timed steps"},
         "clocks": clk.summary(),
         "gpu_launches": 2 * L * S * args.steps,
         "by_block": by_block,
@@ -493,7 +511,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": head["config"],
         "quant_pack": head["quant_pack"], "attention": head["attention"], "roofline": head["roofline"],
-        "roofline_other": head["roofline_other"], "clocks": head["clocks"],
+        "roofline_other": head["roofline_other"], "fused": head["fused"], "clocks": head["clocks"],
         "gpu_launches": sum(r["gpu_launches"] for r in results),
         "timing": "step = one CUDA-graph replay of the whole decode; per-kernel times from graphs of each kernel "
                   "family per block, replayed alone",
@@ -503,7 +521,7 @@ def run_ours(args):
         line["e2e"] = head["e2e"]
     for r in results[1:]:
         line[r["workload"]] = {k: r[k] for k in ("bits", "ms_per_step", "value", "unit", "config", "quant_pack",
-                                                 "attention", "roofline", "roofline_other", "clocks",
+                                                 "attention", "roofline", "roofline_other", "fused", "clocks",
                                                  "gpu_launches", "by_block")}
     if rank == 0 and not args.no_cpu:
         w = WORKLOADS[args.workload]

@@ -54,6 +54,28 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;  // butterfly of commutative adds: identical on every lane
 }
 
+// Fused append: one warp quantizes tensor t (0 = K, 1 = V) of block s for
+// (batch, head) bh into the cache, with the steps of the quantize kernel.
+// (Not inlined: it runs once per CTA, and inlined its registers would crowd
+// the attention loops.)
+template <int BITS>
+__device__ __noinline__ void fused_quantize_unit(const AttnParams& p, int bh, int t, int lane) {
+  const int D = p.D;
+  const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+  const AttnBlockInfo& bi = p.blk[p.s];
+  const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
+  const unsigned char* x = static_cast<const unsigned char*>(t ? p.xv : p.xk);
+  const int64_t sb = t ? p.xv_sb : p.xk_sb, sh = t ? p.xv_sh : p.xk_sh, st = t ? p.xv_st : p.xk_st;
+  const unsigned char* slab = x + (b * sb + h * sh) * p.x_esize;
+  uint32_t* packed = const_cast<uint32_t*>(t ? p.packed_v : p.packed_k) + bi.word_off + static_cast<int64_t>(bh) * bi.W * D;
+  float* scale = const_cast<float*>(t ? p.scale_v : p.scale_k) + p.s * BHD + static_cast<int64_t>(bh) * D;
+  float* zero = const_cast<float*>(t ? p.zero_v : p.zero_k) + p.s * BHD + static_cast<int64_t>(bh) * D;
+  if (p.x_esize == 2)
+    quantize_unit_warp<Bf16Vec, BITS>(slab, st * 2, bi.n, bi.W, D, packed, scale, zero, lane);
+  else
+    quantize_unit_warp<F32Vec, BITS>(slab, st * 4, bi.n, bi.W, D, packed, scale, zero, lane);
+}
+
 template <int BITS, int D>
 __global__ void __launch_bounds__(kSmallWarps * 32) attention_small_kernel(const __grid_constant__ AttnParams p) {
   constexpr int CPW = 32 / BITS;
@@ -65,6 +87,10 @@ __global__ void __launch_bounds__(kSmallWarps * 32) attention_small_kernel(const
   const int b = bh / p.H;
   const int h = bh - b * p.H;
   const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
+  if (p.fused) {  // this CTA's (b, h) of block s into the cache first (warps 0 and 1: K and V)
+    if (warp < 2) fused_quantize_unit<BITS>(p, bh, warp, lane);
+    __syncthreads();
+  }
 
   for (int qi = warp; qi < p.n_q; qi += kSmallWarps) {
     const uint16_t* qrow = p.q + b * p.q_sb + h * p.q_sh + static_cast<int64_t>(qi) * p.q_st;
@@ -82,10 +108,10 @@ __global__ void __launch_bounds__(kSmallWarps * 32) attention_small_kernel(const
 #pragma unroll
       for (int j = 0; j < J; ++j) {
         const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + lane + 32 * j;
-        qp[j] = __fmul_rn(qs[j], p.scale_k[mo]);
-        bias = fmaf(qs[j], p.zero_k[mo], bias);
-        sv[j] = p.scale_v[mo];
-        zv[j] = p.zero_v[mo];
+        qp[j] = __fmul_rn(qs[j], __ldcg(p.scale_k + mo));
+        bias = fmaf(qs[j], __ldcg(p.zero_k + mo), bias);
+        sv[j] = __ldcg(p.scale_v + mo);
+        zv[j] = __ldcg(p.zero_v + mo);
         u[j] = 0.0f;
       }
       bias = warp_sum(bias);
@@ -96,8 +122,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32) attention_small_kernel(const
         uint32_t wk[J], wv[J];
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-          wk[j] = pk[static_cast<int64_t>(w) * D + lane + 32 * j];
-          wv[j] = pv[static_cast<int64_t>(w) * D + lane + 32 * j];
+          wk[j] = __ldcg(pk + static_cast<int64_t>(w) * D + lane + 32 * j);
+          wv[j] = __ldcg(pv + static_cast<int64_t>(w) * D + lane + 32 * j);
         }
         const int nslot = min(CPW, bi.n - w * CPW);
 #pragma unroll
@@ -202,6 +228,10 @@ __global__ void __launch_bounds__(THREADS, 3) attention_cc_kernel(const __grid_c
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
   const int PP = L.PP, NQP = L.NQP, KS = L.KS;
+  if (p.fused) {  // this CTA's (b, h) of block s into the cache first (warps 0 and 1: K and V)
+    if (warp < 2) fused_quantize_unit<BITS>(p, bh, warp, lane);
+    __syncthreads();
+  }
 
   // ---- padding: keys [P, PP) of K^ and V^, rows [n_q, NQP) of q are zero
   for (int e = tid; e < D * (PP - P); e += kCcThreads) {
@@ -249,12 +279,12 @@ __global__ void __launch_bounds__(THREADS, 3) attention_cc_kernel(const __grid_c
         const AttnBlockInfo& bi = p.blk[kb];
         const int64_t off = bi.word_off + static_cast<int64_t>(bh) * bi.W * D + static_cast<int64_t>(w) * D + c;
         const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + c;
-        wk[u] = __ldg(p.packed_k + off);
-        wv[u] = __ldg(p.packed_v + off);
-        sk[u] = __ldg(p.scale_k + mo);
-        zk[u] = __ldg(p.zero_k + mo);
-        sv[u] = __ldg(p.scale_v + mo);
-        zv[u] = __ldg(p.zero_v + mo);
+        wk[u] = __ldcg(p.packed_k + off);
+        wv[u] = __ldcg(p.packed_v + off);
+        sk[u] = __ldcg(p.scale_k + mo);
+        zk[u] = __ldcg(p.zero_k + mo);
+        sv[u] = __ldcg(p.scale_v + mo);
+        zv[u] = __ldcg(p.zero_v + mo);
         j0[u] = key + w * CPW;
         ns[u] = min(CPW, bi.n - w * CPW);
         ch[u] = c;
@@ -404,6 +434,16 @@ namespace {
 // tensor cores. More than 128 queries: two query tiles per work item sharing
 // every dequantized K/V tile; otherwise one query tile per item, the two
 // softmax warpgroups taking the items in turn.
+}  // namespace
+
+// Whether block s's append can run inside its attention launch: every kernel's
+// CTA then quantizes the (batch, head) slabs it attends for, which holds when
+// each (batch, head) is one work item (always for the CUDA-core kernels; up to
+// two 128-row query tiles, i.e. 256 queries, on the tensor cores).
+bool attention_fusable(const AttnParams& p) { return p.n_q <= kSmallMaxQueries || cc_fits(p) || p.n_q <= 256; }
+
+namespace {
+
 template <int BITS, int D>
 cudaError_t launch_attention_typed(const AttnParams& p, cudaStream_t stream) {
   if (p.n_q <= kSmallMaxQueries) return launch_attention_small<BITS, D>(p, stream);

@@ -276,6 +276,16 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  if (p.fused) {
+    // fused append: every warp quantizes units (item, tensor) of this CTA's
+    // items (one item per (batch, head)) into the cache; the fence makes the
+    // stores visible to the bulk copies that read them back
+    const int mine = static_cast<int>(blockIdx.x) < n_items ? (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    for (int u = warp; u < 2 * mine; u += C::THREADS / 32)
+      fused_quantize_unit<BITS>(p, (blockIdx.x + (u >> 1) * gridDim.x) / n_groups, u & 1, lane);
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncthreads();
+  }
 
   if (warp == C::PROD_WARP) {
     // =========================================================== producer thread
@@ -486,10 +496,10 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           if (idx < (p.s + 1) * D) {
             const int kb = idx / D;
             const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + (idx - kb * D);
-            sk[u] = __ldg(p.scale_k + mo);
-            zk[u] = __ldg(p.zero_k + mo);
-            sv[u] = __ldg(p.scale_v + mo);
-            zv[u] = __ldg(p.zero_v + mo);
+            sk[u] = __ldcg(p.scale_k + mo);
+            zk[u] = __ldcg(p.zero_k + mo);
+            sv[u] = __ldcg(p.scale_v + mo);
+            zv[u] = __ldcg(p.zero_v + mo);
           }
         }
 #pragma unroll

@@ -38,6 +38,7 @@
 
 #include <cstdint>
 
+#include "tc_ptx.cuh"
 #include "vq_device.cuh"
 #include "vq_internal.h"
 
@@ -109,6 +110,68 @@ struct F32Vec {
     return __uint_as_float(c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w);
   }
 };
+
+// Channel pair (2k, 2k+1) of a 16-byte vector as two floats (exact widening).
+template <class Vec>
+__device__ __forceinline__ uint64_t vec_pair(const uint4& v, int k) {
+  return tc::f2pack(Vec::elem(v, 2 * k), Vec::elem(v, 2 * k + 1));
+}
+
+// Encode rows 0 .. nvalid-1 of v (one 16-byte channel vector each) into the
+// CH words of one word row, code of row i in bits [BITS*i, BITS*i + BITS).
+// Every step is one IEEE float32 operation per channel: d = x - min (fma(x,
+// pre, -min*pre) when the unit holds a scale below 2^-100), t = d * inv, a
+// clamp to 2^BITS - 1 (only a subnormal scale can push t past it, and such a
+// scale always takes the prescale path), then round half to even by adding
+// 1.5*2^23, whose low mantissa bits are the code. Without a prescale the
+// subtract, multiply and add run on channel pairs as packed .rn operations,
+// each lane rounded on its own exactly like the scalar operation.
+template <class Vec, int BITS, int CPW>
+__device__ __forceinline__ void encode_word_row(const uint4 (&v)[CPW], int nvalid, const float* nmp, const float* inv,
+                                                const float* pre, bool tiny, uint32_t* words) {
+  constexpr int CH = Vec::kCh;
+  constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
+  uint32_t acc[CH];
+#pragma unroll
+  for (int c = 0; c < CH; ++c) acc[c] = 0u;
+  uint32_t corr = 0u;
+  if (!tiny) {
+    uint64_t nm2[CH / 2], iv2[CH / 2];
+#pragma unroll
+    for (int k = 0; k < CH / 2; ++k) {
+      nm2[k] = tc::f2pack(nmp[2 * k], nmp[2 * k + 1]);
+      iv2[k] = tc::f2pack(inv[2 * k], inv[2 * k + 1]);
+    }
+    const uint64_t magic2 = tc::f2pack(kRoundMagic, kRoundMagic);
+#pragma unroll
+    for (int i = 0; i < CPW; ++i) {
+      if (i < nvalid) {
+        corr += kRoundMagicBits << (BITS * i);
+#pragma unroll
+        for (int k = 0; k < CH / 2; ++k) {
+          const uint64_t rq = tc::add2(tc::mul2(tc::add2(vec_pair<Vec>(v[i], k), nm2[k]), iv2[k]), magic2);
+          acc[2 * k] += __float_as_uint(tc::f2lo(rq)) << (BITS * i);
+          acc[2 * k + 1] += __float_as_uint(tc::f2hi(rq)) << (BITS * i);
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < CPW; ++i) {
+      if (i < nvalid) {
+        corr += kRoundMagicBits << (BITS * i);
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const float d = __fmaf_rn(Vec::elem(v[i], c), pre[c], nmp[c]);
+          const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
+          acc[c] += __float_as_uint(__fadd_rn(tq, kRoundMagic)) << (BITS * i);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < CH; ++c) words[c] = acc[c] - corr;
+}
 
 __device__ __forceinline__ uint4 ldg128(const unsigned char* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
@@ -218,6 +281,10 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
         reinterpret_cast<float4*>(zd)[q] = make_float4(zer[4 * q], zer[4 * q + 1], zer[4 * q + 2], zer[4 * q + 3]);
       }
     }
+    bool tiny = false;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) tiny |= (pre[c] != 1.0f);
+    tiny = __any_sync(0xffffffffu, tiny);
     // pass 2: one word-row per lane and vector; every row load issued first
     for (int w = w0 + rsub; w < w1; w += RW) {
       const int tl0 = w * CPW;
@@ -225,28 +292,12 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
       uint4 v[CPW];
 #pragma unroll
       for (int i = 0; i < CPW; ++i) v[i] = ldg128(slab + (tl0 + min(i, nvalid - 1)) * rstride);
-      uint32_t acc[CH];
-#pragma unroll
-      for (int c = 0; c < CH; ++c) acc[c] = 0u;
-      uint32_t corr = 0u;
-#pragma unroll
-      for (int i = 0; i < CPW; ++i) {
-        if (i < nvalid) {
-          corr += kRoundMagicBits << (BITS * i);
-#pragma unroll
-          for (int c = 0; c < CH; ++c) {
-            const float d = __fmaf_rn(Vec::elem(v[i], c), pre[c], nmp[c]);
-            const float t = fminf(__fmul_rn(d, inv[c]), kLevels);
-            const float rq = __fadd_rn(t, kRoundMagic);
-            acc[c] += __float_as_uint(rq) << (BITS * i);
-          }
-        }
-      }
+      uint32_t wd[CH];
+      encode_word_row<Vec, BITS, CPW>(v, nvalid, nmp, inv, pre, tiny, wd);
       uint32_t* dst = T.packed + (static_cast<size_t>(bh) * p.W + w) * D + CH * j;
 #pragma unroll
       for (int q = 0; q < CH / 4; ++q)
-        reinterpret_cast<uint4*>(dst)[q] =
-            make_uint4(acc[4 * q] - corr, acc[4 * q + 1] - corr, acc[4 * q + 2] - corr, acc[4 * q + 3] - corr);
+        reinterpret_cast<uint4*>(dst)[q] = make_uint4(wd[4 * q], wd[4 * q + 1], wd[4 * q + 2], wd[4 * q + 3]);
     }
   }
 }
@@ -379,42 +430,12 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
       uint4 v[CPW];
 #pragma unroll
       for (int i = 0; i < CPW; ++i) v[i] = lds128(slab + (t0 + min(i, nvalid - 1)) * rowb);
-      uint32_t acc[CH];
-#pragma unroll
-      for (int c = 0; c < CH; ++c) acc[c] = 0u;
-      uint32_t corr = 0u;
-      if (!tiny) {
-#pragma unroll
-        for (int i = 0; i < CPW; ++i) {
-          if (i < nvalid) {
-            corr += kRoundMagicBits << (BITS * i);
-#pragma unroll
-            for (int c = 0; c < CH; ++c) {
-              const float d = __fadd_rn(Vec::elem(v[i], c), nmp[c]);  // = x - min
-              const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
-              acc[c] += __float_as_uint(__fadd_rn(tq, kRoundMagic)) << (BITS * i);
-            }
-          }
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < CPW; ++i) {
-          if (i < nvalid) {
-            corr += kRoundMagicBits << (BITS * i);
-#pragma unroll
-            for (int c = 0; c < CH; ++c) {
-              const float d = __fmaf_rn(Vec::elem(v[i], c), pre[c], nmp[c]);
-              const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
-              acc[c] += __float_as_uint(__fadd_rn(tq, kRoundMagic)) << (BITS * i);
-            }
-          }
-        }
-      }
+      uint32_t wd[CH];
+      encode_word_row<Vec, BITS, CPW>(v, nvalid, nmp, inv, pre, tiny, wd);
       uint32_t* dst = T.packed + (static_cast<size_t>(bh) * p.W + w) * D + CH * j;
 #pragma unroll
       for (int q = 0; q < CH / 4; ++q)
-        reinterpret_cast<uint4*>(dst)[q] =
-            make_uint4(acc[4 * q] - corr, acc[4 * q + 1] - corr, acc[4 * q + 2] - corr, acc[4 * q + 3] - corr);
+        reinterpret_cast<uint4*>(dst)[q] = make_uint4(wd[4 * q], wd[4 * q + 1], wd[4 * q + 2], wd[4 * q + 3]);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[b]);
@@ -446,6 +467,87 @@ cudaError_t launch_ring(const QuantParams& p, cudaStream_t stream) {
   kern<<<grid, 32 * (1 + p.RW), quant_ring_smem_bytes(p), stream>>>(p);
   return cudaGetLastError();
 }
+
+}  // namespace
+
+// One warp quantizes one unit (one tensor's n x D slab of one (batch, head)):
+// the streaming kernel's steps with the whole warp on the unit, for the fused
+// append+attention launches, whose CTAs quantize their own (batch, head) before
+// attending. slab: the slab's first row; rstride: bytes between rows; packed:
+// the unit's [W][D] words; scale, zero: its [D] vectors.
+template <class Vec, int BITS>
+__device__ void quantize_unit_warp(const unsigned char* slab, int64_t rstride, int n, int W, int D,
+                                   uint32_t* packed, float* scale, float* zero, int lane) {
+  constexpr int CPW = 32 / BITS;
+  constexpr int CH = Vec::kCh;
+  constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
+  const int V = D / CH;        // 16-byte vectors per row
+  const int RL = 32 / V;       // rows per warp load
+  const int j = lane % V;
+  const int rsub = lane / V;
+  slab += j * 16;
+  uint32_t mn[4], mx[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    mn[k] = Vec::kMnInit;
+    mx[k] = Vec::kMxInit;
+  }
+  for (int r = rsub; r < n; r += kQuantUnroll * RL) {
+    uint4 v[kQuantUnroll];
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) v[u] = ldg128(slab + min(r + u * RL, n - 1) * rstride);
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) Vec::minmax_acc(mn, mx, v[u]);  // repeats of row n-1 change nothing
+  }
+  float fmn[CH], fmx[CH];
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    fmn[c] = Vec::ch(mn, c);
+    fmx[c] = Vec::ch(mx, c);
+  }
+  for (int off = V; off < 32; off <<= 1) {
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      fmn[c] = fminf(fmn[c], __shfl_xor_sync(0xffffffffu, fmn[c], off));
+      fmx[c] = fmaxf(fmx[c], __shfl_xor_sync(0xffffffffu, fmx[c], off));
+    }
+  }
+  float scl[CH], zer[CH], inv[CH], pre[CH], nmp[CH];
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), kLevels);
+    zer[c] = __fadd_rn(fmn[c], 0.0f);
+    pre[c] = (scl[c] > 0.0f && scl[c] < 0x1p-100f) ? 0x1p64f : 1.0f;
+    inv[c] = (scl[c] > 0.0f) ? __frcp_rn(__fmul_rn(scl[c], pre[c])) : 0.0f;
+    nmp[c] = __fmul_rn(-fmn[c], pre[c]);
+  }
+  bool tiny = false;
+#pragma unroll
+  for (int c = 0; c < CH; ++c) tiny |= (pre[c] != 1.0f);
+  tiny = __any_sync(0xffffffffu, tiny);
+  if (rsub == 0) {
+#pragma unroll
+    for (int q = 0; q < CH / 4; ++q) {
+      reinterpret_cast<float4*>(scale + CH * j)[q] = make_float4(scl[4 * q], scl[4 * q + 1], scl[4 * q + 2], scl[4 * q + 3]);
+      reinterpret_cast<float4*>(zero + CH * j)[q] = make_float4(zer[4 * q], zer[4 * q + 1], zer[4 * q + 2], zer[4 * q + 3]);
+    }
+  }
+  for (int w = rsub; w < W; w += RL) {
+    const int t0 = w * CPW;
+    const int nvalid = min(CPW, n - t0);
+    uint4 v[CPW];
+#pragma unroll
+    for (int i = 0; i < CPW; ++i) v[i] = ldg128(slab + (t0 + min(i, nvalid - 1)) * rstride);
+    uint32_t wd[CH];
+    encode_word_row<Vec, BITS, CPW>(v, nvalid, nmp, inv, pre, tiny, wd);
+    uint32_t* dst = packed + static_cast<size_t>(w) * D + CH * j;
+#pragma unroll
+    for (int q = 0; q < CH / 4; ++q)
+      reinterpret_cast<uint4*>(dst)[q] = make_uint4(wd[4 * q], wd[4 * q + 1], wd[4 * q + 2], wd[4 * q + 3]);
+  }
+}
+
+namespace {
 
 template <class Vec, int BITS>
 cudaError_t launch_typed(const QuantParams& p, cudaStream_t stream) {

@@ -15,9 +15,9 @@
 #include "vq_device.cuh"
 #include "vq_internal.h"
 
+#include "quant_pack.cuh"
 #include "attention.cuh"
 #include "dequant.cuh"
-#include "quant_pack.cuh"
 
 namespace {
 
@@ -165,6 +165,55 @@ vq_status launch_quant(const vq_cache_desc* d, int32_t block, vq_dtype dt, int n
   return ok();
 }
 
+// Validates the attention arguments and fills the kernel parameters.
+vq_status build_attention(const vq_cache_desc* desc, const vq_layer_cache* cache, int32_t block, const void* q,
+                          const int64_t q_strides[3], float softmax_scale, void* out, vq_dtype out_dtype,
+                          const int64_t out_strides[3], vq::AttnParams& p) {
+  vq_status st = check_desc(desc);
+  if (st != VQ_OK) return st;
+  if ((st = check_block(desc, block)) != VQ_OK) return st;
+  if (block >= vq::kMaxBlocks) return fail(VQ_ERR_UNSUPPORTED, "attention supports at most %d blocks", vq::kMaxBlocks);
+  if (!cache || !q || !out) return fail(VQ_ERR_INVALID_ARGUMENT, "NULL cache, q or out");
+  if (!cache->packed_k || !cache->packed_v || !cache->scale_k || !cache->zero_k || !cache->scale_v || !cache->zero_v)
+    return fail(VQ_ERR_INVALID_ARGUMENT, "cache has a NULL pointer");
+  if (out_dtype != VQ_F32 && out_dtype != VQ_BF16) return fail(VQ_ERR_UNSUPPORTED, "out dtype unsupported");
+  if (!(softmax_scale > 0.0f) || softmax_scale > 1e6f) return fail(VQ_ERR_INVALID_ARGUMENT, "softmax_scale must be in (0, 1e6]");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(cache->packed_k) || !aligned16(cache->packed_v) ||
+      !aligned16(cache->scale_k) || !aligned16(cache->zero_k) || !aligned16(cache->scale_v) || !aligned16(cache->zero_v))
+    return fail(VQ_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  if ((st = check_strides(q_strides, 2, "q")) != VQ_OK) return st;
+  if ((st = check_strides(out_strides, out_dtype == VQ_F32 ? 4 : 2, "out")) != VQ_OK) return st;
+  p = vq::AttnParams{};
+  p.packed_k = cache->packed_k;
+  p.packed_v = cache->packed_v;
+  p.scale_k = cache->scale_k;
+  p.zero_k = cache->zero_k;
+  p.scale_v = cache->scale_v;
+  p.zero_v = cache->zero_v;
+  p.q = static_cast<const uint16_t*>(q);
+  p.q_sb = q_strides[0];
+  p.q_sh = q_strides[1];
+  p.q_st = q_strides[2];
+  p.out = out;
+  p.o_sb = out_strides[0];
+  p.o_sh = out_strides[1];
+  p.o_st = out_strides[2];
+  p.out_f32 = out_dtype == VQ_F32 ? 1 : 0;
+  p.B = desc->batch;
+  p.H = desc->heads;
+  p.D = desc->head_dim;
+  p.bits = desc->bits;
+  p.s = block;
+  p.n_q = desc->block_tokens[block];
+  p.softmax_scale = softmax_scale;
+  for (int k = 0; k <= block; ++k) {
+    p.blk[k].word_off = block_word_offset(desc, k);
+    p.blk[k].n = desc->block_tokens[k];
+    p.blk[k].W = static_cast<int>(word_rows(desc->block_tokens[k], desc->bits));
+  }
+  return VQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -219,49 +268,51 @@ vq_status vq_cache_append(const vq_cache_desc* desc, const vq_layer_cache* cache
 vq_status vq_attention_block(const vq_cache_desc* desc, const vq_layer_cache* cache, int32_t block, const void* q,
                              const int64_t q_strides[3], float softmax_scale, void* out, vq_dtype out_dtype,
                              const int64_t out_strides[3], void* stream) {
-  vq_status st = check_desc(desc);
-  if (st != VQ_OK) return st;
-  if ((st = check_block(desc, block)) != VQ_OK) return st;
-  if (block >= vq::kMaxBlocks) return fail(VQ_ERR_UNSUPPORTED, "attention supports at most %d blocks", vq::kMaxBlocks);
-  if (!cache || !q || !out) return fail(VQ_ERR_INVALID_ARGUMENT, "NULL cache, q or out");
-  if (!cache->packed_k || !cache->packed_v || !cache->scale_k || !cache->zero_k || !cache->scale_v || !cache->zero_v)
-    return fail(VQ_ERR_INVALID_ARGUMENT, "cache has a NULL pointer");
-  if (out_dtype != VQ_F32 && out_dtype != VQ_BF16) return fail(VQ_ERR_UNSUPPORTED, "out dtype unsupported");
-  if (!(softmax_scale > 0.0f) || softmax_scale > 1e6f) return fail(VQ_ERR_INVALID_ARGUMENT, "softmax_scale must be in (0, 1e6]");
-  if (!aligned16(q) || !aligned16(out) || !aligned16(cache->packed_k) || !aligned16(cache->packed_v) ||
-      !aligned16(cache->scale_k) || !aligned16(cache->zero_k) || !aligned16(cache->scale_v) || !aligned16(cache->zero_v))
-    return fail(VQ_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  if ((st = check_strides(q_strides, 2, "q")) != VQ_OK) return st;
-  if ((st = check_strides(out_strides, out_dtype == VQ_F32 ? 4 : 2, "out")) != VQ_OK) return st;
   vq::AttnParams p{};
-  p.packed_k = cache->packed_k;
-  p.packed_v = cache->packed_v;
-  p.scale_k = cache->scale_k;
-  p.zero_k = cache->zero_k;
-  p.scale_v = cache->scale_v;
-  p.zero_v = cache->zero_v;
-  p.q = static_cast<const uint16_t*>(q);
-  p.q_sb = q_strides[0];
-  p.q_sh = q_strides[1];
-  p.q_st = q_strides[2];
-  p.out = out;
-  p.o_sb = out_strides[0];
-  p.o_sh = out_strides[1];
-  p.o_st = out_strides[2];
-  p.out_f32 = out_dtype == VQ_F32 ? 1 : 0;
-  p.B = desc->batch;
-  p.H = desc->heads;
-  p.D = desc->head_dim;
-  p.bits = desc->bits;
-  p.s = block;
-  p.n_q = desc->block_tokens[block];
-  p.softmax_scale = softmax_scale;
-  for (int k = 0; k <= block; ++k) {
-    p.blk[k].word_off = block_word_offset(desc, k);
-    p.blk[k].n = desc->block_tokens[k];
-    p.blk[k].W = static_cast<int>(word_rows(desc->block_tokens[k], desc->bits));
-  }
+  vq_status st = build_attention(desc, cache, block, q, q_strides, softmax_scale, out, out_dtype, out_strides, p);
+  if (st != VQ_OK) return st;
   cudaError_t e = vq::launch_attention(p, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return ok();
+}
+
+vq_status vq_append_attention_block(const vq_cache_desc* desc, const vq_layer_cache* cache, int32_t block,
+                                    const void* k, const void* v, vq_dtype kv_dtype, const int64_t k_strides[3],
+                                    const int64_t v_strides[3], const void* q, const int64_t q_strides[3],
+                                    float softmax_scale, void* out, vq_dtype out_dtype, const int64_t out_strides[3],
+                                    void* stream) {
+  vq::AttnParams p{};
+  vq_status st = build_attention(desc, cache, block, q, q_strides, softmax_scale, out, out_dtype, out_strides, p);
+  if (st != VQ_OK) return st;
+  if (kv_dtype != VQ_BF16 && kv_dtype != VQ_F32) return fail(VQ_ERR_UNSUPPORTED, "dtype %d unsupported", int(kv_dtype));
+  const int esize = kv_dtype == VQ_BF16 ? 2 : 4;
+  if (!k || !v) return fail(VQ_ERR_INVALID_ARGUMENT, "k/v: NULL pointer");
+  if (!aligned16(k) || !aligned16(v)) return fail(VQ_ERR_MISALIGNED, "k/v: pointers must be 16-byte aligned");
+  if ((st = check_strides(k_strides, esize, "k")) != VQ_OK) return st;
+  if ((st = check_strides(v_strides, esize, "v")) != VQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (vq::attention_fusable(p)) {
+    // one launch: the attention CTAs quantize their own (batch, head) first
+    p.fused = 1;
+    p.x_esize = esize;
+    p.xk = k;
+    p.xv = v;
+    p.xk_sb = k_strides[0];
+    p.xk_sh = k_strides[1];
+    p.xk_st = k_strides[2];
+    p.xv_sb = v_strides[0];
+    p.xv_sh = v_strides[1];
+    p.xv_st = v_strides[2];
+    cudaError_t e = vq::launch_attention(p, s);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "fused append+attention launch");
+    return ok();
+  }
+  // several work items per (batch, head): the append, then the attention
+  st = vq_cache_append(desc, cache, block, k, v, kv_dtype, k_strides, v_strides, stream);
+  if (st != VQ_OK) return st;
+  cudaError_t e = vq::launch_attention(p, s);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return ok();

@@ -81,8 +81,16 @@ struct AttnParams {
   int s;                       // current block
   int n_q;                     // queries (tokens of block s)
   float softmax_scale;
+  // fused append (fused != 0): block s's fresh K and V, which the attention
+  // CTAs quantize into the cache for their own (batch, head) before attending
+  int fused;
+  int x_esize;                 // 2 (bf16) or 4 (float32)
+  const void* xk;
+  const void* xv;
+  int64_t xk_sb, xk_sh, xk_st, xv_sb, xv_sh, xv_st;
   AttnBlockInfo blk[kMaxBlocks];
 };
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t stream);
+bool attention_fusable(const AttnParams& p);
 
 }  // namespace vq

@@ -49,6 +49,8 @@ def _load():
         "vq_quantize_pack_block": [P(vq_cache_desc), I32, VP, I32, I64P, VP, VP, VP, VP],
         "vq_cache_append": [P(vq_cache_desc), P(vq_layer_cache), I32, VP, VP, I32, I64P, I64P, VP],
         "vq_attention_block": [P(vq_cache_desc), P(vq_layer_cache), I32, VP, I64P, F, VP, I32, I64P, VP],
+        "vq_append_attention_block": [P(vq_cache_desc), P(vq_layer_cache), I32, VP, VP, I32, I64P, I64P, VP, I64P, F,
+                                      VP, I32, I64P, VP],
         "vq_dequantize": [P(vq_cache_desc), I32, VP, VP, VP, VP, VP],
         "vq_poll_device_error": [P(ctypes.c_uint32)],
         "vq_status_string": [I32],
@@ -65,7 +67,8 @@ def _load():
 _lib = _load()
 
 EXPORTED = ("vq_cache_layout", "vq_quantize_pack_block", "vq_cache_append", "vq_attention_block",
-            "vq_dequantize", "vq_poll_device_error", "vq_status_string", "vq_last_error", "vq_version")
+            "vq_append_attention_block", "vq_dequantize", "vq_poll_device_error", "vq_status_string",
+            "vq_last_error", "vq_version")
 
 
 def _check(status: int):
@@ -246,6 +249,25 @@ def vq_attention_block(desc: CacheDesc, cache: LayerCache, block: int, q: torch.
     _check(_lib.vq_attention_block(ctypes.byref(desc.c), ctypes.byref(cache.c), block, q.data_ptr(), _strides(q),
                                    ctypes.c_float(softmax_scale), out.data_ptr(), _dtype(out), _strides(out),
                                    _stream(stream)))
+
+
+def vq_append_attention_block(desc: CacheDesc, cache: LayerCache, block: int, k: torch.Tensor, v: torch.Tensor,
+                              q: torch.Tensor, softmax_scale: float, out: torch.Tensor, stream=None):
+    """Append block `block` of K and V ([B][H][n_s][D]) and attend its queries q
+    over blocks 0..block in one call; the same cache and output as
+    vq_cache_append followed by vq_attention_block."""
+    if k.dtype != v.dtype:
+        raise ValueError("k and v must have the same dtype")
+    if q.dtype != torch.bfloat16:
+        raise ValueError("q must be bfloat16")
+    n = _block_tokens(desc, block)
+    for name, t in (("k", k), ("v", v), ("q", q), ("out", out)):
+        _check_slab(name, t, desc, n)
+    _check_devices(("k", k), ("v", v), ("q", q), ("out", out), *_check_cache(desc, cache))
+    _check(_lib.vq_append_attention_block(ctypes.byref(desc.c), ctypes.byref(cache.c), block, k.data_ptr(),
+                                          v.data_ptr(), _dtype(k), _strides(k), _strides(v), q.data_ptr(),
+                                          _strides(q), ctypes.c_float(softmax_scale), out.data_ptr(), _dtype(out),
+                                          _strides(out), _stream(stream)))
 
 
 def vq_dequantize(desc: CacheDesc, block: int, packed: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,

@@ -144,6 +144,24 @@ vq_status vq_attention_block(const vq_cache_desc* desc, const vq_layer_cache* ca
                              float softmax_scale, void* out, vq_dtype out_dtype,
                              const int64_t out_strides[3], void* stream);
 
+/* Append and attend in one call: quantize block `block` of K and V into the
+ * cache (as vq_cache_append) and run that block's attention (as
+ * vq_attention_block). The cache bytes and the output are those of the two
+ * calls in sequence. Block-by-block decoding appends each block just before
+ * its queries attend ("VAR-Q ...", Abstract, paragraph 1; block boundaries
+ * from the generation loop, paragraph 3), so both steps share one launch
+ * wherever the attention has one work item per (batch, head): the attention
+ * CTAs first quantize the slabs of their own (batch, head), then attend, and
+ * the fresh K/V is read from HBM once. That holds for blocks of at most 256
+ * queries; larger blocks run the two launches in order on `stream`. Arguments
+ * are those of vq_cache_append and vq_attention_block, validated the same way
+ * before anything is launched. */
+vq_status vq_append_attention_block(const vq_cache_desc* desc, const vq_layer_cache* cache, int32_t block,
+                                    const void* k, const void* v, vq_dtype kv_dtype,
+                                    const int64_t k_strides[3], const int64_t v_strides[3], const void* q,
+                                    const int64_t q_strides[3], float softmax_scale, void* out,
+                                    vq_dtype out_dtype, const int64_t out_strides[3], void* stream);
+
 /* Check-only: dequantize one packed block, x_hat = fma(code, scale, zero) with
  * one float32 rounding, into out [B][H][n_s][D] (contiguous float32). packed,
  * scale and zero are in the layout written by vq_quantize_pack_block. */

@@ -406,3 +406,76 @@ def test_bf16_output_every_kernel(vq, D):
             assert torch.equal(o32.to(torch.bfloat16), o16), (bits, s, n)
             p0 += n
     assert vq.vq_poll_device_error() == 0
+
+
+# ---------------------------------------------------------------- fused append + attention
+def _fused_decode(vq, desc, cache, sched, k, v, q, sigma, B, H, D, out_dtype=torch.float32):
+    outs = []
+    p0 = 0
+    for s, n in enumerate(sched):
+        out = torch.full((B, H, n, D), float("nan"), dtype=out_dtype, device="cuda")
+        vq.vq_append_attention_block(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n], q[:, :, p0:p0 + n],
+                                     sigma, out)
+        outs.append(out)
+        p0 += n
+    torch.cuda.synchronize()
+    assert vq.vq_poll_device_error() == 0
+    return outs
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_fused_append_attention(vq, D):
+    """vq_append_attention_block block by block: the cache is bit-exact with the
+    oracle's append and every block's attention within the bar of the oracle's
+    attention over it. Blocks of 3, 20, 100 and 200 queries run fused (warp per
+    query, CUDA-core and both tensor-core modes); 300 runs append, then attend."""
+    sched = [3, 20, 100, 200, 300]
+    B, H = 2, 2
+    k, v, q = _ragged_kv(sched, D, H=H, B=B, seed=17)
+    sigma = float(1.0 / np.sqrt(D))
+    for bits in (3, 4, 6):
+        desc = vq.CacheDesc(B, H, D, bits, sched)
+        cache = vq.LayerCache(desc)
+        outs = _fused_decode(vq, desc, cache, sched, k, v, q, sigma, B, H, D)
+        pk, sk, zk = vo.cache_append(_host(k), sched, bits)
+        pv, sv, zv = vo.cache_append(_host(v), sched, bits)
+        np.testing.assert_array_equal(cache.packed_k.cpu().numpy().view(np.uint32), pk)
+        np.testing.assert_array_equal(cache.packed_v.cpu().numpy().view(np.uint32), pv)
+        np.testing.assert_array_equal(cache.scale_k.cpu().numpy().view(np.uint32), sk.view(np.uint32))
+        np.testing.assert_array_equal(cache.zero_v.cpu().numpy().view(np.uint32), zv.view(np.uint32))
+        p0 = 0
+        for s, n in enumerate(sched):
+            khat = vo.dequantize_cache(pk, sk, zk, sched, B, H, D, bits, s)
+            vhat = vo.dequantize_cache(pv, sv, zv, sched, B, H, D, bits, s)
+            ref = vo.attention_f64(_host(q[:, :, p0:p0 + n]), khat, vhat, sigma)
+            err = np.max(np.abs(outs[s].cpu().numpy() - ref)) / np.sqrt(np.mean(ref ** 2))
+            assert err <= ATTN_TOL, (bits, s, n, err)
+            p0 += n
+
+
+def test_fused_matches_two_calls_strided(vq):
+    """Permuted (strided) K/V/Q and output: the fused call leaves the same cache
+    bytes and the same output as vq_cache_append followed by vq_attention_block."""
+    B, H, D, sched, bits = 2, 4, 64, [4, 16, 64, 256], 3
+    N = sum(sched)
+    g = torch.Generator(device="cuda").manual_seed(23)
+    kt = (torch.randn((B, N, H, D), generator=g, device="cuda") * 3).to(torch.bfloat16)
+    vt = torch.randn((B, N, H, D), generator=g, device="cuda").to(torch.bfloat16)
+    qt = torch.randn((B, N, H, D), generator=g, device="cuda").to(torch.bfloat16)
+    k, v, q = kt.permute(0, 2, 1, 3), vt.permute(0, 2, 1, 3), qt.permute(0, 2, 1, 3)
+    desc = vq.CacheDesc(B, H, D, bits, sched)
+    c1, c2 = vq.LayerCache(desc), vq.LayerCache(desc)
+    p0 = 0
+    for s, n in enumerate(sched):
+        o1 = torch.empty((B, n, H, D), dtype=torch.float32, device="cuda").permute(0, 2, 1, 3)
+        o2 = torch.empty((B, H, n, D), dtype=torch.float32, device="cuda")
+        vq.vq_append_attention_block(desc, c1, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n], q[:, :, p0:p0 + n],
+                                     0.125, o1)
+        vq.vq_cache_append(desc, c2, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+        vq.vq_attention_block(desc, c2, s, q[:, :, p0:p0 + n], 0.125, o2)
+        torch.cuda.synchronize()
+        assert torch.equal(c1.packed_k, c2.packed_k) and torch.equal(c1.packed_v, c2.packed_v), s
+        assert torch.equal(c1.scale_k, c2.scale_k) and torch.equal(c1.zero_v, c2.zero_v), s
+        assert torch.equal(o1, o2), s
+        p0 += n
+    assert vq.vq_poll_device_error() == 0
