@@ -124,8 +124,9 @@ __device__ __forceinline__ uint64_t vec_pair(const uint4& v, int k) {
 // clamp to 2^BITS - 1 (only a subnormal scale can push t past it, and such a
 // scale always takes the prescale path), then round half to even by adding
 // 1.5*2^23, whose low mantissa bits are the code. Without a prescale the
-// subtract, multiply and add run on channel pairs as packed .rn operations,
-// each lane rounded on its own exactly like the scalar operation.
+// subtract and the multiply run on channel pairs as packed .rn operations
+// (each lane rounded on its own, like the scalar operation); the rounding add
+// is scalar.
 template <class Vec, int BITS, int CPW>
 __device__ __forceinline__ void encode_word_row(const uint4 (&v)[CPW], int nvalid, const float* nmp, const float* inv,
                                                 const float* pre, bool tiny, uint32_t* words) {
@@ -142,16 +143,18 @@ __device__ __forceinline__ void encode_word_row(const uint4 (&v)[CPW], int nvali
       nm2[k] = tc::f2pack(nmp[2 * k], nmp[2 * k + 1]);
       iv2[k] = tc::f2pack(inv[2 * k], inv[2 * k + 1]);
     }
-    const uint64_t magic2 = tc::f2pack(kRoundMagic, kRoundMagic);
 #pragma unroll
     for (int i = 0; i < CPW; ++i) {
       if (i < nvalid) {
         corr += kRoundMagicBits << (BITS * i);
 #pragma unroll
         for (int k = 0; k < CH / 2; ++k) {
-          const uint64_t rq = tc::add2(tc::mul2(tc::add2(vec_pair<Vec>(v[i], k), nm2[k]), iv2[k]), magic2);
-          acc[2 * k] += __float_as_uint(tc::f2lo(rq)) << (BITS * i);
-          acc[2 * k + 1] += __float_as_uint(tc::f2hi(rq)) << (BITS * i);
+          // packed d = x - min and t = d * inv; the rounding add stays scalar:
+          // a packed multiply followed by a packed add was found contracted
+          // into one rounding (codes differed from the oracle)
+          const uint64_t t = tc::mul2(tc::add2(vec_pair<Vec>(v[i], k), nm2[k]), iv2[k]);
+          acc[2 * k] += __float_as_uint(__fadd_rn(tc::f2lo(t), kRoundMagic)) << (BITS * i);
+          acc[2 * k + 1] += __float_as_uint(__fadd_rn(tc::f2hi(t), kRoundMagic)) << (BITS * i);
         }
       }
     }
