@@ -29,6 +29,10 @@ emulated exactly, and `attention_f64`, which is float64. Function by function:
   dequantize        x_hat = fma(code, scale, zero), one rounding
   attention_f64     softmax(sigma * q . k_hat) . v_hat over blocks 0..s, float64
   paper_kv_gib      KV-memory accounting of the results tables (closed form)
+  scale_zero_fp16   scale and zero rounded to fp16: one 32-bit pair per group
+  paper_*           the storage format those tables count: per block one
+                    padding-free stream of codes over (b, h, token, channel),
+                    floor(32/b) per word, and the 32-bit metadata pairs
 
 Parity status: every function here is pinned by tests that do not re-type its
 formula (brute force on tiny inputs, closed forms, special cases, the printed
@@ -174,16 +178,38 @@ def unpack(words: np.ndarray, bits: int, n_tokens: int) -> np.ndarray:
     return codes
 
 
-def quantize_pack_block(x: np.ndarray, bits: int):
-    """One block of one tensor: float32 [B][H][n][D] -> (words, scale, zero)."""
+def to_fp16(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest fp16 (ties to even), widened back exactly."""
+    return np.asarray(x, dtype=F32).astype(np.float16).astype(F32)
+
+
+def scale_zero_fp16(mn: np.ndarray, mx: np.ndarray, bits: int):
+    """Metadata of one 32-bit (scale, zero) pair per group, the size the results
+    tables count: the float32 scale and zero of `scale_zero`, each rounded to
+    the nearest fp16. Codes are then taken against this stored grid (inputs
+    must stay inside the fp16 range, |x| < 65504)."""
+    scale, zero = scale_zero(mn, mx, bits)
+    return to_fp16(scale), to_fp16(zero)
+
+
+def quantize_pack_block(x: np.ndarray, bits: int, meta_fp16: bool = False):
+    """One block of one tensor: float32 [B][H][n][D] -> (words, scale, zero).
+
+    meta_fp16: scale and zero are the fp16-rounded pair and the codes the
+    nearest levels of that grid, clamped to [0, 2^b - 1] (zero can sit above
+    the min and zero + (2^b - 1) * scale below the max)."""
     x = np.asarray(x, dtype=F32)
     mn, mx = group_min_max(x)
-    scale, zero = scale_zero(mn, mx, bits)
-    codes = encode(x, mn, scale, bits)
+    if meta_fp16:
+        scale, zero = scale_zero_fp16(mn, mx, bits)
+        codes = encode(x, zero, scale, bits)
+    else:
+        scale, zero = scale_zero(mn, mx, bits)
+        codes = encode(x, mn, scale, bits)
     return pack(codes, bits), scale, zero
 
 
-def cache_append(x_layer: np.ndarray, block_tokens, bits: int):
+def cache_append(x_layer: np.ndarray, block_tokens, bits: int, meta_fp16: bool = False):
     """Quantize every block of one layer's tensor [B][H][N][D] into a full cache.
 
     Returns (packed words [words_per_tensor] uint32, scale [S*B*H*D], zero [S*B*H*D])
@@ -197,7 +223,7 @@ def cache_append(x_layer: np.ndarray, block_tokens, bits: int):
     zero = np.zeros(meta, dtype=F32)
     t0 = 0
     for s, n in enumerate(block_tokens):
-        w, sc, z = quantize_pack_block(x_layer[:, :, t0:t0 + n, :], bits)
+        w, sc, z = quantize_pack_block(x_layer[:, :, t0:t0 + n, :], bits, meta_fp16)
         packed[offs[s]:offs[s + 1]] = w.reshape(-1)
         scale[s * B * H * D:(s + 1) * B * H * D] = sc.reshape(-1)
         zero[s * B * H * D:(s + 1) * B * H * D] = z.reshape(-1)
@@ -294,3 +320,62 @@ def paper_kv_gib(layers: int, hidden: int, tokens: int, blocks: int, batch_eff: 
         return elems * 2 / 2**30, None
     bpe = payload_bits(bits) + 32.0 * blocks / tokens
     return elems * bpe / 8 / 2**30, 100.0 * (1.0 - bpe / 16.0)
+
+
+# ---------------------------------------------------------------- paper-exact storage
+def paper_layout(block_tokens, batch: int, heads: int, head_dim: int, bits: int):
+    """Storage the results tables count, for one layer and one tensor.
+
+    Block s is one stream of its B*H*n_s*D codes in (b, h, token, channel)
+    order, code i in word i // cpw at bits [b*(i % cpw), b*(i % cpw) + b): no
+    per-(block, channel) padding, only the last word of the block may hold
+    unused slots. Metadata: one 32-bit word per (block, b, h, channel), fp16
+    scale in the low half, fp16 zero in the high half.
+    Returns (words_per_tensor, meta_words_per_tensor, block_word_offset[S+1]).
+    """
+    cpw = codes_per_word(bits)
+    offs = [0]
+    for n in block_tokens:
+        offs.append(offs[-1] + -(-(batch * heads * n * head_dim) // cpw))
+    return offs[-1], len(block_tokens) * batch * heads * head_dim, offs
+
+
+def paper_pack_block(codes: np.ndarray, bits: int) -> np.ndarray:
+    """Codes [B][H][n][D] of one block -> its padding-free word stream (uint32)."""
+    cpw = codes_per_word(bits)
+    flat = np.asarray(codes, dtype=np.uint32).reshape(-1)
+    nw = -(-flat.size // cpw)
+    padded = np.zeros(nw * cpw, dtype=np.uint32)
+    padded[:flat.size] = flat
+    slots = padded.reshape(nw, cpw)
+    words = np.zeros(nw, dtype=np.uint32)
+    for i in range(cpw):
+        words |= slots[:, i] << np.uint32(bits * i)
+    return words
+
+
+def paper_unpack_block(words: np.ndarray, bits: int, B: int, H: int, n: int, D: int) -> np.ndarray:
+    """Inverse of `paper_pack_block`: the block's stream -> codes [B][H][n][D] (uint8)."""
+    cpw = codes_per_word(bits)
+    mask = np.uint32((1 << bits) - 1)
+    w = np.asarray(words, dtype=np.uint32)
+    slots = np.stack([(w >> np.uint32(bits * i)) & mask for i in range(cpw)], axis=1).reshape(-1)
+    return slots[:B * H * n * D].reshape(B, H, n, D).astype(np.uint8)
+
+
+def paper_meta(scale: np.ndarray, zero: np.ndarray) -> np.ndarray:
+    """fp16 scale in the low 16 bits, fp16 zero in the high 16 bits, per group."""
+    s16 = np.asarray(scale, dtype=F32).astype(np.float16).view(np.uint16).astype(np.uint32)
+    z16 = np.asarray(zero, dtype=F32).astype(np.float16).view(np.uint16).astype(np.uint32)
+    return s16 | (z16 << np.uint32(16))
+
+
+def paper_from_cache(packed, scale, zero, block_tokens, B, H, D, bits):
+    """A layer-tensor cache in the word-row layout -> (paper stream, metadata words)."""
+    _, _, offs = cache_layout(block_tokens, B, H, D, bits)
+    streams = []
+    for s, n in enumerate(block_tokens):
+        W = word_rows(n, bits)
+        codes = unpack(np.asarray(packed[offs[s]:offs[s + 1]]).reshape(B, H, W, D), bits, n)
+        streams.append(paper_pack_block(codes, bits))
+    return np.concatenate(streams), paper_meta(scale, zero)

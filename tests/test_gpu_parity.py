@@ -465,6 +465,9 @@ def test_fused_matches_two_calls_strided(vq):
     k, v, q = kt.permute(0, 2, 1, 3), vt.permute(0, 2, 1, 3), qt.permute(0, 2, 1, 3)
     desc = vq.CacheDesc(B, H, D, bits, sched)
     c1, c2 = vq.LayerCache(desc), vq.LayerCache(desc)
+    for c in (c1, c2):   # blocks not appended yet compare equal too
+        for t in (c.packed_k, c.packed_v, c.scale_k, c.zero_k, c.scale_v, c.zero_v):
+            t.zero_()
     p0 = 0
     for s, n in enumerate(sched):
         o1 = torch.empty((B, n, H, D), dtype=torch.float32, device="cuda").permute(0, 2, 1, 3)

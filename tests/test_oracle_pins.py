@@ -465,3 +465,98 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(vo, "payload_bits", lambda bits: float(bits))
     with pytest.raises(AssertionError):
         check_kv_memory(vo.paper_kv_gib)
+
+
+# ------------------------------------------------------------------ paper-exact storage
+VAR_SCHED = tuple(r * r for r in (1, 2, 3, 4, 5, 6, 8, 10, 13, 16))
+INF_SCHED = tuple(r * r for r in (1, 2, 4, 6, 8, 12, 16, 20, 24, 32, 40, 48, 64))
+# table shape -> (layers, heads, head_dim, schedule)
+PAPER_SHAPES = {"var20": (20, 20, 64, VAR_SCHED), "var24": (24, 24, 64, VAR_SCHED),
+                "var30": (30, 30, 64, VAR_SCHED), "infinity2": (32, 16, 128, INF_SCHED)}
+
+
+def check_paper_layout(paper_layout):
+    """Bytes of the paper storage format for every VAR-Q image row of Tables
+    2a/2b whose model shape is known equal the printed KV GiB and saving."""
+    n = 0
+    for r in _golden_rows():
+        if r["bits"] is None or r["ds"] not in PAPER_SHAPES:
+            continue
+        L, H, D, sched = PAPER_SHAPES[r["ds"]]
+        words, meta, _ = paper_layout(sched, 2 * r["batch"], H, D, r["bits"])
+        gib = L * 2 * (words + meta) * 4 / 2**30
+        assert round(gib, 2) == r["kv"], (r, gib)
+        bf16 = L * 2 * 2 * r["batch"] * H * D * sum(sched) * 2 / 2**30
+        assert round(100 * (1 - gib / bf16), 2) == r["saving"], (r, gib)
+        n += 1
+    assert n == 9   # VAR-d20/d24/d30 INT4 and INT3, Infinity-2B INT8, INT4 and INT3
+
+
+def test_paper_layout_reproduces_printed_kv_memory():
+    check_paper_layout(vo.paper_layout)
+
+
+def test_paper_stream_bit_layout_and_round_trip():
+    rng = np.random.default_rng(11)
+    for bits in (2, 3, 4, 6, 8):
+        cpw = 32 // bits
+        for B, H, n, D in ((1, 1, 1, 4), (2, 3, 5, 8), (1, 2, 7, 6)):
+            codes = rng.integers(0, 1 << bits, size=(B, H, n, D)).astype(np.uint8)
+            words = vo.paper_pack_block(codes, bits)
+            assert words.shape == (-(-(B * H * n * D) // cpw),)
+            np.testing.assert_array_equal(vo.paper_unpack_block(words, bits, B, H, n, D), codes)
+            flat = codes.reshape(-1)
+            for wi, word in enumerate(int(x) for x in words):
+                for pos in range(32):
+                    slot, j = divmod(pos, bits)
+                    i = wi * cpw + slot
+                    want = 0 if (slot >= cpw or i >= flat.size) else (int(flat[i]) >> j) & 1
+                    assert (word >> pos) & 1 == want
+
+
+def check_fp16_metadata_grid(quantize_pack_block, rng):
+    """fp16 metadata: scale and zero are fp16 values (the pair packs into 32
+    bits and unpacks exactly), zero is the min rounded to fp16, and every code
+    is the nearest level of the stored grid, clamped to [0, 2^b - 1]."""
+    for bits in (2, 3, 4, 6, 8):
+        x = _rand_block(rng, 1, 2, 19, 8)
+        words, scale, zero = quantize_pack_block(x, bits, meta_fp16=True)
+        np.testing.assert_array_equal(scale, scale.astype(np.float16).astype(np.float32))
+        np.testing.assert_array_equal(zero, zero.astype(np.float16).astype(np.float32))
+        meta = vo.paper_meta(scale, zero)
+        np.testing.assert_array_equal((meta & 0xffff).astype(np.uint16).view(np.float16).astype(np.float32), scale)
+        np.testing.assert_array_equal((meta >> 16).astype(np.uint16).view(np.float16).astype(np.float32), zero)
+        codes = vo.unpack(words, bits, 19).astype(np.int64)
+        levels = (1 << bits) - 1
+        for h in range(2):
+            for c in range(8):
+                col = [float(v) for v in x[0, h, :, c]]
+                assert float(zero[0, h, c]) == float(np.float16(min(col)))
+                s = Fraction(float(scale[0, h, c]))
+                z = Fraction(float(zero[0, h, c]))
+                for t in range(19):
+                    if s == 0:
+                        assert codes[0, h, t, c] == 0
+                        continue
+                    te = min(max((Fraction(col[t]) - z) / s, Fraction(0)), Fraction(levels))
+                    assert abs(codes[0, h, t, c] - te) <= Fraction(1, 2) + Fraction(1, 2**16), (bits, h, c, t)
+
+
+def test_fp16_metadata_grid():
+    check_fp16_metadata_grid(vo.quantize_pack_block, np.random.default_rng(12))
+
+
+def test_paper_from_cache_matches_per_block_streams():
+    rng = np.random.default_rng(13)
+    sched, B, H, D = (1, 4, 9, 16), 2, 3, 8
+    x = rng.standard_normal((B, H, sum(sched), D)).astype(np.float32) * 5
+    for bits in (3, 4):
+        packed, sc, z = vo.cache_append(x, sched, bits, meta_fp16=True)
+        stream, meta = vo.paper_from_cache(packed, sc, z, sched, B, H, D, bits)
+        words, metaw, offs = vo.paper_layout(sched, B, H, D, bits)
+        assert stream.size == words and meta.size == metaw
+        t0 = 0
+        for s, n in enumerate(sched):
+            codes = vo.unpack(vo.quantize_pack_block(x[:, :, t0:t0 + n], bits, meta_fp16=True)[0], bits, n)
+            np.testing.assert_array_equal(stream[offs[s]:offs[s + 1]], vo.paper_pack_block(codes, bits))
+            t0 += n
