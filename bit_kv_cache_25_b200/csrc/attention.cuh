@@ -71,9 +71,9 @@ __device__ __noinline__ void fused_quantize_unit(const AttnParams& p, int bh, in
   float* scale = const_cast<float*>(t ? p.scale_v : p.scale_k) + p.s * BHD + static_cast<int64_t>(bh) * D;
   float* zero = const_cast<float*>(t ? p.zero_v : p.zero_k) + p.s * BHD + static_cast<int64_t>(bh) * D;
   if (p.x_esize == 2)
-    quantize_unit_warp<Bf16Vec, BITS>(slab, st * 2, bi.n, bi.W, D, packed, scale, zero, lane);
+    quantize_unit_warp<Bf16Vec, BITS>(slab, st * 2, bi.n, bi.W, D, packed, scale, zero, p.meta16 != 0, lane);
   else
-    quantize_unit_warp<F32Vec, BITS>(slab, st * 4, bi.n, bi.W, D, packed, scale, zero, lane);
+    quantize_unit_warp<F32Vec, BITS>(slab, st * 4, bi.n, bi.W, D, packed, scale, zero, p.meta16 != 0, lane);
 }
 
 template <int BITS, int D>

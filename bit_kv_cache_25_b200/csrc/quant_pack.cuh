@@ -34,6 +34,7 @@
 //     into the word with shifts and a final constant correction, then stored
 //     with 128-bit coalesced stores.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -111,6 +112,26 @@ struct F32Vec {
   }
 };
 
+// Scale, zero and encode constants of one group from its exact min and max:
+// scale = (max - min) / (2^bits - 1) and zero = min (+0 for a zero min), each
+// rounded to fp16 when meta16 (one 32-bit metadata pair per group, the codes
+// then taken against that stored grid); pre = 2^64 for a scale below 2^-100
+// (1/scale would overflow from 2^-128 down: d and scale are both multiplied
+// by it, exactly), inv = 1/(scale * pre), nmp = -zero * pre, so that
+// d = fma(x, pre, nmp) = RN(x - zero) * pre.
+__device__ __forceinline__ void group_params(float mn, float mx, float levels, bool meta16, float& scl, float& zer,
+                                             float& inv, float& pre, float& nmp) {
+  scl = __fdiv_rn(__fsub_rn(mx, mn), levels);
+  zer = __fadd_rn(mn, 0.0f);
+  if (meta16) {
+    scl = __half2float(__float2half_rn(scl));
+    zer = __half2float(__float2half_rn(zer));
+  }
+  pre = (scl > 0.0f && scl < 0x1p-100f) ? 0x1p64f : 1.0f;
+  inv = (scl > 0.0f) ? __frcp_rn(__fmul_rn(scl, pre)) : 0.0f;
+  nmp = __fmul_rn(-zer, pre);
+}
+
 // Channel pair (2k, 2k+1) of a 16-byte vector as two floats (exact widening).
 template <class Vec>
 __device__ __forceinline__ uint64_t vec_pair(const uint4& v, int k) {
@@ -119,11 +140,12 @@ __device__ __forceinline__ uint64_t vec_pair(const uint4& v, int k) {
 
 // Encode rows 0 .. nvalid-1 of v (one 16-byte channel vector each) into the
 // CH words of one word row, code of row i in bits [BITS*i, BITS*i + BITS).
-// Every step is one IEEE float32 operation per channel: d = x - min (fma(x,
-// pre, -min*pre) when the unit holds a scale below 2^-100), t = d * inv, a
-// clamp to 2^BITS - 1 (only a subnormal scale can push t past it, and such a
-// scale always takes the prescale path), then round half to even by adding
-// 1.5*2^23, whose low mantissa bits are the code. Without a prescale the
+// Every step is one IEEE float32 operation per channel: d = x - zero
+// (fma(x, pre, -zero*pre) on the slow path), t = d * inv, on the slow path a
+// clamp to [0, 2^BITS - 1], then round half to even by adding 1.5*2^23, whose
+// low mantissa bits are the code. The clamp can act only for a subnormal scale
+// (always behind a prescale) or fp16 metadata (zero rounded above the min);
+// both take the slow path. Without a prescale the
 // subtract and the multiply run on channel pairs as packed .rn operations
 // (each lane rounded on its own, like the scalar operation); the rounding add
 // is scalar.
@@ -166,7 +188,7 @@ __device__ __forceinline__ void encode_word_row(const uint4 (&v)[CPW], int nvali
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
           const float d = __fmaf_rn(Vec::elem(v[i], c), pre[c], nmp[c]);
-          const float tq = fminf(__fmul_rn(d, inv[c]), kLevels);
+          const float tq = fminf(fmaxf(__fmul_rn(d, inv[c]), 0.0f), kLevels);
           acc[c] += __float_as_uint(__fadd_rn(tq, kRoundMagic)) << (BITS * i);
         }
       }
@@ -186,6 +208,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
   constexpr int CH = Vec::kCh;
   constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
   extern __shared__ __align__(16) float qred[];  // [2][groups][P][2][D]
+  const bool META16 = p.meta16 != 0;
   const int D = p.D;
   const int V = p.vecs_per_row;
   const int TL = p.TL;            // lanes per unit (team): a warp takes 32/TL units at once when P == 1
@@ -269,11 +292,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
     float scl[CH], zer[CH], inv[CH], pre[CH], nmp[CH];
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
-      scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), kLevels);
-      zer[c] = __fadd_rn(fmn[c], 0.0f);
-      pre[c] = (scl[c] > 0.0f && scl[c] < 0x1p-100f) ? 0x1p64f : 1.0f;
-      inv[c] = (scl[c] > 0.0f) ? __frcp_rn(__fmul_rn(scl[c], pre[c])) : 0.0f;
-      nmp[c] = __fmul_rn(-fmn[c], pre[c]);
+      group_params(fmn[c], fmx[c], kLevels, META16, scl[c], zer[c], inv[c], pre[c], nmp[c]);
     }
     if (live && part == 0 && rsub == 0) {
       float* sd = T.scale + static_cast<size_t>(bh) * D + CH * j;
@@ -287,7 +306,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
     bool tiny = false;
 #pragma unroll
     for (int c = 0; c < CH; ++c) tiny |= (pre[c] != 1.0f);
-    tiny = __any_sync(0xffffffffu, tiny);
+    tiny = __any_sync(0xffffffffu, tiny) || META16;
     // pass 2: one word-row per lane and vector; every row load issued first
     for (int w = w0 + rsub; w < w1; w += RW) {
       const int tl0 = w * CPW;
@@ -316,6 +335,7 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
   constexpr int CH = Vec::kCh;
   constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
   extern __shared__ __align__(128) unsigned char rsm[];
+  const bool META16 = p.meta16 != 0;
   const int RW = p.RW, NS = p.NSLOT;
   uint64_t* full = reinterpret_cast<uint64_t*>(rsm);        // [RW][NS]
   uint64_t* empty = full + kRingMaxWarps * 4;               // [RW][NS]
@@ -408,11 +428,7 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
       float scl[CH], zer[CH];
 #pragma unroll
       for (int c = 0; c < CH; ++c) {
-        scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), kLevels);
-        zer[c] = __fadd_rn(fmn[c], 0.0f);
-        pre[c] = (scl[c] > 0.0f && scl[c] < 0x1p-100f) ? 0x1p64f : 1.0f;
-        inv[c] = (scl[c] > 0.0f) ? __frcp_rn(__fmul_rn(scl[c], pre[c])) : 0.0f;
-        nmp[c] = __fmul_rn(-fmn[c], pre[c]);
+        group_params(fmn[c], fmx[c], kLevels, META16, scl[c], zer[c], inv[c], pre[c], nmp[c]);
         tiny |= (pre[c] != 1.0f);
       }
       if (rsub == 0) {
@@ -425,7 +441,7 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
         }
       }
     }
-    tiny = __any_sync(0xffffffffu, tiny);
+    tiny = __any_sync(0xffffffffu, tiny) || META16;
     // pass 2: word rows of this lane's vector
     for (int w = rsub; w < p.W; w += RL) {
       const int t0 = w * CPW;
@@ -480,7 +496,7 @@ cudaError_t launch_ring(const QuantParams& p, cudaStream_t stream) {
 // the unit's [W][D] words; scale, zero: its [D] vectors.
 template <class Vec, int BITS>
 __device__ void quantize_unit_warp(const unsigned char* slab, int64_t rstride, int n, int W, int D,
-                                   uint32_t* packed, float* scale, float* zero, int lane) {
+                                   uint32_t* packed, float* scale, float* zero, bool META16, int lane) {
   constexpr int CPW = 32 / BITS;
   constexpr int CH = Vec::kCh;
   constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
@@ -518,16 +534,12 @@ __device__ void quantize_unit_warp(const unsigned char* slab, int64_t rstride, i
   float scl[CH], zer[CH], inv[CH], pre[CH], nmp[CH];
 #pragma unroll
   for (int c = 0; c < CH; ++c) {
-    scl[c] = __fdiv_rn(__fsub_rn(fmx[c], fmn[c]), kLevels);
-    zer[c] = __fadd_rn(fmn[c], 0.0f);
-    pre[c] = (scl[c] > 0.0f && scl[c] < 0x1p-100f) ? 0x1p64f : 1.0f;
-    inv[c] = (scl[c] > 0.0f) ? __frcp_rn(__fmul_rn(scl[c], pre[c])) : 0.0f;
-    nmp[c] = __fmul_rn(-fmn[c], pre[c]);
+    group_params(fmn[c], fmx[c], kLevels, META16, scl[c], zer[c], inv[c], pre[c], nmp[c]);
   }
   bool tiny = false;
 #pragma unroll
   for (int c = 0; c < CH; ++c) tiny |= (pre[c] != 1.0f);
-  tiny = __any_sync(0xffffffffu, tiny);
+  tiny = __any_sync(0xffffffffu, tiny) || META16;
   if (rsub == 0) {
 #pragma unroll
     for (int q = 0; q < CH / 4; ++q) {

@@ -18,6 +18,7 @@
 #include "quant_pack.cuh"
 #include "attention.cuh"
 #include "dequant.cuh"
+#include "paper.cuh"
 
 namespace {
 
@@ -52,6 +53,7 @@ vq_status check_desc(const vq_cache_desc* d) {
   if (d->bits != 2 && d->bits != 3 && d->bits != 4 && d->bits != 6 && d->bits != 8)
     return fail(VQ_ERR_UNSUPPORTED, "bits %d unsupported (2, 3, 4, 6 or 8)", d->bits);
   if (d->num_blocks < 1) return fail(VQ_ERR_INVALID_ARGUMENT, "num_blocks must be >= 1");
+  if (d->meta_fp16 != 0 && d->meta_fp16 != 1) return fail(VQ_ERR_INVALID_ARGUMENT, "meta_fp16 must be 0 or 1");
   if (!d->block_tokens) return fail(VQ_ERR_INVALID_ARGUMENT, "block_tokens is NULL");
   int64_t total = 0;
   for (int s = 0; s < d->num_blocks; ++s) {
@@ -143,6 +145,7 @@ vq_status launch_quant(const vq_cache_desc* d, int32_t block, vq_dtype dt, int n
   p.esize = esize;
   p.vecs_per_row = p.D * esize / 16;
   p.units = ntensors * p.B * p.H;
+  p.meta16 = d->meta_fp16 ? 1 : 0;
   for (int i = 0; i < ntensors; ++i) {
     const char* nm = i == 0 ? "k/x" : "v";
     if (!x[i] || !packed[i] || !scale[i] || !zero[i]) return fail(VQ_ERR_INVALID_ARGUMENT, "%s: NULL pointer", nm);
@@ -206,6 +209,7 @@ vq_status build_attention(const vq_cache_desc* desc, const vq_layer_cache* cache
   p.s = block;
   p.n_q = desc->block_tokens[block];
   p.softmax_scale = softmax_scale;
+  p.meta16 = desc->meta_fp16 ? 1 : 0;
   for (int k = 0; k <= block; ++k) {
     p.blk[k].word_off = block_word_offset(desc, k);
     p.blk[k].n = desc->block_tokens[k];
@@ -340,6 +344,78 @@ vq_status vq_dequantize(const vq_cache_desc* desc, int32_t block, const uint32_t
   cudaError_t e = vq::launch_dequant(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
   return ok();
+}
+
+vq_status vq_paper_layout(const vq_cache_desc* desc, size_t* words_per_tensor, size_t* meta_words_per_tensor,
+                          size_t* block_word_offset_out) {
+  vq_status st = check_desc(desc);
+  if (st != VQ_OK) return st;
+  if (!words_per_tensor || !meta_words_per_tensor) return fail(VQ_ERR_INVALID_ARGUMENT, "output pointers are NULL");
+  const int64_t bhd = int64_t(desc->batch) * desc->heads * desc->head_dim;
+  const int cpw = codes_per_word(desc->bits);
+  int64_t off = 0;
+  for (int s = 0; s <= desc->num_blocks; ++s) {
+    if (block_word_offset_out) block_word_offset_out[s] = static_cast<size_t>(off);
+    if (s < desc->num_blocks) off += (bhd * desc->block_tokens[s] + cpw - 1) / cpw;
+  }
+  *words_per_tensor = static_cast<size_t>(off);
+  *meta_words_per_tensor = static_cast<size_t>(int64_t(desc->num_blocks) * bhd);
+  return ok();
+}
+
+namespace {
+
+vq_status paper_convert(const vq_cache_desc* desc, const vq_layer_cache* cache, bool pack, uint32_t* const words[2],
+                        uint32_t* const meta[2], void* stream) {
+  vq_status st = check_desc(desc);
+  if (st != VQ_OK) return st;
+  if (!cache || !cache->packed_k || !cache->packed_v || !cache->scale_k || !cache->zero_k || !cache->scale_v ||
+      !cache->zero_v)
+    return fail(VQ_ERR_INVALID_ARGUMENT, "NULL cache or cache pointer");
+  for (int t = 0; t < 2; ++t) {
+    if (!words[t] || !meta[t]) return fail(VQ_ERR_INVALID_ARGUMENT, "NULL stream or metadata pointer");
+    if (!aligned16(words[t]) || !aligned16(meta[t])) return fail(VQ_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  }
+  if (!aligned16(cache->packed_k) || !aligned16(cache->packed_v) || !aligned16(cache->scale_k) ||
+      !aligned16(cache->zero_k) || !aligned16(cache->scale_v) || !aligned16(cache->zero_v))
+    return fail(VQ_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t BH = int64_t(desc->batch) * desc->heads;
+  const int cpw = codes_per_word(desc->bits);
+  uint32_t* const rows[2] = {cache->packed_k, cache->packed_v};
+  float* const scale[2] = {cache->scale_k, cache->scale_v};
+  float* const zero[2] = {cache->zero_k, cache->zero_v};
+  for (int t = 0; t < 2; ++t) {
+    int64_t soff = 0;
+    for (int b = 0; b < desc->num_blocks; ++b) {
+      const int n = desc->block_tokens[b];
+      uint32_t* r = rows[t] + block_word_offset(desc, b);
+      cudaError_t e = pack ? vq::launch_paper_block(desc->bits, true, r, words[t] + soff, BH, n, desc->head_dim, s)
+                           : vq::launch_paper_block(desc->bits, false, words[t] + soff, r, BH, n, desc->head_dim, s);
+      if (e != cudaSuccess) return cuda_fail(e, "paper format launch");
+      soff += (BH * desc->head_dim * n + cpw - 1) / cpw;
+    }
+    const int64_t groups = int64_t(desc->num_blocks) * BH * desc->head_dim;
+    cudaError_t e = vq::launch_paper_meta(pack, scale[t], zero[t], meta[t], scale[t], zero[t], groups, s);
+    if (e != cudaSuccess) return cuda_fail(e, "paper metadata launch");
+  }
+  return ok();
+}
+
+}  // namespace
+
+vq_status vq_paper_pack(const vq_cache_desc* desc, const vq_layer_cache* cache, uint32_t* k_words, uint32_t* v_words,
+                        uint32_t* k_meta, uint32_t* v_meta, void* stream) {
+  uint32_t* const w[2] = {k_words, v_words};
+  uint32_t* const m[2] = {k_meta, v_meta};
+  return paper_convert(desc, cache, true, w, m, stream);
+}
+
+vq_status vq_paper_unpack(const vq_cache_desc* desc, const uint32_t* k_words, const uint32_t* v_words,
+                          const uint32_t* k_meta, const uint32_t* v_meta, const vq_layer_cache* cache, void* stream) {
+  uint32_t* const w[2] = {const_cast<uint32_t*>(k_words), const_cast<uint32_t*>(v_words)};
+  uint32_t* const m[2] = {const_cast<uint32_t*>(k_meta), const_cast<uint32_t*>(v_meta)};
+  return paper_convert(desc, cache, false, w, m, stream);
 }
 
 vq_status vq_poll_device_error(uint32_t* code) {

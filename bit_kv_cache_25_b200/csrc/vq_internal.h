@@ -30,6 +30,7 @@ struct QuantParams {
   int P;                // warps per unit (1, 2, 4, 8 or 16)
   int WP;               // word-rows per warp of a unit (ceil(W / P))
   int TL;               // lanes per unit when P == 1 (vecs_per_row * rows per load; 32 / TL units per warp)
+  int meta16;           // scale and zero rounded to fp16, codes against that grid
   // ring kernel (ring == 1): each unit's slab is bulk-copied into a shared-memory
   // slot of slot_bytes; RW consumer warps with NSLOT slots each
   int ring;
@@ -54,6 +55,13 @@ struct DequantParams {
   int B, H, D, n, W, bits;
 };
 cudaError_t launch_dequant(const DequantParams& p, cudaStream_t stream);
+
+// Conversions between the word-row cache and the storage format the results
+// tables count (paper.cuh).
+cudaError_t launch_paper_block(int bits, bool pack, const uint32_t* src, uint32_t* dst, int64_t BH, int n, int D,
+                               cudaStream_t stream);
+cudaError_t launch_paper_meta(bool pack, const float* scale, const float* zero, uint32_t* meta, float* scale_out,
+                              float* zero_out, int64_t n, cudaStream_t stream);
 
 // Attention of one block's queries over the packed cache of blocks 0..s.
 struct AttnBlockInfo {
@@ -84,6 +92,7 @@ struct AttnParams {
   // fused append (fused != 0): block s's fresh K and V, which the attention
   // CTAs quantize into the cache for their own (batch, head) before attending
   int fused;
+  int meta16;                  // the cache's metadata is fp16-valued (quantize against it)
   int x_esize;                 // 2 (bf16) or 4 (float32)
   const void* xk;
   const void* xv;

@@ -29,7 +29,7 @@ class VqError(RuntimeError):
 class vq_cache_desc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("bits", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
-                ("block_tokens", ctypes.POINTER(ctypes.c_int32))]
+                ("block_tokens", ctypes.POINTER(ctypes.c_int32)), ("meta_fp16", ctypes.c_int32)]
 
 
 class vq_layer_cache(ctypes.Structure):
@@ -52,6 +52,9 @@ def _load():
         "vq_append_attention_block": [P(vq_cache_desc), P(vq_layer_cache), I32, VP, VP, I32, I64P, I64P, VP, I64P, F,
                                       VP, I32, I64P, VP],
         "vq_dequantize": [P(vq_cache_desc), I32, VP, VP, VP, VP, VP],
+        "vq_paper_layout": [P(vq_cache_desc), P(SZ), P(SZ), P(SZ)],
+        "vq_paper_pack": [P(vq_cache_desc), P(vq_layer_cache), VP, VP, VP, VP, VP],
+        "vq_paper_unpack": [P(vq_cache_desc), VP, VP, VP, VP, P(vq_layer_cache), VP],
         "vq_poll_device_error": [P(ctypes.c_uint32)],
         "vq_status_string": [I32],
         "vq_last_error": [],
@@ -67,8 +70,8 @@ def _load():
 _lib = _load()
 
 EXPORTED = ("vq_cache_layout", "vq_quantize_pack_block", "vq_cache_append", "vq_attention_block",
-            "vq_append_attention_block", "vq_dequantize", "vq_poll_device_error", "vq_status_string",
-            "vq_last_error", "vq_version")
+            "vq_append_attention_block", "vq_dequantize", "vq_paper_layout", "vq_paper_pack", "vq_paper_unpack",
+            "vq_poll_device_error", "vq_status_string", "vq_last_error", "vq_version")
 
 
 def _check(status: int):
@@ -79,10 +82,11 @@ def _check(status: int):
 class CacheDesc:
     """Host-side vq_cache_desc plus the int32 block schedule it points to."""
 
-    def __init__(self, batch: int, heads: int, head_dim: int, bits: int, block_tokens: Sequence[int]):
+    def __init__(self, batch: int, heads: int, head_dim: int, bits: int, block_tokens: Sequence[int],
+                 meta_fp16: bool = False):
         self.block_tokens = list(int(n) for n in block_tokens)
         self._arr = (ctypes.c_int32 * max(1, len(self.block_tokens)))(*self.block_tokens)
-        self.c = vq_cache_desc(batch, heads, head_dim, bits, len(self.block_tokens), self._arr)
+        self.c = vq_cache_desc(batch, heads, head_dim, bits, len(self.block_tokens), self._arr, int(bool(meta_fp16)))
 
     @property
     def batch(self): return self.c.batch
@@ -98,6 +102,9 @@ class CacheDesc:
 
     @property
     def num_blocks(self): return self.c.num_blocks
+
+    @property
+    def meta_fp16(self): return bool(self.c.meta_fp16)
 
     def word_rows(self, s: int) -> int:
         cpw = 32 // self.bits
@@ -268,6 +275,41 @@ def vq_append_attention_block(desc: CacheDesc, cache: LayerCache, block: int, k:
                                           v.data_ptr(), _dtype(k), _strides(k), _strides(v), q.data_ptr(),
                                           _strides(q), ctypes.c_float(softmax_scale), out.data_ptr(), _dtype(out),
                                           _strides(out), _stream(stream)))
+
+
+def vq_paper_layout(desc: CacheDesc):
+    """-> (words_per_tensor, meta_words_per_tensor, block_word_offset list of S+1) of the storage
+    format the results tables count (one padding-free stream per block, 32-bit metadata pairs)."""
+    w, m = ctypes.c_size_t(), ctypes.c_size_t()
+    offs = (ctypes.c_size_t * (desc.num_blocks + 1))()
+    _check(_lib.vq_paper_layout(ctypes.byref(desc.c), ctypes.byref(w), ctypes.byref(m), offs))
+    return w.value, m.value, list(offs)
+
+
+def vq_paper_pack(desc: CacheDesc, cache: LayerCache, k_words: torch.Tensor, v_words: torch.Tensor,
+                  k_meta: torch.Tensor, v_meta: torch.Tensor, stream=None):
+    """Write the layer cache in the storage format (lossless when desc.meta_fp16)."""
+    words, meta, _ = vq_paper_layout(desc)
+    for name, t, n in (("k_words", k_words, words), ("v_words", v_words, words), ("k_meta", k_meta, meta),
+                       ("v_meta", v_meta, meta)):
+        _check_flat(name, t, n, _WORDS)
+    _check_devices(("k_words", k_words), ("v_words", v_words), ("k_meta", k_meta), ("v_meta", v_meta),
+                   *_check_cache(desc, cache))
+    _check(_lib.vq_paper_pack(ctypes.byref(desc.c), ctypes.byref(cache.c), k_words.data_ptr(), v_words.data_ptr(),
+                              k_meta.data_ptr(), v_meta.data_ptr(), _stream(stream)))
+
+
+def vq_paper_unpack(desc: CacheDesc, k_words: torch.Tensor, v_words: torch.Tensor, k_meta: torch.Tensor,
+                    v_meta: torch.Tensor, cache: LayerCache, stream=None):
+    """Fill the layer cache from the storage format."""
+    words, meta, _ = vq_paper_layout(desc)
+    for name, t, n in (("k_words", k_words, words), ("v_words", v_words, words), ("k_meta", k_meta, meta),
+                       ("v_meta", v_meta, meta)):
+        _check_flat(name, t, n, _WORDS)
+    _check_devices(("k_words", k_words), ("v_words", v_words), ("k_meta", k_meta), ("v_meta", v_meta),
+                   *_check_cache(desc, cache))
+    _check(_lib.vq_paper_unpack(ctypes.byref(desc.c), k_words.data_ptr(), v_words.data_ptr(), k_meta.data_ptr(),
+                                v_meta.data_ptr(), ctypes.byref(cache.c), _stream(stream)))
 
 
 def vq_dequantize(desc: CacheDesc, block: int, packed: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,

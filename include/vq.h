@@ -82,6 +82,13 @@ typedef struct {
   int32_t bits;                /* 2, 3, 4, 6 or 8 */
   int32_t num_blocks;          /* S >= 1: number of blocks (scales) in the schedule */
   const int32_t* block_tokens; /* host array [S]; n_s >= 1 tokens in block s */
+  int32_t meta_fp16;           /* 0: float32 scale and zero; 1: both rounded to fp16 (one
+                                  32-bit pair per group, the size "VAR-Q results data
+                                  (Tables 2-4)", Tables 2a/2b, count) and the codes taken
+                                  against that stored grid, clamped to [0, 2^bits - 1];
+                                  inputs must then stay inside the fp16 range. The cache
+                                  still stores them as float32 (exactly); vq_paper_pack
+                                  writes the 32-bit pairs. */
 } vq_cache_desc;
 
 /* One layer's cache. All device pointers, owned by the caller, sized by
@@ -161,6 +168,33 @@ vq_status vq_append_attention_block(const vq_cache_desc* desc, const vq_layer_ca
                                     const int64_t k_strides[3], const int64_t v_strides[3], const void* q,
                                     const int64_t q_strides[3], float softmax_scale, void* out,
                                     vq_dtype out_dtype, const int64_t out_strides[3], void* stream);
+
+/* Storage format counted by the KV-memory column of "VAR-Q results data
+ * (Tables 2-4)", Tables 2a/2b, for one layer and one tensor: block s is one
+ * padding-free stream of its B*H*n_s*D codes in (b, h, token, channel) order,
+ * floor(32/bits) codes per 32-bit word (code i in word i / cpw, bits
+ * [bits*(i % cpw), bits*(i % cpw) + bits)); the metadata is one 32-bit word per
+ * (block, b, h, channel) group, fp16 scale in the low half and fp16 zero in the
+ * high half. With the tables' shapes and effective batch its size reproduces
+ * every printed VAR-Q image row to the digits shown. `words_per_tensor`: words
+ * of all streams; `meta_words_per_tensor`: S*B*H*D; `block_word_offset` (may be
+ * NULL) receives S+1 offsets. Host only; no CUDA call. */
+vq_status vq_paper_layout(const vq_cache_desc* desc, size_t* words_per_tensor, size_t* meta_words_per_tensor,
+                          size_t* block_word_offset);
+
+/* Write a layer's cache (word-row layout) in the storage format above: k_words,
+ * v_words hold words_per_tensor words each, k_meta, v_meta meta_words_per_tensor
+ * words each (device, caller-owned). The metadata is rounded to fp16, so the
+ * conversion is lossless for a cache quantized with desc->meta_fp16 = 1 (whose
+ * scale and zero are fp16 values) and rounds the metadata otherwise. */
+vq_status vq_paper_pack(const vq_cache_desc* desc, const vq_layer_cache* cache, uint32_t* k_words,
+                        uint32_t* v_words, uint32_t* k_meta, uint32_t* v_meta, void* stream);
+
+/* The inverse: fill a layer's cache (word-row layout, padding slots zero) from
+ * the storage format. */
+vq_status vq_paper_unpack(const vq_cache_desc* desc, const uint32_t* k_words, const uint32_t* v_words,
+                          const uint32_t* k_meta, const uint32_t* v_meta, const vq_layer_cache* cache,
+                          void* stream);
 
 /* Check-only: dequantize one packed block, x_hat = fma(code, scale, zero) with
  * one float32 rounding, into out [B][H][n_s][D] (contiguous float32). packed,

@@ -3,8 +3,11 @@ rejects bad arguments on the host before any CUDA call (no GPU needed)."""
 import ctypes
 import os
 import re
+import sys
 
 import pytest
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))  # the printed-table pins are shared
 
 from bit_kv_cache_25_b200 import vq
 
@@ -97,3 +100,20 @@ def test_launch_without_gpu_reports_cuda_error():
         pytest.skip("a GPU is present")
     d = _desc()
     assert _call_quant(d, 1, BAD, [3 * 30 * 64, 30 * 64, 64]) == vq.VQ_ERR_CUDA
+
+
+def test_paper_layout_through_the_abi_reproduces_printed_kv_memory():
+    """The C entry point's storage format sizes give the printed KV GiB of every
+    VAR-Q image row of Tables 2a/2b (same check as the oracle's pin)."""
+    import test_oracle_pins as pins
+
+    def layout(sched, batch, heads, head_dim, bits):
+        return vq.vq_paper_layout(vq.CacheDesc(batch, heads, head_dim, bits, sched))
+    pins.check_paper_layout(layout)
+
+
+def test_meta_fp16_flag_validated():
+    d = _desc()
+    d.c.meta_fp16 = 2
+    with pytest.raises(vq.VqError):
+        vq.vq_cache_layout(d)

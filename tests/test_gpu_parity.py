@@ -482,3 +482,67 @@ def test_fused_matches_two_calls_strided(vq):
         assert torch.equal(o1, o2), s
         p0 += n
     assert vq.vq_poll_device_error() == 0
+
+
+# ---------------------------------------------------------------- fp16 metadata, storage format
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp16_metadata_and_paper_format(vq, D):
+    """Caches quantized with fp16 metadata: codes and the fp16-valued scale and
+    zero bit-exact with the oracle (streaming, ring and fused quantize paths),
+    attention within the bar over that cache, the storage format written by
+    vq_paper_pack equal to the oracle's, and vq_paper_unpack restoring the
+    word-row cache exactly."""
+    sched = [1, 9, 81, 300]
+    B, H = 2, 2
+    k, v, q = _ragged_kv(sched, D, H=H, B=B, seed=29)
+    sigma = float(1.0 / np.sqrt(D))
+    for bits in (3, 4):
+        desc = vq.CacheDesc(B, H, D, bits, sched, meta_fp16=True)
+        cache = vq.LayerCache(desc)
+        fused = vq.LayerCache(desc)
+        p0 = 0
+        for s, n in enumerate(sched):
+            vq.vq_cache_append(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+            out = torch.empty((B, H, n, D), dtype=torch.float32, device="cuda")
+            vq.vq_append_attention_block(desc, fused, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n],
+                                         q[:, :, p0:p0 + n], sigma, out)
+            p0 += n
+        torch.cuda.synchronize()
+        pk, sk, zk = vo.cache_append(_host(k), sched, bits, meta_fp16=True)
+        pv, sv, zv = vo.cache_append(_host(v), sched, bits, meta_fp16=True)
+        for c in (cache, fused):
+            np.testing.assert_array_equal(c.packed_k.cpu().numpy().view(np.uint32), pk)
+            np.testing.assert_array_equal(c.packed_v.cpu().numpy().view(np.uint32), pv)
+            np.testing.assert_array_equal(c.scale_k.cpu().numpy().view(np.uint32), sk.view(np.uint32))
+            np.testing.assert_array_equal(c.zero_v.cpu().numpy().view(np.uint32), zv.view(np.uint32))
+        p0 = 0
+        for s, n in enumerate(sched):
+            out = torch.empty((B, H, n, D), dtype=torch.float32, device="cuda")
+            vq.vq_attention_block(desc, cache, s, q[:, :, p0:p0 + n], sigma, out)
+            torch.cuda.synchronize()
+            khat = vo.dequantize_cache(pk, sk, zk, sched, B, H, D, bits, s)
+            vhat = vo.dequantize_cache(pv, sv, zv, sched, B, H, D, bits, s)
+            ref = vo.attention_f64(_host(q[:, :, p0:p0 + n]), khat, vhat, sigma)
+            err = np.max(np.abs(out.cpu().numpy() - ref)) / np.sqrt(np.mean(ref ** 2))
+            assert err <= ATTN_TOL, (bits, s, err)
+            p0 += n
+        words, meta, _ = vq.vq_paper_layout(desc)
+        kw = torch.zeros(words, dtype=torch.int32, device="cuda")
+        vw = torch.zeros(words, dtype=torch.int32, device="cuda")
+        km = torch.zeros(meta, dtype=torch.int32, device="cuda")
+        vm = torch.zeros(meta, dtype=torch.int32, device="cuda")
+        vq.vq_paper_pack(desc, cache, kw, vw, km, vm)
+        torch.cuda.synchronize()
+        ref_kw, ref_km = vo.paper_from_cache(pk, sk, zk, sched, B, H, D, bits)
+        ref_vw, ref_vm = vo.paper_from_cache(pv, sv, zv, sched, B, H, D, bits)
+        np.testing.assert_array_equal(kw.cpu().numpy().view(np.uint32), ref_kw)
+        np.testing.assert_array_equal(vw.cpu().numpy().view(np.uint32), ref_vw)
+        np.testing.assert_array_equal(km.cpu().numpy().view(np.uint32), ref_km)
+        np.testing.assert_array_equal(vm.cpu().numpy().view(np.uint32), ref_vm)
+        back = vq.LayerCache(desc)
+        vq.vq_paper_unpack(desc, kw, vw, km, vm, back)
+        torch.cuda.synchronize()
+        for a, b in ((back.packed_k, cache.packed_k), (back.packed_v, cache.packed_v), (back.scale_k, cache.scale_k),
+                     (back.zero_k, cache.zero_k), (back.scale_v, cache.scale_v), (back.zero_v, cache.zero_v)):
+            assert torch.equal(a, b)
+    assert vq.vq_poll_device_error() == 0
