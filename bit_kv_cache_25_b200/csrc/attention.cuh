@@ -87,7 +87,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32) attention_small_kernel(const
   const int b = bh / p.H;
   const int h = bh - b * p.H;
   const int64_t BHD = static_cast<int64_t>(p.B) * p.H * D;
-  if (p.fused) {  // this CTA's (b, h) of block s into the cache first (warps 0 and 1: K and V)
+  if (p.fused) {  // this CTA's (b, h) of block s into the cache first (warps 0 and 1: K and V);
+    // the cache is then read with plain loads, which see the CTA's own writes after the barrier
     if (warp < 2) fused_quantize_unit<BITS>(p, bh, warp, lane);
     __syncthreads();
   }
@@ -108,10 +109,10 @@ __global__ void __launch_bounds__(kSmallWarps * 32) attention_small_kernel(const
 #pragma unroll
       for (int j = 0; j < J; ++j) {
         const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + lane + 32 * j;
-        qp[j] = __fmul_rn(qs[j], __ldcg(p.scale_k + mo));
-        bias = fmaf(qs[j], __ldcg(p.zero_k + mo), bias);
-        sv[j] = __ldcg(p.scale_v + mo);
-        zv[j] = __ldcg(p.zero_v + mo);
+        qp[j] = __fmul_rn(qs[j], p.scale_k[mo]);
+        bias = fmaf(qs[j], p.zero_k[mo], bias);
+        sv[j] = p.scale_v[mo];
+        zv[j] = p.zero_v[mo];
         u[j] = 0.0f;
       }
       bias = warp_sum(bias);
@@ -122,8 +123,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32) attention_small_kernel(const
         uint32_t wk[J], wv[J];
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-          wk[j] = __ldcg(pk + static_cast<int64_t>(w) * D + lane + 32 * j);
-          wv[j] = __ldcg(pv + static_cast<int64_t>(w) * D + lane + 32 * j);
+          wk[j] = pk[static_cast<int64_t>(w) * D + lane + 32 * j];
+          wv[j] = pv[static_cast<int64_t>(w) * D + lane + 32 * j];
         }
         const int nslot = min(CPW, bi.n - w * CPW);
 #pragma unroll
@@ -279,12 +280,14 @@ __global__ void __launch_bounds__(THREADS, 3) attention_cc_kernel(const __grid_c
         const AttnBlockInfo& bi = p.blk[kb];
         const int64_t off = bi.word_off + static_cast<int64_t>(bh) * bi.W * D + static_cast<int64_t>(w) * D + c;
         const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + c;
-        wk[u] = __ldcg(p.packed_k + off);
-        wv[u] = __ldcg(p.packed_v + off);
-        sk[u] = __ldcg(p.scale_k + mo);
-        zk[u] = __ldcg(p.zero_k + mo);
-        sv[u] = __ldcg(p.scale_v + mo);
-        zv[u] = __ldcg(p.zero_v + mo);
+        // plain loads (not the read-only path): with a fused append this CTA
+        // wrote block s's words just before
+        wk[u] = p.packed_k[off];
+        wv[u] = p.packed_v[off];
+        sk[u] = p.scale_k[mo];
+        zk[u] = p.zero_k[mo];
+        sv[u] = p.scale_v[mo];
+        zv[u] = p.zero_v[mo];
         j0[u] = key + w * CPW;
         ns[u] = min(CPW, bi.n - w * CPW);
         ch[u] = c;
