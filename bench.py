@@ -11,7 +11,11 @@ numbers (quantize+pack GB/s, attention tokens/s, roofline fractions) are in
 the `quant_pack` / `attention` / `roofline` keys.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload var_d30] [--bits 3]
+                  [--also infinity_2b|none]   # further workloads, each its own sub-record
   python bench.py --impl reference ...   # the CPU oracle, bounded sample
+
+Each workload also times the same decode through vq_append_attention_block
+(`fused`: append and attention in one launch where possible).
 """
 from __future__ import annotations
 
@@ -48,8 +52,9 @@ def load_peaks():
 # (profiles/dram_traffic.json); valid only while the kernels' sources are the
 # ones that capture ran.
 KERNEL_SOURCES = {
-    "attention": ("attention.cuh", "attention_pipe.cuh", "tc_ptx.cuh", "vq_device.cuh", "vq_api.cu"),
-    "quant_pack": ("quant_pack.cuh", "vq_device.cuh", "vq_api.cu"),
+    "attention": ("attention.cuh", "attention_pipe.cuh", "quant_pack.cuh", "tc_ptx.cuh", "vq_device.cuh",
+                  "vq_internal.h", "vq_api.cu"),
+    "quant_pack": ("quant_pack.cuh", "tc_ptx.cuh", "vq_device.cuh", "vq_internal.h", "vq_api.cu"),
 }
 
 
