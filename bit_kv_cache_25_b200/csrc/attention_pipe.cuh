@@ -9,16 +9,21 @@
 // dequantized in shared memory to the cache's own fp32 values
 // x^ = fma(code, scale, zero) of each token's block, times a power of two 2^-e
 // chosen per (batch, head) so that the largest |x^| over blocks 0..s lies in
-// [2^14, 2^15), and split into two fp16 parts: hi = x^ with its mantissa cut to
-// 10 bits (exact in fp16), lo = x^ - hi rounded to fp16, so
-// hi + lo = x^ (1 + O(2^-21)). The bf16 queries are exact in fp16 after a
+// [2^14, 2^15), and split into two 16-bit parts. K, whose rounding moves every
+// logit, takes fp16: hi = x^ with its mantissa cut to 10 bits (exact in fp16),
+// lo = x^ - hi rounded to fp16, so hi + lo = x^ (1 + O(2^-21)). V takes bf16,
+// as P does: hi = x^ rounded to bf16, lo = x^ - hi rounded to bf16, so
+// hi + lo = x^ (1 + O(2^-16)). The bf16 queries are exact in fp16 after a
 // power-of-two scale per row. Per tile, for the 128 query rows of a work item,
 // all accumulation in fp32:
-//   S  = q . (K^hi + K^lo)^T                      2 MMAs per 16-wide k-step
-//   O += Phi . V^hi + Plo . V^hi + Phi . V^lo     3 MMAs per 16-key step
-// with P = exp(logit - m) split the same way into fp16 hi/lo and written to
-// tensor memory over S. The dropped Plo . V^lo term is below 2^-20 of O. The
-// scales live in the operands, so O collects every block directly.
+//   S  = q . (K^hi + K^lo)^T                      2 fp16 MMAs per 16-wide k-step
+//   O += Phi . V^hi + Plo . V^hi + Phi . V^lo     3 bf16 MMAs per 16-key step
+// with P = exp(logit - m) split into bf16 hi/lo and written to tensor memory
+// over S. The dropped Plo . V^lo term is below 2^-16 of each product. bf16
+// has the range of fp32, so P may sit far above its reference maximum without
+// overflowing: O is rescaled only when a row maximum grows by more than
+// kPipeTau = 40 (natural-log units), which the data essentially never does.
+// The scales live in the operands, so O collects every block directly.
 //
 // Roles of one CTA (one CTA per SM, 512 threads, NQT = 1 or 2 query tiles of
 // 128 rows of one (batch, head) per work item):
@@ -29,7 +34,7 @@
 //     normalisation and output. With two query tiles the two warpgroups take
 //     turns on the tensor cores and hide each other's tensor-memory latency;
 //   unpack warps (8 with one query tile, 6 with two): staged packed words ->
-//     dequantized fp16 hi/lo K and V tiles (ring of NKV slots) shared by the
+//     dequantized hi/lo K (fp16) and V (bf16) tiles (ring of NKV slots) shared by the
 //     item's query tiles, and the per-(batch, head) powers of two. With a
 //     two-slot ring (head_dim 128) K and V of a slot are released and refilled
 //     separately: the next K overlaps the PV that still reads this slot's V;
@@ -59,7 +64,9 @@
 namespace vq {
 namespace {
 
-constexpr float kPipeTau = 10.5f;  // lazy-rescale threshold (natural-log units): p <= e^10.5 < 2^16 fits fp16
+// lazy-rescale threshold (natural-log units): p <= e^40 < 2^58 as bf16, and
+// O <= 2^15 * e^40 * (2^15 keys) stays far below the fp32 maximum
+constexpr float kPipeTau = 40.0f;
 constexpr float kPipeHead = 2.5f;  // an item's first reference maximum sits this far above its first tile's
 constexpr int kPipeMaxTable = 4096;  // tiles per item whose key counts are tabled in shared memory
 
@@ -86,14 +93,24 @@ struct PipeCfg {
   static constexpr int QPF = (STAGE_Q && NQT == 1) ? 2 : 1;  // items ahead the query staging runs
   static constexpr int UNPACK_WARPS = (NQT == 1) ? 8 : 6;
   static constexpr int UNPACK_THREADS = UNPACK_WARPS * 32;
-  static constexpr int UNPACK_T0 = NQT * 128;
-  static constexpr int PROD_WARP = (NQT * 128 + UNPACK_THREADS) / 32;
+  // Warp roles: softmax warps 0 .. 4 NQT - 1 (warp w reads tensor-memory lanes
+  // 32 (w % 4) ..), then the unpack warps, the producer and the MMA warp. (With
+  // the MMA warp and the producer moved next to the softmax warps only, the
+  // MMA issue was no faster: the tensor pipe itself takes 68-93 cycles per
+  // M=128, K=16 MMA of N <= 128, and the unpack warps lost a sub-partition.)
+  static constexpr int SOFTMAX_WARPS = 4 * NQT;
+  static constexpr int UNPACK_T0 = SOFTMAX_WARPS * 32;
+  static constexpr int PROD_WARP = SOFTMAX_WARPS + UNPACK_WARPS;
   static constexpr int MMA_WARP = PROD_WARP + 1;
   static constexpr int THREADS = (MMA_WARP + 1) * 32;
+  // index of warp w among the unpack warps, -1 for the other roles
+  static __host__ __device__ constexpr int unpack_index(int w) {
+    return (w < SOFTMAX_WARPS || w >= PROD_WARP) ? -1 : w - SOFTMAX_WARPS;
+  }
   // ---- shared memory (byte offsets from a 1024-aligned base)
   static constexpr int Q_SZ = Q_TMEM ? 0 : 128 * D * 2;    // fp16 q [128][D] per query tile, K-major SW128
   static constexpr int Q0 = 0;
-  static constexpr int TILE_SZ = KT * D * 2;               // fp16 [KT][D], K-major SW128
+  static constexpr int TILE_SZ = KT * D * 2;               // 16-bit [KT][D], K-major SW128
   static constexpr int KV0 = Q0 + NQT * Q_SZ;              // NKV x {K hi, K lo, V hi, V lo}
   static constexpr int KV_SZ = 4 * TILE_SZ;
   static constexpr int QST0 = KV0 + NKV * KV_SZ;           // QPF x bf16 [128][D] query staging per query tile
@@ -265,10 +282,11 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     }
     fence_barrier_init();
   }
-  if (tid >= C::UNPACK_T0 && tid < C::UNPACK_T0 + C::UNPACK_THREADS) {
+  if (C::unpack_index(warp) >= 0) {
     // key rows past a tile's valid keys are read by the MMAs (times zero
     // probabilities) and must hold finite values
-    for (int i = C::KV0 + (tid - C::UNPACK_T0) * 16; i < C::KV0 + NKV * C::KV_SZ; i += C::UNPACK_THREADS * 16)
+    for (int i = C::KV0 + (C::unpack_index(warp) * 32 + lane) * 16; i < C::KV0 + NKV * C::KV_SZ;
+         i += C::UNPACK_THREADS * 16)
       tc::sts128(sbase + i, 0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
@@ -276,6 +294,11 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  // The CTA holds all 512 columns (one CTA per SM), so its allocation starts
+  // at lane 0, column 0: the MMA warp then uses constant tensor-memory
+  // addresses. Anything else is recorded and every role skips its work.
+  const bool tmem_at_zero = (tmem == 0u);
+  if (!tmem_at_zero && tid == 0) atomicOr(&g_device_error, kDevErrBadShape);
   if (p.fused) {
     // fused append: every warp quantizes units (item, tensor) of this CTA's
     // items (one item per (batch, head)) into the cache; the fence makes the
@@ -287,7 +310,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     __syncthreads();
   }
 
-  if (warp == C::PROD_WARP) {
+  if (!tmem_at_zero) {
+    // (recorded above: straight to the teardown)
+  } else if (warp == C::PROD_WARP) {
     // =========================================================== producer thread
     if (lane == 0) {
       bool ok = true;
@@ -341,9 +366,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     // elected lane issues each tcgen05 instruction. With a single thread
     // running it, consecutive MMAs issued 85-110 cycles apart in the kernel.
     {
-      const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+      constexpr uint32_t tm = 0u;  // tensor-memory base (checked at set-up)
       constexpr uint32_t kLbo = KT * 128;  // 64-channel groups of a [KT][D] V tile read MN-major
-      const uint32_t idesc_pv = tc::idesc_f16_f32(128, D, /*b_mn_major=*/true);
+      const uint32_t idesc_pv = tc::idesc_f16_f32(128, D, /*b_mn_major=*/true, /*bf16=*/true);
       const uint64_t qdesc = tc::sw128_desc(sbase + C::Q0);
       const uint64_t kdesc0 = tc::sw128_desc(sbase + C::KV0);
       const uint64_t vdesc0 = tc::sw128_desc_mn(sbase + C::KV0 + 2 * C::TILE_SZ, kLbo);
@@ -473,9 +498,9 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
         if (ok) tc::commit_warp(&v_empty[prev_kvs]);
       }
     }
-  } else if (tid >= C::UNPACK_T0) {
+  } else if (warp >= C::SOFTMAX_WARPS) {
     // =========================================================== unpack warps
-    const int ut = tid - C::UNPACK_T0;
+    const int ut = C::unpack_index(warp) * 32 + lane;
     const float cmax = static_cast<float>(C::MASK);
     // Powers of two of the k-th item of this CTA: max |x^| over blocks 0..s.
     // Each warp reduces its share of the scale/zero vectors and posts its
@@ -614,11 +639,20 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
                 const uint64_t cb = tc::f2pack(__uint_as_float(((wd[2 * u] >> sh) & C::MASK) | 0x4B000000u),
                                                __uint_as_float(((wd[2 * u + 1] >> sh) & C::MASK) | 0x4B000000u));
                 const uint64_t x = tc::fma2(tc::sub2(cb, kMagic2), sc2[u], ze2[u]);
-                const float h0 = __uint_as_float(__float_as_uint(tc::f2lo(x)) & 0xffffe000u);
-                const float h1 = __uint_as_float(__float_as_uint(tc::f2hi(x)) & 0xffffe000u);
-                const uint64_t l = tc::sub2(x, tc::f2pack(h0, h1));
-                hi[u] = tc::cvt_half2(h0, h1);
-                lo[u] = tc::cvt_half2(tc::f2lo(l), tc::f2hi(l));
+                if (tsel) {
+                  // V: bf16 hi rounded to nearest, lo = x - hi (exact in fp32) rounded
+                  const uint32_t hb = tc::cvt_bf162(tc::f2lo(x), tc::f2hi(x));
+                  const uint64_t l = tc::sub2(x, tc::bf162_to_f2(hb));
+                  hi[u] = hb;
+                  lo[u] = tc::cvt_bf162(tc::f2lo(l), tc::f2hi(l));
+                } else {
+                  // K: fp16 hi = x cut to 10 mantissa bits, lo = x - hi rounded
+                  const float h0 = __uint_as_float(__float_as_uint(tc::f2lo(x)) & 0xffffe000u);
+                  const float h1 = __uint_as_float(__float_as_uint(tc::f2hi(x)) & 0xffffe000u);
+                  const uint64_t l = tc::sub2(x, tc::f2pack(h0, h1));
+                  hi[u] = tc::cvt_half2(h0, h1);
+                  lo[u] = tc::cvt_half2(tc::f2lo(l), tc::f2hi(l));
+                }
               }
               const uint32_t off = row * 128 + ((oct ^ (row & 7)) << 4);
               tc::sts128(dst + off, hi[0], hi[1], hi[2], hi[3]);
@@ -770,36 +804,42 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
       const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
       const int64_t obase = b * p.o_sb + h * p.o_sh + static_cast<int64_t>(r) * p.o_st;
       const float scl = vmul / l;
+      // 32 columns per round: two loads in flight, one wait
 #pragma unroll 1
-      for (int c16 = 0; c16 < D; c16 += 16) {
-        uint32_t o[16];
-        tc::tmem_ld16(tq + C::COL_O + c16, o);
+      for (int c32 = 0; c32 < D; c32 += 32) {
+        uint32_t o[32];
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          tc::tmem_ld16(tq + C::COL_O + c32 + 16 * k, *reinterpret_cast<uint32_t(*)[16]>(&o[16 * k]));
         tc::tmem_wait_ld();
         if (!valid) continue;
         if (p.out_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + c16);
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + c32);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
+          for (int k = 0; k < 8; ++k)
             dst[k] = make_float4(__uint_as_float(o[4 * k]) * scl, __uint_as_float(o[4 * k + 1]) * scl,
                                  __uint_as_float(o[4 * k + 2]) * scl, __uint_as_float(o[4 * k + 3]) * scl);
         } else {
-          uint32_t bf[8];
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + obase + c32);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            uint32_t pair = 0;
+          for (int q = 0; q < 4; ++q) {
+            uint32_t bf[4];
 #pragma unroll
-            for (int uu = 0; uu < 2; ++uu) {
-              const uint32_t x = __float_as_uint(__uint_as_float(o[2 * k + uu]) * scl);
-              pair |= ((x + 0x7fffu + ((x >> 16) & 1u)) >> 16) << (16 * uu);
+            for (int k = 0; k < 4; ++k) {
+              uint32_t pair = 0;
+#pragma unroll
+              for (int uu = 0; uu < 2; ++uu) {
+                const uint32_t x = __float_as_uint(__uint_as_float(o[8 * q + 2 * k + uu]) * scl);
+                pair |= ((x + 0x7fffu + ((x >> 16) & 1u)) >> 16) << (16 * uu);
+              }
+              bf[k] = pair;
             }
-            bf[k] = pair;
+            dst[q] = make_uint4(bf[0], bf[1], bf[2], bf[3]);
           }
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + obase + c16);
-          dst[0] = make_uint4(bf[0], bf[1], bf[2], bf[3]);
-          dst[1] = make_uint4(bf[4], bf[5], bf[6], bf[7]);
         }
       }
     };
+    // (rare: runs while the tile's S is held in registers, so 16 columns at a time)
     auto scale_o = [&](float alpha) {
 #pragma unroll 1
       for (int c16 = 0; c16 < D; c16 += 16) {
@@ -909,8 +949,8 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
           const float c2 = -m_ref * kLog2e;
           const uint64_t up2v = tc::f2pack(up2, up2), c2v = tc::f2pack(c2, c2);
           uint64_t rs2 = tc::f2pack(0.0f, 0.0f);
-          // pass 2: p = 2^(S up log2e - m log2e); hi = p cut to 10 mantissa bits,
-          // lo = p - hi; both as fp16 pairs in place over S, 64 keys at a time
+          // pass 2: p = 2^(S up log2e - m log2e); hi = p rounded to bf16,
+          // lo = p - hi rounded to bf16; both as bf16 pairs in place over S
 #pragma unroll 1
           for (int c0 = 0; c0 < KT; c0 += 64) {
             if (c0 < nk16) {
@@ -922,17 +962,16 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
 #pragma unroll
                   for (int u = 0; u < 8; ++u) {
                     // two keys per packed op: t = S up log2e - m log2e, p = 2^t,
-                    // hi = p cut to 10 mantissa bits, lo = p - hi
+                    // hi = bf16(p), lo = bf16(p - hi)
                     const uint64_t t = tc::fma2(tc::f2pack(__uint_as_float(sr[c16 + 2 * u]),
                                                            __uint_as_float(sr[c16 + 2 * u + 1])), up2v, c2v);
                     const float p0 = tc::ex2(tc::f2lo(t)), p1 = tc::ex2(tc::f2hi(t));
-                    const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffffe000u);
-                    const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffffe000u);
                     const uint64_t pp = tc::f2pack(p0, p1);
-                    const uint64_t l = tc::sub2(pp, tc::f2pack(h0, h1));
+                    const uint32_t hb = tc::cvt_bf162(p0, p1);
+                    const uint64_t l = tc::sub2(pp, tc::bf162_to_f2(hb));
                     rs2 = tc::add2(rs2, pp);
-                    hi[u] = tc::cvt_half2(h0, h1);
-                    lo[u] = tc::cvt_half2(tc::f2lo(l), tc::f2hi(l));
+                    hi[u] = hb;
+                    lo[u] = tc::cvt_bf162(tc::f2lo(l), tc::f2hi(l));
                   }
                   // keys c0+c16 .. +15: P hi at the 8 columns from c0+c16, lo at the 8 after
                   tc::tmem_st8(t_s + c0 + c16, hi);

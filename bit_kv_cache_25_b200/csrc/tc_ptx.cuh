@@ -54,9 +54,9 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int k, int ro
 
 // Instruction descriptor: kind::f16 with f16 A and B, f32 accumulator,
 // A K-major, B K-major (b_mn_major = false) or MN-major, M x N.
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major = false) {
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major = false, bool bf16 = false) {
   return (1u << 4)                                   // D format: F32
-         | (0u << 7) | (0u << 10)                    // A, B format: F16
+         | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10)  // A, B format: F16 (0) or BF16 (1), the same for both
          | ((b_mn_major ? 1u : 0u) << 16)            // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
@@ -212,6 +212,17 @@ __device__ __forceinline__ uint32_t cvt_half2(float lo, float hi) {
   uint32_t d;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
+}
+
+// {lo, hi} fp32 -> bf16x2 (lo in the low half), round to nearest even
+__device__ __forceinline__ uint32_t cvt_bf162(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+// the two bf16 halves of a bf16x2 word as an fp32 pair (exact)
+__device__ __forceinline__ uint64_t bf162_to_f2(uint32_t h) {
+  return f2pack(__uint_as_float(h << 16), __uint_as_float(h & 0xffff0000u));
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {

@@ -82,6 +82,35 @@ def test_layout_fits_one_cta(BITS, D, NQT):
     assert not bad, (BITS, D, NQT, bad, c["SMEM_ALLOC"])
 
 
+def warp_roles(NQT):
+    """Role of each warp: softmax 0 .. 4 NQT - 1, then the unpack warps, the
+    producer and the MMA warp."""
+    UW = 8 if NQT == 1 else 6
+    SOFT = 4 * NQT
+    PROD, MMA = SOFT + UW, SOFT + UW + 1
+    nwarps = MMA + 1
+    roles = {}
+    for w in range(nwarps):
+        if w < SOFT:
+            roles[w] = ("softmax", w // 4, w % 4)
+        elif w in (MMA, PROD):
+            roles[w] = ("mma",) if w == MMA else ("producer",)
+        else:
+            roles[w] = ("unpack", w - SOFT)
+    return roles, nwarps, MMA, PROD, UW
+
+
+@pytest.mark.parametrize("NQT", [1, 2])
+def test_warp_roles(NQT):
+    roles, nwarps, MMA, PROD, UW = warp_roles(NQT)
+    assert nwarps * 32 <= 512 and MMA < nwarps and PROD < nwarps
+    # every unpack index 0 .. UW-1 exactly once; softmax warps cover each
+    # query tile's four tensor-memory lane quarters
+    assert sorted(r[1] for r in roles.values() if r[0] == "unpack") == list(range(UW))
+    assert sorted((r[1], r[2]) for r in roles.values() if r[0] == "softmax") == [
+        (qt, q) for qt in range(NQT) for q in range(4)]
+
+
 # ------------------------------------------------------------------ tiles and unpack
 def sw128_offset(row, k, rows):
     slab, kin = k >> 6, k & 63

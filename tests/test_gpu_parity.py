@@ -253,6 +253,38 @@ def test_few_queries_over_many_keys(vq, D):
         _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D, B=2, H=2)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_reference_moves_mid_item(vq, D):
+    """Logits that jump far above an item's running reference maximum: keys
+    aligned with every query, +50 nats in the middle of the second key tile,
+    +110 nats in a later tile. The tensor-core kernel moves the reference
+    inside a tile (rescaling the P chunks already written, O and the row
+    sums) and still matches, for the paired query tiles (block 2, 200
+    queries) and the alternating mode (block 1, 48 queries)."""
+    sched = [64, 48, 200]
+    B, H = 1, 2
+    N = sum(sched)
+    g = torch.Generator(device="cuda").manual_seed(17)
+    u = torch.ones(D, device="cuda")
+    q = (u + 0.5 * torch.randn((B, H, N, D), generator=g, device="cuda")).to(torch.bfloat16)
+    k = torch.randn((B, H, N, D), generator=g, device="cuda")
+    v = torch.randn((B, H, N, D), generator=g, device="cuda") + 1.0
+    kt = 64 if D == 64 else 48
+    first = [kt + 20 + i for i in range(6)]   # second key tile, a chunk after its first
+    later = [kt * 4 + 3 + i for i in range(3)]  # a later tile's first chunk
+    k[:, :, first, :] += (50.0 / D ** 0.5) * u
+    k[:, :, later, :] += (110.0 / D ** 0.5) * u
+    k, v = k.to(torch.bfloat16), v.to(torch.bfloat16)
+    for bits in (4, 8):
+        desc = vq.CacheDesc(B, H, D, bits, sched)
+        cache = vq.LayerCache(desc)
+        p0 = 0
+        for s, n in enumerate(sched):
+            vq.vq_cache_append(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+            p0 += n
+        _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D, B=B, H=H)
+
+
 def _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D, B=1, H=3):
     sigma = 1.0 / np.sqrt(D)
     ok_, sk, zk = vo.cache_append(_host(k), sched, bits)
