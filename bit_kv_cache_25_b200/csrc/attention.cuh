@@ -207,9 +207,12 @@ __host__ __device__ inline CcLayout cc_layout(int n_q, int P, int D) {
 }
 
 // THREADS: 128 for up to 16 queries, 256 above (more warps for the same
-// shared memory once there are enough row and key tasks to share)
+// shared memory once there are enough row and key tasks to share). The
+// 128-thread form is held to 80 registers so that six CTAs fit an SM: its
+// small blocks are latency-bound (VAR-d30 blocks 2-3 took 14 % less time
+// than at three CTAs).
 template <int BITS, int D, int THREADS>
-__global__ void __launch_bounds__(THREADS, 3) attention_cc_kernel(const __grid_constant__ AttnParams p, int P) {
+__global__ void __launch_bounds__(THREADS, THREADS == 128 ? 6 : 3) attention_cc_kernel(const __grid_constant__ AttnParams p, int P) {
   constexpr int kCcThreads = THREADS;
   constexpr int kCcWarps = THREADS / 32;
   constexpr int kCcBatch = THREADS == 128 ? 4 : 2;  // dequantize items per thread with loads in flight together

@@ -7,13 +7,16 @@
 // key tiles of KT tokens (64 at head_dim 64, 48 at 128) that may
 // span several blocks (at most MAXSEG block segments per tile). Each tile is
 // dequantized in shared memory to the cache's own fp32 values
-// x^ = fma(code, scale, zero) of each token's block, times a power of two 2^-e
-// chosen per (batch, head) so that the largest |x^| over blocks 0..s lies in
-// [2^14, 2^15), and split into two 16-bit parts. K, whose rounding moves every
-// logit, takes fp16: hi = x^ with its mantissa cut to 10 bits (exact in fp16),
+// x^ = fma(code, scale, zero) of each token's block and split into two 16-bit
+// parts. K, whose rounding moves every logit, takes fp16, after a power of two
+// 2^-e chosen per (batch, head) so that the largest |K^| over blocks 0..s lies
+// in [2^14, 2^15): hi = x^ with its mantissa cut to 10 bits (exact in fp16),
 // lo = x^ - hi rounded to fp16, so hi + lo = x^ (1 + O(2^-21)). V takes bf16,
-// as P does: hi = x^ rounded to bf16, lo = x^ - hi rounded to bf16, so
-// hi + lo = x^ (1 + O(2^-16)). The bf16 queries are exact in fp16 after a
+// as P does, with no scaling (bf16 has the range of fp32): hi = x^ rounded to
+// bf16, lo = x^ - hi rounded to bf16, so hi + lo = x^ (1 + O(2^-16)). (With
+// fp16 hi/lo for P alone, or for V alone, or bf16 hi/lo for K, the worst
+// output error on the VAR-d30 and Infinity-2B shapes rose to 1e-3 .. 7e-3 of
+// the output RMS in a float64 emulation, against 1e-4 here.) The bf16 queries are exact in fp16 after a
 // power-of-two scale per row. Per tile, for the 128 query rows of a work item,
 // all accumulation in fp32:
 //   S  = q . (K^hi + K^lo)^T                      2 fp16 MMAs per 16-wide k-step
@@ -123,8 +126,8 @@ struct PipeCfg {
   static constexpr int STG_SZ = STG_ROWS + (2 * MAXSEG + 4) * 4;
   static constexpr int HDR0 = STG0 + NSTG * STG_SZ;        // NKV x {2^eK, 2^eV, -, -}
   static constexpr int NRED = 5;                           // exponent reduction slots (> NKV)
-  static constexpr int RED0 = HDR0 + NKV * 16;             // NRED x {K, V} x UNPACK_WARPS floats
-  static constexpr int BARS = RED0 + NRED * 2 * UNPACK_WARPS * 4;
+  static constexpr int RED0 = HDR0 + NKV * 16;             // NRED x UNPACK_WARPS floats (K maxima)
+  static constexpr int BARS = RED0 + NRED * UNPACK_WARPS * 4;
   static constexpr int QBARS = 1 + 3 * NS;                 // per query tile: q_full, s_full, p_full, pv_done
   static constexpr int NBARS = 2 * NSTG + 4 * NKV + NRED + NQT * QBARS;
   static constexpr int TMEM_SLOT = BARS + NBARS * 8;
@@ -502,71 +505,60 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
     // =========================================================== unpack warps
     const int ut = C::unpack_index(warp) * 32 + lane;
     const float cmax = static_cast<float>(C::MASK);
-    // Powers of two of the k-th item of this CTA: max |x^| over blocks 0..s.
+    // Power of two of the k-th item's keys: max |K^| over blocks 0..s.
     // Each warp reduces its share of the scale/zero vectors and posts its
     // maxima in slot k % NRED; the item's first tile reads them all. A warp
     // runs at most NKV - 1 tiles ahead of another, so NRED > NKV slots never
     // alias a slot that is still to be read.
     auto pow2_post = [&](int item, int k) {
       const int bh = item / n_groups;
-      float ak = 0.0f, av = 0.0f;
+      float ak = 0.0f;
       // up to kPow2Batch (block, channel) pairs per thread in flight at once
       constexpr int kPow2Batch = 8;
       for (int base = 0; base < (p.s + 1) * D; base += kPow2Batch * C::UNPACK_THREADS) {
-        float sk[kPow2Batch], zk[kPow2Batch], sv[kPow2Batch], zv[kPow2Batch];
+        float sk[kPow2Batch], zk[kPow2Batch];
 #pragma unroll
         for (int u = 0; u < kPow2Batch; ++u) {
           const int idx = base + u * C::UNPACK_THREADS + ut;
-          sk[u] = zk[u] = sv[u] = zv[u] = 0.0f;
+          sk[u] = zk[u] = 0.0f;
           if (idx < (p.s + 1) * D) {
             const int kb = idx / D;
             const int64_t mo = kb * BHD + static_cast<int64_t>(bh) * D + (idx - kb * D);
             sk[u] = __ldcg(p.scale_k + mo);
             zk[u] = __ldcg(p.zero_k + mo);
-            sv[u] = __ldcg(p.scale_v + mo);
-            zv[u] = __ldcg(p.zero_v + mo);
           }
         }
 #pragma unroll
-        for (int u = 0; u < kPow2Batch; ++u) {
-          ak = fmaxf(ak, fmaxf(fabsf(zk[u]), fabsf(fmaf(cmax, sk[u], zk[u]))));
-          av = fmaxf(av, fmaxf(fabsf(zv[u]), fabsf(fmaf(cmax, sv[u], zv[u]))));
-        }
+        for (int u = 0; u < kPow2Batch; ++u) ak = fmaxf(ak, fmaxf(fabsf(zk[u]), fabsf(fmaf(cmax, sk[u], zk[u]))));
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, o));
-        av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, o));
-      }
+      for (int o = 16; o > 0; o >>= 1) ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, o));
       const int slot = k % C::NRED;
       if (lane == 0) {
-        red[(slot * 2 + 0) * C::UNPACK_WARPS + (ut >> 5)] = ak;
-        red[(slot * 2 + 1) * C::UNPACK_WARPS + (ut >> 5)] = av;
+        red[slot * C::UNPACK_WARPS + (ut >> 5)] = ak;
         mbar_arrive(&red_bar[slot]);
       }
       __syncwarp();
     };
-    auto pow2_take = [&](int k, float& kmul, float& kinv, float& vmul, float& vinv) -> bool {
+    auto pow2_take = [&](int k, float& kmul, float& kinv) -> bool {
       const int slot = k % C::NRED;
       if (!mbar_wait_bounded(&red_bar[slot], (k / C::NRED) & 1)) return false;
-      const float* r = red + slot * 2 * C::UNPACK_WARPS;
-      float ak = 0.0f, av = 0.0f;
+      const float* r = red + slot * C::UNPACK_WARPS;
+      float ak = 0.0f;
 #pragma unroll
-      for (int w = 0; w < C::UNPACK_WARPS; ++w) {
-        ak = fmaxf(ak, r[w]);
-        av = fmaxf(av, r[C::UNPACK_WARPS + w]);
-      }
+      for (int w = 0; w < C::UNPACK_WARPS; ++w) ak = fmaxf(ak, r[w]);
       pipe_pow2(ak, kmul, kinv);
-      pipe_pow2(av, vmul, vinv);
       return true;
     };
 
-    float kmul = 1.0f, kinv = 1.0f, vmul = 1.0f, vinv = 1.0f;
+    // V needs no power of two: bf16 hi/lo keeps the cache's values at any magnitude
+    constexpr float vmul = 1.0f, vinv = 1.0f;
+    float kmul = 1.0f, kinv = 1.0f;
     if (static_cast<int>(blockIdx.x) < n_items) pow2_post(blockIdx.x, 0);
     int g = 0;
     bool ok = true;
     for (int item = blockIdx.x, k = 0; ok && item < n_items; item += gridDim.x, ++k) {
-      if (!(ok = pow2_take(k, kmul, kinv, vmul, vinv))) break;
+      if (!(ok = pow2_take(k, kmul, kinv))) break;
       for (int j = 0; j < T; ++j, ++g) {
         const int st = g % NSTG;
         const int kvs = g % NKV;

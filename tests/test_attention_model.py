@@ -54,7 +54,7 @@ def pipe_cfg(BITS, D, NQT):
     HDR0 = STG0 + NSTG * STG_SZ
     NRED = 5
     RED0 = HDR0 + NKV * 16
-    BARS = RED0 + NRED * 2 * UW * 4
+    BARS = RED0 + NRED * UW * 4
     NBARS = 2 * NSTG + 4 * NKV + NRED + NQT * (1 + 3 * NS)
     TMEM_SLOT = BARS + NBARS * 8
     NKTAB = TMEM_SLOT + 16
