@@ -549,29 +549,50 @@ def run_e2e(args, vq, w, bits, desc, caches, outs, dev, world):
     """Same decode through the public API with host inputs: every step copies each
     layer's K, V, Q from pinned host memory, runs its appends and attentions, and
     copies its outputs back. The host holds one layer of inputs, reused for
-    every layer; the device holds one layer of inputs at a time."""
+    every layer. Three streams overlap the work of neighbouring layers: the
+    inputs of layer l+1 go up and the outputs of layer l-1 come down while
+    layer l computes (two device buffers of each, ordered by events)."""
     L, S = w.layers, w.num_blocks
     k0, v0 = make_kv(w, 0, seed=7, device="cpu")
     q0 = make_q(w, 0, seed=7, device="cpu")
     hk, hv, hq = k0.pin_memory(), v0.pin_memory(), q0.pin_memory()
-    dk, dv, dq = torch.empty_like(hk, device=dev), torch.empty_like(hv, device=dev), torch.empty_like(hq, device=dev)
+    dk = [torch.empty_like(hk, device=dev) for _ in range(2)]
+    dv = [torch.empty_like(hv, device=dev) for _ in range(2)]
+    dq = [torch.empty_like(hq, device=dev) for _ in range(2)]
     B, H, D, N = w.batch, w.heads, w.head_dim, w.tokens
-    dout = torch.empty((B, H, N, D), dtype=torch.float32, device=dev)
+    dout = [torch.empty((B, H, N, D), dtype=torch.float32, device=dev) for _ in range(2)]
     hout = torch.empty((B, H, N, D), dtype=torch.float32).pin_memory()
     sigma = default_softmax_scale(w)
     stream = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
 
     def step():
         for layer in range(L):
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            dq.copy_(hq, non_blocking=True)
+            b = layer % 2
+            up.wait_event(computed[b])           # buffer b's previous layer has been used
+            with torch.cuda.stream(up):
+                dk[b].copy_(hk, non_blocking=True)
+                dv[b].copy_(hv, non_blocking=True)
+                dq[b].copy_(hq, non_blocking=True)
+                in_ready[b].record(up)
+            stream.wait_event(in_ready[b])
+            stream.wait_event(out_done[b])       # dout[b] has been copied out
             for s in range(S):
                 p0, n = w.prefix(s), w.block_tokens[s]
-                vq.vq_cache_append(desc, caches[layer], s, dk[:, :, p0:p0 + n], dv[:, :, p0:p0 + n], stream=stream)
-                vq.vq_attention_block(desc, caches[layer], s, dq[:, :, p0:p0 + n], sigma, dout[:, :, p0:p0 + n],
-                                      stream=stream)
-            hout.copy_(dout, non_blocking=True)
+                vq.vq_cache_append(desc, caches[layer], s, dk[b][:, :, p0:p0 + n], dv[b][:, :, p0:p0 + n],
+                                   stream=stream)
+                vq.vq_attention_block(desc, caches[layer], s, dq[b][:, :, p0:p0 + n], sigma,
+                                      dout[b][:, :, p0:p0 + n], stream=stream)
+            computed[b].record(stream)
+            down.wait_event(computed[b])
+            with torch.cuda.stream(down):
+                hout.copy_(dout[b], non_blocking=True)
+                out_done[b].record(down)
+        # the step ends when its last outputs are on the host
+        stream.wait_event(out_done[(L - 1) % 2])
 
     steps = max(1, min(args.steps, args.e2e_steps))
     for _ in range(1):
@@ -580,6 +601,7 @@ def run_e2e(args, vq, w, bits, desc, caches, outs, dev, world):
     barrier(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    up.wait_event(a)  # no copy of the timed steps starts before the clock does
     for _ in range(steps):
         step()
     b.record(stream)
@@ -588,7 +610,8 @@ def run_e2e(args, vq, w, bits, desc, caches, outs, dev, world):
     h2d = L * sum(t.numel() * t.element_size() for t in (hk, hv, hq))
     d2h = L * hout.numel() * hout.element_size()
     return {"value": world * B * N * L / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
+            "overlap": "inputs of layer l+1 and outputs of layer l-1 copied while layer l computes"}
 
 
 def main():

@@ -326,9 +326,11 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
 
 // ---- ring variant: the slab of each unit is bulk-copied into a shared-memory
 // slot, so min/max and the encode both read it from shared memory and HBM sees
-// every input byte once. Warp 0 (one lane) is the producer; consumer warp w
-// owns NSLOT slots and takes every RW-th unit of its CTA, one unit per warp,
-// no CTA-wide barrier: full/empty mbarriers per slot, waits bounded.
+// every input byte once. Warp 0 (one lane) is the producer; consumer team t (RG
+// warps) owns NSLOT slots and takes every RW-th unit of its CTA. The team's
+// warps split the unit's rows (pass 1) and word rows (pass 2) and merge their
+// min/max partials in shared memory behind a named barrier of the team; no
+// CTA-wide barrier: full/empty mbarriers per slot, waits bounded.
 template <class Vec, int BITS>
 __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel(const __grid_constant__ QuantParams p) {
   constexpr int CPW = 32 / BITS;
@@ -340,6 +342,11 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
   uint64_t* full = reinterpret_cast<uint64_t*>(rsm);        // [RW][NS]
   uint64_t* empty = full + kRingMaxWarps * 4;               // [RW][NS]
   unsigned char* slots = rsm + 2 * kRingMaxWarps * 4 * 8;   // [RW][NS][slot_bytes]
+  const int RG = p.RG;
+  // [RW][2][RG][2][D] min/max partials of the team's warps (double-buffered),
+  // then [RW][2] failed-wait marks (unit index + 1 of a wait that timed out)
+  float* part = reinterpret_cast<float*>(slots + static_cast<size_t>(RW) * NS * p.slot_bytes);
+  volatile int* tfail = reinterpret_cast<volatile int*>(part + static_cast<size_t>(RW) * 2 * RG * 2 * p.D);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
   const int D = p.D, V = p.vecs_per_row;
@@ -347,8 +354,9 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
   if (threadIdx.x == 0) {
     for (int i = 0; i < RW * NS; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], RG);
     }
+    for (int i = 0; i < 2 * RW; ++i) tfail[i] = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -379,17 +387,22 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
     return;
   }
   // ------------------------------------------------------------------ consumers
-  const int cw = warp - 1;
-  if (cw >= RW) return;
+  const int team = (warp - 1) / RG, gw = (warp - 1) - team * RG;
+  if (team >= RW) return;
   const int j = lane % V;          // 16-byte channel vector of this lane
   const int rsub = lane / V;       // row (or word row) offset of this lane
   const int RL = 32 / V;           // rows (word rows) one warp step covers
-  for (int k = cw;; k += RW) {
+  const int r0 = rsub + gw * RL;   // this warp's first row (word row); step RL * RG
+  for (int k = team;; k += RW) {
     const int u = blockIdx.x + k * gridDim.x;
     if (u >= p.units) break;
     const int s = (k / RW) % NS, use = k / (RW * NS);
-    const int b = cw * NS + s;
-    if (!mbar_wait_bounded(&full[b], use & 1)) break;
+    const int b = team * NS + s;
+    const int par = (k / RW) & 1;
+    // a team leaves together: with more than one warp, a failed wait is
+    // published and every warp of the team stops after the team's barrier
+    const bool got = mbar_wait_bounded(&full[b], use & 1);
+    if (RG == 1 && !got) break;
     const unsigned char* slab = slots + static_cast<size_t>(b) * p.slot_bytes + j * 16;
     const QuantTensor& T = p.t[u / BH];
     const int bh = u % BH;
@@ -400,10 +413,10 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
       mn[q] = Vec::kMnInit;
       mx[q] = Vec::kMxInit;
     }
-    for (int r = rsub; r < p.n; r += 8 * RL) {
+    for (int r = got ? r0 : p.n; r < p.n; r += 8 * RL * RG) {
       uint4 v[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = lds128(slab + min(r + q * RL, p.n - 1) * rowb);
+      for (int q = 0; q < 8; ++q) v[q] = lds128(slab + min(r + q * RL * RG, p.n - 1) * rowb);
 #pragma unroll
       for (int q = 0; q < 8; ++q) Vec::minmax_acc(mn, mx, v[q]);  // repeats of row n-1 change nothing
     }
@@ -420,6 +433,28 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
         fmx[c] = fmaxf(fmx[c], __shfl_xor_sync(0xffffffffu, fmx[c], off));
       }
     }
+    if (RG > 1) {
+      // the team's partials meet in shared memory (a buffer is written again
+      // only after the team's next barrier, which every reader has passed)
+      float* pb = part + static_cast<size_t>((team * 2 + par) * RG) * 2 * D;
+      if (!got && lane == 0) tfail[team * 2 + par] = k + 1;
+      if (rsub == 0) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          pb[gw * 2 * D + CH * j + c] = fmn[c];
+          pb[gw * 2 * D + D + CH * j + c] = fmx[c];
+        }
+      }
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(32 * RG) : "memory");
+      if (tfail[team * 2 + par] == k + 1) break;
+      for (int q = 0; q < RG; ++q) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          fmn[c] = fminf(fmn[c], pb[q * 2 * D + CH * j + c]);
+          fmx[c] = fmaxf(fmx[c], pb[q * 2 * D + D + CH * j + c]);
+        }
+      }
+    }
     // scale, zero and encode constants (2^64 prescale of tiny scales, see the
     // streaming kernel)
     float inv[CH], pre[CH], nmp[CH];
@@ -431,7 +466,7 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
         group_params(fmn[c], fmx[c], kLevels, META16, scl[c], zer[c], inv[c], pre[c], nmp[c]);
         tiny |= (pre[c] != 1.0f);
       }
-      if (rsub == 0) {
+      if (rsub == 0 && gw == 0) {
         float* sd = T.scale + static_cast<size_t>(bh) * D + CH * j;
         float* zd = T.zero + static_cast<size_t>(bh) * D + CH * j;
 #pragma unroll
@@ -443,7 +478,7 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
     }
     tiny = __any_sync(0xffffffffu, tiny) || META16;
     // pass 2: word rows of this lane's vector
-    for (int w = rsub; w < p.W; w += RL) {
+    for (int w = r0; w < p.W; w += RL * RG) {
       const int t0 = w * CPW;
       const int nvalid = min(CPW, p.n - t0);
       uint4 v[CPW];
@@ -462,7 +497,8 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
 }
 
 size_t quant_ring_smem_bytes(const QuantParams& p) {
-  return static_cast<size_t>(2 * kRingMaxWarps * 4 * 8) + static_cast<size_t>(p.RW) * p.NSLOT * p.slot_bytes;
+  return static_cast<size_t>(2 * kRingMaxWarps * 4 * 8) + static_cast<size_t>(p.RW) * p.NSLOT * p.slot_bytes +
+         static_cast<size_t>(p.RW) * 2 * p.RG * 2 * p.D * sizeof(float) + static_cast<size_t>(p.RW) * 2 * sizeof(int);
 }
 
 template <class Vec, int BITS>
@@ -476,14 +512,15 @@ cudaError_t launch_ring(const QuantParams& p, cudaStream_t stream) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             2 * kRingMaxWarps * 4 * 8 + kRingSmemBudget);
+                             2 * kRingMaxWarps * 4 * 8 + kRingSmemBudget + kRingMaxWarps * 2 * 2 * 128 * 4 +
+                                 kRingMaxWarps * 2 * 4);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
   const int grid = p.units < sm_count[dev] ? p.units : sm_count[dev];
-  kern<<<grid, 32 * (1 + p.RW), quant_ring_smem_bytes(p), stream>>>(p);
+  kern<<<grid, 32 * (1 + p.RW * p.RG), quant_ring_smem_bytes(p), stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -7,6 +7,7 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -109,7 +110,8 @@ bool plan_quant(vq::QuantParams& p) {
   if (p.TL > 32) p.TL = 32;
   // Ring kernel for slabs from 8 KB up to half the slot budget: every unit is
   // bulk-copied into a shared-memory slot and read from there twice. Two slots
-  // per consumer warp while that leaves at least four warps, else one.
+  // per slot owner while that leaves at least four owners, else one; each
+  // owner is a team of warps that shares its units' rows.
   p.ring = 0;
   const int64_t slab = int64_t(p.n) * p.D * p.esize;
   if (slab >= 8192 && slab <= vq::kRingSmemBudget / 2) {
@@ -125,6 +127,8 @@ bool plan_quant(vq::QuantParams& p) {
       p.RW = static_cast<int>(rwarps);
       p.NSLOT = ns;
       p.slot_bytes = static_cast<int>(slab);
+      // the remaining consumer warps join the slot owners: teams of up to 6
+      p.RG = std::min(vq::kRingMaxWarps / p.RW, 6);
     }
   }
   return true;

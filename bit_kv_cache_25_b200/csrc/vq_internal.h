@@ -32,14 +32,15 @@ struct QuantParams {
   int TL;               // lanes per unit when P == 1 (vecs_per_row * rows per load; 32 / TL units per warp)
   int meta16;           // scale and zero rounded to fp16, codes against that grid
   // ring kernel (ring == 1): each unit's slab is bulk-copied into a shared-memory
-  // slot of slot_bytes; RW consumer warps with NSLOT slots each
+  // slot of slot_bytes; RW consumer teams of RG warps, NSLOT slots per team
   int ring;
   int RW;
+  int RG;
   int NSLOT;
   int slot_bytes;
 };
 
-constexpr int kRingMaxWarps = 12;            // consumer warps per CTA
+constexpr int kRingMaxWarps = 12;            // consumer warps per CTA (teams x warps per team)
 constexpr int kRingSmemBudget = 200 * 1024;  // bytes of slots per CTA
 
 

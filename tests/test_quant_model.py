@@ -88,7 +88,7 @@ def ring_plan(n, D, esize):
     if rw < 4:
         ns, rw = 1, RING_BUDGET // slab
     rw = min(rw, RING_MAX_WARPS)
-    return (rw, ns, slab) if rw >= 2 else None
+    return (rw, ns, slab, min(RING_MAX_WARPS // rw, 6)) if rw >= 2 else None
 
 
 @pytest.mark.parametrize("D,esize", [(64, 2), (128, 2), (64, 4), (128, 4)])
@@ -102,9 +102,31 @@ def test_ring_quant_plan_and_protocol(D, esize):
         pl = ring_plan(n, D, esize)
         if pl is None:
             continue
-        rw, ns, slab = pl
+        rw, ns, slab, rg = pl
         assert 2 <= rw <= RING_MAX_WARPS and ns in (1, 2) and slab % 16 == 0
         assert rw * ns * slab <= RING_BUDGET and rw * ns <= RING_MAX_WARPS * 4
+        # teams: at most 12 consumer warps, named barriers 1 .. rw, and the
+        # shared memory (barriers, slots, [rw][2][rg][2][D] partials) fits the opt-in
+        assert 1 <= rg <= 6 and rw * rg <= RING_MAX_WARPS and rw + 1 <= 16
+        assert 2 * RING_MAX_WARPS * 4 * 8 + rw * ns * slab + rw * 2 * rg * 2 * D * 4 <= 232448
+        # the team's warps split rows (pass 1, 8 loads per lane per step) and
+        # word rows (pass 2): every one is taken exactly once
+        V = D * esize // 16
+        RL = 32 // V
+        for bits in (2, 3, 4, 6, 8):
+            W = -(-n // (32 // bits))
+            rows, wrows = [], []
+            for gw in range(rg):
+                for rsub in range(RL):
+                    r = rsub + gw * RL
+                    while r < n:
+                        rows += [r + q * RL * rg for q in range(8) if r + q * RL * rg < n]
+                        r += 8 * RL * rg
+                    w = rsub + gw * RL
+                    while w < W:
+                        wrows.append(w)
+                        w += RL * rg
+            assert sorted(rows) == list(range(n)) and sorted(wrows) == list(range(W))
         for units, grid in ((7680, 148), (256, 148), (5, 3)):
             grid = min(grid, units)
             seen = {}
