@@ -142,8 +142,9 @@ vq_status vq_cache_append(const vq_cache_desc* desc, const vq_layer_cache* cache
  *        gives the accuracy the tests check; VQ_BF16 rounds the float32 result);
  *   softmax_scale: the logit multiplier, usually 1/sqrt(head_dim).
  * Arithmetic: float32 accumulation of logits, softmax and output over the
- * cache's dequantized values (on the tensor cores as exact-sum fp16 hi/lo
- * operand pairs); the result is within 2e-3 x output RMS of float64 attention
+ * cache's dequantized values (on the tensor cores as hi/lo 16-bit operand
+ * pairs: fp16 for K, bf16 for V and the probabilities); the result is within
+ * 2e-3 x output RMS of float64 attention
  * over the same dequantized cache. See the kernel sources for the operand
  * precision of each kernel. */
 vq_status vq_attention_block(const vq_cache_desc* desc, const vq_layer_cache* cache,
