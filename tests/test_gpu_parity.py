@@ -237,6 +237,39 @@ def test_ragged_blocks_all_bit_widths(vq, D):
 
 
 @pytest.mark.parametrize("D", [64, 128])
+def test_ragged_blocks_fp32_inputs(vq, D):
+    """fp32 K/V through both quantize kernels: slabs of 8-100 KB take the
+    shared-memory ring (teams of 1 to 6 warps at these sizes), the rest the
+    register-streaming kernel; codes, scales and zeros bit-exact, attention
+    within the bar."""
+    sched = [1, 33, 81, 300, 1100]
+    k, v, q = _ragged_kv(sched, D, dtype=torch.float32, seed=9)
+    B, H = 1, 3
+    for bits in (3, 4):
+        desc = vq.CacheDesc(B, H, D, bits, sched)
+        cache = vq.LayerCache(desc)
+        kh, vh = _host(k), _host(v)
+        p0 = 0
+        for s, n in enumerate(sched):
+            vq.vq_cache_append(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+            torch.cuda.synchronize()
+            W = desc.word_rows(s)
+            offs = cache.block_word_offset
+            for x, packed, scale, zero in ((kh, cache.packed_k, cache.scale_k, cache.zero_k),
+                                           (vh, cache.packed_v, cache.scale_v, cache.zero_v)):
+                words, s_ref, z_ref = vo.quantize_pack_block(x[:, :, p0:p0 + n], bits)
+                np.testing.assert_array_equal(
+                    packed[offs[s]:offs[s + 1]].cpu().numpy().view(np.uint32).reshape(B, H, W, D), words)
+                np.testing.assert_array_equal(scale[s * B * H * D:(s + 1) * B * H * D].cpu().numpy().view(np.uint32),
+                                              s_ref.reshape(-1).view(np.uint32))
+                np.testing.assert_array_equal(zero[s * B * H * D:(s + 1) * B * H * D].cpu().numpy().view(np.uint32),
+                                              z_ref.reshape(-1).view(np.uint32))
+            p0 += n
+        assert vq.vq_poll_device_error() == 0
+        _check_ragged_attention(vq, desc, cache, sched, q, k, v, bits, D)
+
+
+@pytest.mark.parametrize("D", [64, 128])
 def test_few_queries_over_many_keys(vq, D):
     """Blocks of 5 and 3 queries after 500 cached tokens: too many keys for the
     CUDA-core kernel's shared memory, so they run on the tensor-core kernel
