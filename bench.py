@@ -15,7 +15,7 @@ the `quant_pack` / `attention` / `roofline` keys.
   python bench.py --impl reference ...   # the CPU oracle, bounded sample
 
 Each workload also times the same decode through vq_append_attention_block
-(`fused`: append and attention in one launch where possible).
+(`fused`: append and attention in one launch where that is faster).
 """
 from __future__ import annotations
 
@@ -483,7 +483,8 @@ def measure(args, vq, w, bits, world, seed, dev):
         "fused": {"ms_per_step": fused_ms, "value": weak_scaling_value(tokens_step, world, fused_ms),
                   "unit": "tokens/s", "launches_per_step": L * sum(1 if n <= 256 else 2 for n in w.block_tokens),
                   "note": "the same decode through vq_append_attention_block (append and attention in one launch "
-                          "for blocks of at most 256 queries), replayed alone after the timed steps"},
+                          "where that is faster: CUDA-core blocks with at most 4 (batch, head) per SM; two "
+                          "launches otherwise), replayed alone after the timed steps"},
         "clocks": clk.summary(),
         "gpu_launches": 2 * L * S * args.steps,
         "by_block": by_block,

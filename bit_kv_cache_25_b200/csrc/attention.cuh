@@ -442,11 +442,26 @@ namespace {
 // softmax warpgroups taking the items in turn.
 }  // namespace
 
-// Whether block s's append can run inside its attention launch: every kernel's
-// CTA then quantizes the (batch, head) slabs it attends for, which holds when
-// each (batch, head) is one work item (always for the CUDA-core kernels; up to
-// two 128-row query tiles, i.e. 256 queries, on the tensor cores).
-bool attention_fusable(const AttnParams& p) { return p.n_q <= kSmallMaxQueries || cc_fits(p) || p.n_q <= 256; }
+// Whether block s's append runs inside its attention launch: the CUDA-core
+// kernels' CTAs (one per (batch, head)) then quantize their own (batch, head)
+// slabs before attending. That saves a launch, but the CTA's quantize is a
+// serial prologue, so it only pays while the grid is about one wave: measured
+// with CUDA graphs, Infinity-2B blocks 0-2 (128 (batch, head)) took 6-12 us
+// fused against 9-17 us as two launches, VAR-d30 blocks 0-4 (3840) 32-152
+// against 16-128. On the tensor-core kernel the prologue never overlapped the
+// attention (Infinity blocks 5-6 8-10 % slower, VAR-d30 blocks 5-9 4-15 %), so
+// those blocks always run the two launches.
+bool attention_fusable(const AttnParams& p) {
+  if (!(p.n_q <= kSmallMaxQueries || cc_fits(p))) return false;
+  static int sms[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (sms[dev] == 0 && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    sms[dev] = 0;
+    return false;
+  }
+  return static_cast<int64_t>(p.B) * p.H <= 4 * static_cast<int64_t>(sms[dev]);
+}
 
 namespace {
 

@@ -302,17 +302,6 @@ __global__ void __launch_bounds__(PipeCfg<BITS, D, NQT>::THREADS, 1)
   // addresses. Anything else is recorded and every role skips its work.
   const bool tmem_at_zero = (tmem == 0u);
   if (!tmem_at_zero && tid == 0) atomicOr(&g_device_error, kDevErrBadShape);
-  if (p.fused) {
-    // fused append: every warp quantizes units (item, tensor) of this CTA's
-    // items (one item per (batch, head)) into the cache; the fence makes the
-    // stores visible to the bulk copies that read them back
-    const int mine = static_cast<int>(blockIdx.x) < n_items ? (n_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-    for (int u = warp; u < 2 * mine; u += C::THREADS / 32)
-      fused_quantize_unit<BITS>(p, (blockIdx.x + (u >> 1) * gridDim.x) / n_groups, u & 1, lane);
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-    __syncthreads();
-  }
-
   if (!tmem_at_zero) {
     // (recorded above: straight to the teardown)
   } else if (warp == C::PROD_WARP) {

@@ -158,10 +158,12 @@ vq_status vq_attention_block(const vq_cache_desc* desc, const vq_layer_cache* ca
  * calls in sequence. Block-by-block decoding appends each block just before
  * its queries attend ("VAR-Q ...", Abstract, paragraph 1; block boundaries
  * from the generation loop, paragraph 3), so both steps share one launch
- * wherever the attention has one work item per (batch, head): the attention
- * CTAs first quantize the slabs of their own (batch, head), then attend, and
- * the fresh K/V is read from HBM once. That holds for blocks of at most 256
- * queries; larger blocks run the two launches in order on `stream`. Arguments
+ * where that is faster: blocks that run on the CUDA-core kernels (at most 32
+ * queries) when batch * heads is at most four per SM; there each attention
+ * CTA first quantizes the slabs of its own (batch, head), then attends, and
+ * the fresh K/V is read from HBM once. Every other block runs the two
+ * launches in order on `stream` (the quantize prologue serializes in front of
+ * the attention and costs more than the extra launch). Arguments
  * are those of vq_cache_append and vq_attention_block, validated the same way
  * before anything is launched. */
 vq_status vq_append_attention_block(const vq_cache_desc* desc, const vq_layer_cache* cache, int32_t block,

@@ -492,8 +492,8 @@ def _fused_decode(vq, desc, cache, sched, k, v, q, sigma, B, H, D, out_dtype=tor
 def test_fused_append_attention(vq, D):
     """vq_append_attention_block block by block: the cache is bit-exact with the
     oracle's append and every block's attention within the bar of the oracle's
-    attention over it. Blocks of 3, 20, 100 and 200 queries run fused (warp per
-    query, CUDA-core and both tensor-core modes); 300 runs append, then attend."""
+    attention over it. Blocks of 3 and 20 queries run fused (warp per query and
+    CUDA-core kernels, 4 (batch, head)); 100, 200 and 300 run append, then attend."""
     sched = [3, 20, 100, 200, 300]
     B, H = 2, 2
     k, v, q = _ragged_kv(sched, D, H=H, B=B, seed=17)
