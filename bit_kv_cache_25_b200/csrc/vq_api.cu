@@ -20,6 +20,7 @@
 #include "attention.cuh"
 #include "dequant.cuh"
 #include "paper.cuh"
+#include "selftest.cuh"
 
 namespace {
 
@@ -420,6 +421,14 @@ vq_status vq_paper_unpack(const vq_cache_desc* desc, const uint32_t* k_words, co
   uint32_t* const w[2] = {const_cast<uint32_t*>(k_words), const_cast<uint32_t*>(v_words)};
   uint32_t* const m[2] = {const_cast<uint32_t*>(k_meta), const_cast<uint32_t*>(v_meta)};
   return paper_convert(desc, cache, false, w, m, stream);
+}
+
+vq_status vq_check_wait_timeout(uint32_t max_iters, void* stream) {
+  if (max_iters < 1 || max_iters > (1u << 24))
+    return fail(VQ_ERR_INVALID_ARGUMENT, "max_iters must be in [1, 2^24]");
+  cudaError_t e = vq::launch_wait_timeout(max_iters, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wait-timeout self-test launch");
+  return ok();
 }
 
 vq_status vq_poll_device_error(uint32_t* code) {

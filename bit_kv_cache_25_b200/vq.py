@@ -56,6 +56,7 @@ def _load():
         "vq_paper_pack": [P(vq_cache_desc), P(vq_layer_cache), VP, VP, VP, VP, VP],
         "vq_paper_unpack": [P(vq_cache_desc), VP, VP, VP, VP, P(vq_layer_cache), VP],
         "vq_poll_device_error": [P(ctypes.c_uint32)],
+        "vq_check_wait_timeout": [ctypes.c_uint32, VP],
         "vq_status_string": [I32],
         "vq_last_error": [],
         "vq_version": [],
@@ -71,7 +72,7 @@ _lib = _load()
 
 EXPORTED = ("vq_cache_layout", "vq_quantize_pack_block", "vq_cache_append", "vq_attention_block",
             "vq_append_attention_block", "vq_dequantize", "vq_paper_layout", "vq_paper_pack", "vq_paper_unpack",
-            "vq_poll_device_error", "vq_status_string", "vq_last_error", "vq_version")
+            "vq_poll_device_error", "vq_check_wait_timeout", "vq_status_string", "vq_last_error", "vq_version")
 
 
 def _check(status: int):
@@ -332,6 +333,12 @@ def vq_poll_device_error() -> int:
     code = ctypes.c_uint32()
     _check(_lib.vq_poll_device_error(ctypes.byref(code)))
     return code.value
+
+
+def vq_check_wait_timeout(max_iters: int, stream=None):
+    """Launch the self-test whose bounded wait times out (see vq.h); the device
+    error word then holds flag 1 once the stream has run it."""
+    _check(_lib.vq_check_wait_timeout(max_iters, _stream(stream)))
 
 
 def vq_version() -> int:

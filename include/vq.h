@@ -212,6 +212,16 @@ vq_status vq_dequantize(const vq_cache_desc* desc, int32_t block, const uint32_t
  * (a blocking copy). */
 vq_status vq_poll_device_error(uint32_t* code);
 
+/* Self-test of the device error path (no counterpart on the pages; it checks
+ * the library's own failure handling). Launches one thread on `stream` that
+ * waits on a shared-memory barrier nothing arrives at, giving up after
+ * max_iters polls (1 .. 2^24; each poll after the 64th sleeps ~100 ns), so
+ * the wait times out: the kernel ORs flag 1 into the device error word and
+ * returns normally, and the context stays usable. Read the flag with
+ * vq_poll_device_error after the stream completes. Allocates nothing.
+ * VQ_ERR_INVALID_ARGUMENT for max_iters outside the range. */
+vq_status vq_check_wait_timeout(uint32_t max_iters, void* stream);
+
 /* Static text for a status code. */
 const char* vq_status_string(vq_status status);
 

@@ -117,3 +117,11 @@ def test_meta_fp16_flag_validated():
     d.c.meta_fp16 = 2
     with pytest.raises(vq.VqError):
         vq.vq_cache_layout(d)
+
+
+def test_wait_timeout_selftest_validates_before_launch():
+    """The error-path self-test rejects an iteration limit outside 1 .. 2^24
+    before any CUDA call."""
+    lib = vq.raw_lib()
+    for bad in (0, (1 << 24) + 1):
+        assert lib.vq_check_wait_timeout(bad, None) == vq.VQ_ERR_INVALID_ARGUMENT

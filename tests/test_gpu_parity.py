@@ -611,3 +611,25 @@ def test_fp16_metadata_and_paper_format(vq, D):
                      (back.zero_k, cache.zero_k), (back.scale_v, cache.scale_v), (back.zero_v, cache.zero_v)):
             assert torch.equal(a, b)
     assert vq.vq_poll_device_error() == 0
+
+
+# ---------------------------------------------------------------- failure path
+def test_bounded_wait_timeout_sets_flag_and_context_survives(vq):
+    """A wait that nothing completes gives up after its iteration limit: the
+    kernel records flag 1 in the device error word and returns, the poll reads
+    and clears it, and the context keeps working (a small append + attention
+    afterwards is still bit-exact / within the bar)."""
+    assert vq.vq_poll_device_error() == 0
+    vq.vq_check_wait_timeout(2000)
+    torch.cuda.synchronize()
+    assert vq.vq_poll_device_error() == 1
+    assert vq.vq_poll_device_error() == 0
+    sched = [1, 9, 40]
+    k, v, q = _ragged_kv(sched, 64, seed=3)
+    desc = vq.CacheDesc(1, 3, 64, 4, sched)
+    cache = vq.LayerCache(desc)
+    p0 = 0
+    for s, n in enumerate(sched):
+        vq.vq_cache_append(desc, cache, s, k[:, :, p0:p0 + n], v[:, :, p0:p0 + n])
+        p0 += n
+    _check_ragged_attention(vq, desc, cache, sched, q, k, v, 4, 64)
