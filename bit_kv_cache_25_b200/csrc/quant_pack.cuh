@@ -326,8 +326,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1) quant_pack_kernel(const __gr
 
 // ---- ring variant: the slab of each unit is bulk-copied into a shared-memory
 // slot, so min/max and the encode both read it from shared memory and HBM sees
-// every input byte once. Warp 0 (one lane) is the producer; consumer team t (RG
-// warps) owns NSLOT slots and takes every RW-th unit of its CTA. The team's
+// every input byte once. Consumer team t (RG warps) owns NSLOT slots and takes
+// every RW-th unit of its CTA; a one-warp team copies its own units, larger
+// teams are served by a producer warp (one lane). The team's
 // warps split the unit's rows (pass 1) and word rows (pass 2) and merge their
 // min/max partials in shared memory behind a named barrier of the team; no
 // CTA-wide barrier: full/empty mbarriers per slot, waits bounded.
@@ -360,35 +361,50 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
     fence_barrier_init();
   }
   __syncthreads();
-  if (warp == 0) {
+  // Copy of the CTA's k-th unit into slot (k % RW, (k / RW) % NS).
+  auto issue = [&](int k) {
+    const int u = blockIdx.x + k * gridDim.x;
+    const int b = (k % RW) * NS + (k / RW) % NS;
+    const QuantTensor& T = p.t[u / BH];
+    const int bh = u % BH;
+    const unsigned char* src =
+        static_cast<const unsigned char*>(T.x) + ((bh / p.H) * T.sb + (bh % p.H) * T.sh) * p.esize;
+    unsigned char* dst = slots + static_cast<size_t>(b) * p.slot_bytes;
+    const uint32_t bytes = static_cast<uint32_t>(p.n * rowb);
+    mbar_arrive_expect_tx(&full[b], bytes);
+    if (T.st * p.esize == rowb) {
+      bulk_copy_g2s(dst, src, bytes, &full[b]);  // contiguous rows: one copy
+    } else {
+      for (int r = 0; r < p.n; ++r)
+        bulk_copy_g2s(dst + r * rowb, src + r * T.st * p.esize, static_cast<uint32_t>(rowb), &full[b]);
+    }
+  };
+  // Teams of one warp copy their own units (each slot refilled as soon as its
+  // warp has left it; measured faster on the 8 KB slabs of many one-warp
+  // teams); larger teams are served by warp 0, which refills the slots in
+  // unit order.
+  const bool self_copy = (RG == 1);
+  if (!self_copy && warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       for (int k = 0;; ++k) {
         const int u = blockIdx.x + k * gridDim.x;
         if (u >= p.units) break;
-        const int w = k % RW, s = (k / RW) % NS, use = k / (RW * NS);
-        const int b = w * NS + s;
+        const int b = (k % RW) * NS + (k / RW) % NS, use = k / (RW * NS);
         if (use > 0 && !mbar_wait_bounded(&empty[b], (use - 1) & 1)) break;
-        const QuantTensor& T = p.t[u / BH];
-        const int bh = u % BH;
-        const unsigned char* src =
-            static_cast<const unsigned char*>(T.x) + ((bh / p.H) * T.sb + (bh % p.H) * T.sh) * p.esize;
-        unsigned char* dst = slots + static_cast<size_t>(b) * p.slot_bytes;
-        const uint32_t bytes = static_cast<uint32_t>(p.n * rowb);
-        mbar_arrive_expect_tx(&full[b], bytes);
-        if (T.st * p.esize == rowb) {
-          bulk_copy_g2s(dst, src, bytes, &full[b]);  // contiguous rows: one copy
-        } else {
-          for (int r = 0; r < p.n; ++r)
-            bulk_copy_g2s(dst + r * rowb, src + r * T.st * p.esize, static_cast<uint32_t>(rowb), &full[b]);
-        }
+        issue(k);
       }
     }
     return;
   }
   // ------------------------------------------------------------------ consumers
-  const int team = (warp - 1) / RG, gw = (warp - 1) - team * RG;
+  const int cw = self_copy ? warp : warp - 1;
+  const int team = cw / RG, gw = cw - team * RG;
   if (team >= RW) return;
+  if (self_copy && lane == 0) {
+    for (int q = 0; q < NS; ++q)
+      if (blockIdx.x + (team + q * RW) * gridDim.x < p.units) issue(team + q * RW);
+  }
   const int j = lane % V;          // 16-byte channel vector of this lane
   const int rsub = lane / V;       // row (or word row) offset of this lane
   const int RL = 32 / V;           // rows (word rows) one warp step covers
@@ -492,7 +508,15 @@ __global__ void __launch_bounds__(32 * (1 + kRingMaxWarps), 1) quant_ring_kernel
         reinterpret_cast<uint4*>(dst)[q] = make_uint4(wd[4 * q], wd[4 * q + 1], wd[4 * q + 2], wd[4 * q + 3]);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[b]);
+    if (self_copy) {
+      // this warp has left slot b: its unit NS ahead goes in
+      if (lane == 0 && blockIdx.x + (k + NS * RW) * gridDim.x < p.units) {
+        fence_proxy_async_smem();
+        issue(k + NS * RW);
+      }
+    } else if (lane == 0) {
+      mbar_arrive(&empty[b]);
+    }
   }
 }
 
@@ -520,7 +544,8 @@ cudaError_t launch_ring(const QuantParams& p, cudaStream_t stream) {
     configured[dev] = true;
   }
   const int grid = p.units < sm_count[dev] ? p.units : sm_count[dev];
-  kern<<<grid, 32 * (1 + p.RW * p.RG), quant_ring_smem_bytes(p), stream>>>(p);
+  // one warp per consumer, plus the producer warp for teams of several warps
+  kern<<<grid, 32 * (p.RW * p.RG + (p.RG == 1 ? 0 : 1)), quant_ring_smem_bytes(p), stream>>>(p);
   return cudaGetLastError();
 }
 

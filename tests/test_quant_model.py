@@ -94,9 +94,11 @@ def ring_plan(n, D, esize):
 @pytest.mark.parametrize("D,esize", [(64, 2), (128, 2), (64, 4), (128, 4)])
 def test_ring_quant_plan_and_protocol(D, esize):
     """Ring kernel: the slots fit the shared-memory budget (and the barrier
-    arrays), every unit goes to exactly one consumer warp, and each slot is
-    filled and drained in the same order by its producer and its warp, so the
-    parity of every full/empty wait is the use count of that slot."""
+    arrays), every unit goes to exactly one team, and each slot is filled and
+    drained in the same order (by the producer warp, or, for one-warp teams,
+    by the team itself: its first NS units at once, then unit i + NS into the
+    slot unit i leaves), so the parity of every full/empty wait is the use
+    count of that slot."""
     ran = 0
     for n in (16, 36, 64, 100, 144, 169, 256, 300, 400, 576, 800):
         pl = ring_plan(n, D, esize)
@@ -147,6 +149,14 @@ def test_ring_quant_plan_and_protocol(D, esize):
                         drains.append((w * ns + (kk // rw) % ns, kk // (rw * ns), u))
                         kk += rw
                     assert drains == [f for f in fills if f[0] // ns == w]
+                    if rg == 1:
+                        # self-copying team: units 0 .. ns-1 first, then unit i + ns
+                        # into the slot unit i has just left
+                        own = [d[:2] for d in drains[:ns]]
+                        for i in range(len(drains) - ns):
+                            assert drains[i + ns][:2] == (drains[i][0], drains[i][1] + 1)
+                            own.append(drains[i + ns][:2])
+                        assert own == [d[:2] for d in drains]
             assert len(seen) == units
             ran += 1
     assert ran > 0
