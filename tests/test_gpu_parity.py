@@ -369,6 +369,46 @@ def test_strided_inputs_and_outputs(vq):
     assert torch.equal(o_strided.permute(0, 2, 1, 3), o_contig)
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("n", [64, 169])
+def test_ring_slot_refills_with_strided_rows(vq, n):
+    """Slabs that take the shared-memory ring (8 KB with one-warp teams that copy
+    their own units; 21.6 KB with three-warp teams served by the producer warp),
+    with enough (batch, head) that every CTA refills its slots many times. Rows
+    [B][N][H][D] viewed as [B][H][N][D] are copied row by row; the cache must
+    hold the same bytes as from contiguous slabs, and those match the oracle
+    on a sample of units."""
+    B, H, D, bits = 128, 30, 64, 3
+    sched = [n]
+    g = torch.Generator(device="cuda").manual_seed(17 + n)
+    kt = (torch.randn((B, n, H, D), generator=g, device="cuda") * 2).to(torch.bfloat16)
+    vt = torch.randn((B, n, H, D), generator=g, device="cuda").to(torch.bfloat16)
+    k, v = kt.permute(0, 2, 1, 3), vt.permute(0, 2, 1, 3)
+    desc = vq.CacheDesc(B, H, D, bits, sched)
+    c1, c2 = vq.LayerCache(desc), vq.LayerCache(desc)
+    vq.vq_cache_append(desc, c1, 0, k, v)
+    vq.vq_cache_append(desc, c2, 0, k.contiguous(), v.contiguous())
+    torch.cuda.synchronize()
+    assert vq.vq_poll_device_error() == 0
+    for a, b in ((c1.packed_k, c2.packed_k), (c1.packed_v, c2.packed_v), (c1.scale_k, c2.scale_k),
+                 (c1.zero_k, c2.zero_k), (c1.scale_v, c2.scale_v), (c1.zero_v, c2.zero_v)):
+        assert torch.equal(a, b)
+    # a sample of (b, h) units against the oracle: scale, zero and packed words of K and V
+    W = -(-n // (32 // bits))
+    pk = c2.packed_k.view(B, H, W, D).cpu().numpy().view(np.uint32)
+    pv = c2.packed_v.view(B, H, W, D).cpu().numpy().view(np.uint32)
+    sk, zk = c2.scale_k.view(B, H, D).cpu().numpy(), c2.zero_k.view(B, H, D).cpu().numpy()
+    sv, zv = c2.scale_v.view(B, H, D).cpu().numpy(), c2.zero_v.view(B, H, D).cpu().numpy()
+    rng = np.random.default_rng(n)
+    for bb, hh in zip(rng.integers(0, B, 6), rng.integers(0, H, 6)):
+        for x, pw, sc, ze in ((k, pk, sk, zk), (v, pv, sv, zv)):
+            xs = _host(x[bb:bb + 1, hh:hh + 1])  # [1][1][n][D] float32
+            words, s_o, z_o = vo.quantize_pack_block(xs, bits)
+            np.testing.assert_array_equal(sc[bb, hh].view(np.uint32), s_o[0, 0].view(np.uint32))
+            np.testing.assert_array_equal(ze[bb, hh].view(np.uint32), z_o[0, 0].view(np.uint32))
+            np.testing.assert_array_equal(pw[bb, hh], words[0, 0])
+
+
 def test_degenerate_groups(vq):
     """Constant channels (scale 0), a zero min stored as +0, a single-token block,
     and groups whose range is in the float32 subnormal range (scale below
