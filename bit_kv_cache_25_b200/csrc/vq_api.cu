@@ -111,14 +111,17 @@ bool plan_quant(vq::QuantParams& p) {
   if (p.TL > 32) p.TL = 32;
   // Ring kernel for slabs from 8 KB up to half the slot budget: every unit is
   // bulk-copied into a shared-memory slot and read from there twice. Two slots
-  // per slot owner while that leaves at least four owners, else one; each
-  // owner is a team of warps that shares its units' rows.
+  // per slot owner while that still leaves kRingMaxWarps owners, else one slot
+  // each and as many owners as the budget holds (CUDA-graph A/B on VAR-d30:
+  // 12.8 KB slabs 35.6 -> 33.5 us, 21.6 KB 57.8 -> 54.6 us per append against
+  // two slots each; 8 KB slabs best with two); each owner is a team of warps
+  // that shares its units' rows.
   p.ring = 0;
   const int64_t slab = int64_t(p.n) * p.D * p.esize;
   if (slab >= 8192 && slab <= vq::kRingSmemBudget / 2) {
     int ns = 2;
     int64_t rwarps = vq::kRingSmemBudget / (2 * slab);
-    if (rwarps < 4) {
+    if (rwarps < vq::kRingMaxWarps) {
       ns = 1;
       rwarps = vq::kRingSmemBudget / slab;
     }

@@ -85,7 +85,7 @@ def ring_plan(n, D, esize):
     if not (8192 <= slab <= RING_BUDGET // 2):
         return None
     ns, rw = 2, RING_BUDGET // (2 * slab)
-    if rw < 4:
+    if rw < RING_MAX_WARPS:
         ns, rw = 1, RING_BUDGET // slab
     rw = min(rw, RING_MAX_WARPS)
     return (rw, ns, slab, min(RING_MAX_WARPS // rw, 6)) if rw >= 2 else None
