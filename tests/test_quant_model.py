@@ -160,3 +160,21 @@ def test_ring_quant_plan_and_protocol(D, esize):
             assert len(seen) == units
             ran += 1
     assert ran > 0
+
+
+def test_ring_plans_of_the_workload_slabs():
+    """The ring plans the measurements chose, for the bf16 slabs of the VAR-d30
+    (head_dim 64) and Infinity-2B (head_dim 128) blocks that take the ring:
+    (teams, slots per team, slab bytes, warps per team). Two slots per team
+    only for 8 KB slabs (twelve one-warp teams still fit); one slot and as
+    many teams as the budget holds above that; the smallest slabs fall to the
+    streaming kernel."""
+    want = {
+        (36, 64): None, (64, 64): (12, 2, 8192, 1), (100, 64): (12, 1, 12800, 1),
+        (169, 64): (9, 1, 21632, 1), (256, 64): (6, 1, 32768, 2),
+        (16, 128): None, (36, 128): (12, 1, 9216, 1), (64, 128): (12, 1, 16384, 1),
+        (144, 128): (5, 1, 36864, 2), (256, 128): (3, 1, 65536, 4), (400, 128): (2, 1, 102400, 6),
+        (576, 128): None,
+    }
+    for (n, D), plan in want.items():
+        assert ring_plan(n, D, 2) == plan, (n, D)
